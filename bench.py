@@ -1,0 +1,468 @@
+#!/usr/bin/env python3
+"""Benchmark of the TBQ4 attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tbq4|reference]
+
+One step is one decode step at 262,144 cached tokens (24 query heads over 4
+KV heads, head_dim 128, K with 4 outlier channels per head x10): the new
+token's K and V rows are quantise-appended into the TBQ4 caches, then decode
+attention runs over all 262,144 keys (split kernel + log-sum-exp combine
+with the inverse rotation).  `value` is effective HBM throughput: the
+algorithmic bytes of one step (the TBQ4 K and V blocks read, plus q, the
+output and the appended rows) divided by the device time of the step.
+
+The same line also carries the chunked-prefill figure (512 new tokens over
+131,072 cached tokens, causal, after appending the chunk) in TFLOP/s, the
+roofline of the dominant kernel, an end-to-end figure through the public
+API with host buffers, and the fp64 CPU oracle timed on the host cores.
+
+Timing: W untimed warm-up steps, then exactly K steps, each bracketed by
+CUDA events on the launching stream; the L2 cache is flushed (a 512 MiB
+memset) before every timed step, outside the events.  With N > 1 (torchrun)
+every rank runs an independent replica and the time is the max over ranks.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "TBQ4 flash-decode effective HBM GB/s & % peak at 262K ctx; prefill TFLOP/s"
+D = 128
+BLOCK = 66
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="tbq4", choices=["tbq4", "reference"])
+    ap.add_argument("--prefill-steps", type=int, default=5)
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- helpers
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "long_context_attention_tbq4_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        h.update(name.encode())
+        h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(kernel)
+    if not rec or rec.get("source_sha256") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class Clocks:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    Q = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.p is not None:
+            self.p.terminate()
+            self.p.wait()
+
+    def summary(self):
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10 or (self.uuid and self.uuid not in parts[1]):
+                continue
+            try:
+                rows.append((float(parts[2]), float(parts[3]), parts[6:10], parts[5]))
+            except ValueError:
+                continue
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2]) if v == "Active"})
+        return {"sm_mhz": float(np.median([r[0] for r in rows])),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- workloads
+def decode_workload():
+    from long_context_attention_tbq4_b200 import workloads as W
+    case = W.decode_262k()
+    N = int(case.seq_lens[0])
+    bytes_kv = 2 * case.Hkv * N * BLOCK
+    bytes_q = case.B * case.Hq * D * 4
+    bytes_out = case.B * case.Hq * D * 2
+    bytes_append = 2 * case.Hkv * (D * 4 + BLOCK)          # new token: read fp32, write block
+    return case, N, bytes_kv + bytes_q + bytes_out + bytes_append, bytes_kv + bytes_q
+
+
+def prefill_flops(n_cached, n_new, Hq):
+    keys = sum(n_cached + i + 1 for i in range(n_new))
+    return 4.0 * D * Hq * keys
+
+
+# --------------------------------------------------------------- GPU legs
+def timing_events(torch, n):
+    """n quadruples of timing events (step start/end, kernel start/end).
+    torch creates an event lazily at its first record, so each is recorded
+    once here to exist before its handle is given to the library."""
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(n)]
+    for quad in ev:
+        for e in quad:
+            e.record()
+    torch.cuda.synchronize()
+    return ev
+
+
+def bench_decode(T, torch, case, N, step_bytes, kernel_bytes, steps, warmup, flush):
+    dev = torch.device("cuda")
+    cap = N
+    K, V = case.k[0], case.v[0]
+    kc = T.empty_cache(1, case.Hkv, cap)
+    vc = T.empty_cache(1, case.Hkv, cap)
+    zero = torch.zeros(1, dtype=torch.int32, device=dev)
+    for cache, x in ((kc, K), (vc, V)):
+        src = torch.from_numpy(np.ascontiguousarray(x[:N - 1])[None]).to(dev)
+        T.tbq4_quantize_append(src, zero, cache, case.sign_seed)
+        del src
+    k_new = torch.from_numpy(np.ascontiguousarray(K[N - 1:N])[None]).to(dev)
+    v_new = torch.from_numpy(np.ascontiguousarray(V[N - 1:N])[None]).to(dev)
+    pos = torch.tensor([N - 1], dtype=torch.int32, device=dev)
+    q = torch.from_numpy(case.q).to(dev)
+    lens = torch.tensor([N], dtype=torch.int32, device=dev)
+    ws = torch.empty(T.tbq4_decode_workspace_bytes(1, case.Hq, case.Hkv, N), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty((1, case.Hq, D), dtype=torch.float16, device=dev)
+
+    def step(qq=q, kn=k_new, vn=v_new, o=out):
+        T.tbq4_quantize_append(kn, pos, kc, case.sign_seed)
+        T.tbq4_quantize_append(vn, pos, vc, case.sign_seed)
+        T.tbq4_attn_decode(qq, kc, vc, lens, N, case.softmax_scale, case.sign_seed,
+                           workspace=ws, out=o)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    assert T.tbq4_get_device_status() == 0
+
+    ev = timing_events(torch, steps)
+    barrier()
+    torch.cuda.synchronize()
+    for e0, e1, k0, k1 in ev:
+        flush.zero_()
+        T.tbq4_set_timing_events(k0, k1)
+        e0.record()
+        step()
+        e1.record()
+    T.tbq4_set_timing_events(None, None)
+    torch.cuda.synchronize()
+    barrier()
+    step_ms = [e0.elapsed_time(e1) for e0, e1, _, _ in ev]
+    kern_ms = [k0.elapsed_time(k1) for _, _, k0, k1 in ev]
+
+    # end to end: the step's inputs from pinned host memory, the output back
+    q_h = torch.from_numpy(case.q).pin_memory()
+    kn_h = torch.from_numpy(np.ascontiguousarray(K[N - 1:N])[None]).pin_memory()
+    vn_h = torch.from_numpy(np.ascontiguousarray(V[N - 1:N])[None]).pin_memory()
+    out_h = torch.empty((1, case.Hq, D), dtype=torch.float16).pin_memory()
+    q_d, kn_d, vn_d = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
+
+    def e2e_step():
+        q_d.copy_(q_h, non_blocking=True)
+        kn_d.copy_(kn_h, non_blocking=True)
+        vn_d.copy_(vn_h, non_blocking=True)
+        step(q_d, kn_d, vn_d, out)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+    barrier()
+    for e0, e1 in e2e_ev:
+        flush.zero_()
+        e0.record()
+        e2e_step()
+        e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = [e0.elapsed_time(e1) for e0, e1 in e2e_ev]
+    assert T.tbq4_get_device_status() == 0
+    h2d = q_h.numel() * 4 + kn_h.numel() * 4 + vn_h.numel() * 4
+    d2h = out_h.numel() * 2
+    return {"step_ms": step_ms, "kern_ms": kern_ms, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
+            "launches_per_step": 4, "out": out.float().cpu().numpy()}
+
+
+def bench_prefill(T, torch, steps, warmup, flush):
+    from long_context_attention_tbq4_b200 import workloads as W
+    c = W.prefill_131k()
+    dev = torch.device("cuda")
+    cap = W.round_capacity(c.n_cached + c.n_new)
+    kc = T.empty_cache(1, c.Hkv, cap)
+    vc = T.empty_cache(1, c.Hkv, cap)
+    zero = torch.zeros(1, dtype=torch.int32, device=dev)
+    for cache, x in ((kc, c.k), (vc, c.v)):
+        src = torch.from_numpy(np.ascontiguousarray(x[:c.n_cached])[None]).to(dev)
+        T.tbq4_quantize_append(src, zero, cache, c.sign_seed)
+        del src
+    kch = torch.from_numpy(np.ascontiguousarray(c.k[c.n_cached:])[None]).to(dev)
+    vch = torch.from_numpy(np.ascontiguousarray(c.v[c.n_cached:])[None]).to(dev)
+    pos = torch.tensor([c.n_cached], dtype=torch.int32, device=dev)
+    q = torch.from_numpy(c.q_bf16.view(np.int16)).to(dev).view(torch.bfloat16)
+    ws = torch.empty(T.tbq4_prefill_workspace_bytes(c.n_new, c.Hq, c.Hkv, c.n_cached),
+                     dtype=torch.uint8, device=dev)
+    out = torch.empty((c.n_new, c.Hq, D), dtype=torch.bfloat16, device=dev)
+
+    def step():
+        T.tbq4_quantize_append(kch, pos, kc, c.sign_seed)
+        T.tbq4_quantize_append(vch, pos, vc, c.sign_seed)
+        T.tbq4_attn_prefill_chunk(q, c.n_cached, kc[0], vc[0], c.softmax_scale, c.sign_seed,
+                                  workspace=ws, out=out)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = timing_events(torch, steps)
+    barrier()
+    for e0, e1, k0, k1 in ev:
+        flush.zero_()
+        T.tbq4_set_timing_events(k0, k1)
+        e0.record()
+        step()
+        e1.record()
+    T.tbq4_set_timing_events(None, None)
+    torch.cuda.synchronize()
+    barrier()
+    assert T.tbq4_get_device_status() == 0
+    flops = prefill_flops(c.n_cached, c.n_new, c.Hq)
+    step_ms = float(np.mean([a.elapsed_time(b) for a, b, _, _ in ev]))
+    kern_ms = float(np.mean([a.elapsed_time(b) for _, _, a, b in ev]))
+    return {"workload": c.name, "n_cached": c.n_cached, "n_new": c.n_new, "Hq": c.Hq,
+            "Hkv": c.Hkv, "flops_per_step": flops, "ms_per_step": step_ms,
+            "tflops": flops / (step_ms * 1e-3) / 1e12, "attn_kernel_ms": kern_ms,
+            "attn_kernel_tflops": flops / (kern_ms * 1e-3) / 1e12, "steps": steps}
+
+
+# ------------------------------------------------------------ CPU baseline
+def oracle_decode_sample(case, N, rows):
+    """Oracle caches (built once, untimed) and a timed call on `rows`."""
+    import oracle
+    cap = N
+    ko = np.zeros((1, case.Hkv, cap, BLOCK), np.uint8)
+    vo = np.zeros((1, case.Hkv, cap, BLOCK), np.uint8)
+    oracle.quantize_append(case.k[0][:N - 1][None], np.zeros(1, np.int32), cap,
+                           case.sign_seed, ko)
+    oracle.quantize_append(case.v[0][:N - 1][None], np.zeros(1, np.int32), cap,
+                           case.sign_seed, vo)
+    lens = np.array([N], np.int32)
+    pos = np.array([N - 1], np.int32)
+    knew = case.k[0][N - 1:N][None]
+    vnew = case.v[0][N - 1:N][None]
+
+    def step():
+        oracle.quantize_append(knew, pos, cap, case.sign_seed, ko)
+        oracle.quantize_append(vnew, pos, cap, case.sign_seed, vo)
+        return oracle.attn_decode(case.q, ko, vo, lens, case.softmax_scale, case.sign_seed,
+                                  rows=rows)
+    return step
+
+
+def cpu_baseline(case, N, step_bytes, sample_rows=24, reps=5):
+    import oracle
+    rows = np.arange(sample_rows, dtype=np.int32)
+    step = oracle_decode_sample(case, N, rows)
+    step()
+    t = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        step()
+        t.append(time.perf_counter() - t0)
+    t_full = float(np.median(t)) * (case.B * case.Hq / sample_rows)
+    return {"value": step_bytes / t_full / 1e9, "unit": "GB/s", "cores": oracle.get_threads(),
+            "kind": "oracle",
+            "sample": (f"decode_262k, {sample_rows} of {case.B * case.Hq} query-head rows "
+                       f"over all {N} keys plus the new token's append, median of {reps} "
+                       f"steps; time scaled by {case.B * case.Hq}/{sample_rows}"),
+            "sample_seconds": float(np.median(t))}
+
+
+# ------------------------------------------------------------- distributed
+_dist = None
+
+
+def barrier():
+    if _dist is not None:
+        _dist.barrier()
+
+
+def max_over_ranks(torch, x):
+    if _dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    _dist.all_reduce(t, op=_dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# -------------------------------------------------------------------- main
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    case, N, step_bytes, _ = decode_workload()
+    sample_rows = case.B * case.Hq
+    step = oracle_decode_sample(case, N, np.arange(sample_rows, dtype=np.int32))
+    for _ in range(args.warmup):
+        step()
+    t = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        step()
+        t.append(time.perf_counter() - t0)
+    import oracle
+    scale = case.B * case.Hq / sample_rows
+    ms = float(np.mean(t)) * scale * 1e3
+    value = step_bytes / (ms * 1e-3) / 1e9
+    sample = (f"decode_262k, {sample_rows} of {case.B * case.Hq} query-head rows over all "
+              f"{N} keys per step plus the new token's append; time scaled by {scale:g}")
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": "decode_262k", "batch": 1, "ctx": N, "Hq": case.Hq,
+                       "Hkv": case.Hkv, "head_dim": D},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.get_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    global _dist
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        _dist = dist
+    import long_context_attention_tbq4_b200 as T
+
+    peaks = measured_peaks()
+    case, N, step_bytes, kernel_bytes = decode_workload()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    uuid = str(getattr(torch.cuda.get_device_properties(local), "uuid", "") or "")
+    with Clocks(uuid) as clk:
+        dec = bench_decode(T, torch, case, N, step_bytes, kernel_bytes, args.steps,
+                           args.warmup, flush)
+        pre = None if args.no_prefill else bench_prefill(T, torch, args.prefill_steps,
+                                                         min(args.warmup, 3), flush)
+    clocks = clk.summary()
+
+    total_ms = max_over_ranks(torch, float(np.sum(dec["step_ms"])))
+    ms_per_step = total_ms / args.steps
+    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+    e2e_ms = max_over_ranks(torch, float(np.mean(dec["e2e_ms"])))
+    kern_ms = float(np.mean(dec["kern_ms"]))
+    achieved = kernel_bytes / (kern_ms * 1e-3) / 1e9
+    traffic = recorded_traffic("decode_split_kernel")
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "decode_262k", "batch": 1, "ctx": N, "Hq": case.Hq,
+                   "Hkv": case.Hkv, "head_dim": D, "kv_format": "tbq4 (66 B / 128 values)",
+                   "l2": "flushed (512 MiB memset) before every timed step",
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "step_bytes": step_bytes,
+        "pct_hbm_peak": value / world / peaks["hbm_gbs"],
+        "roofline": {"kernel": "decode_split_kernel", "bound": "hbm", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "algorithmic_bytes": kernel_bytes, "kernel_ms": kern_ms,
+                     "peak_source": peaks["source"]},
+        "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": dec["h2d"],
+                "d2h_bytes_per_step": dec["d2h"]},
+        "gpu_launches": dec["launches_per_step"] * args.steps,
+        "clocks": clocks,
+    }
+    if pre is not None:
+        pk = peaks["bf16_tflops"]
+        pre["roofline"] = {"bound": "tensor", "achieved": pre["attn_kernel_tflops"],
+                           "peak": pk, "unit": "TFLOP/s",
+                           "frac": pre["attn_kernel_tflops"] / pk,
+                           "peak_source": peaks["source"] + " (bf16 burst)"}
+        line["prefill"] = pre
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(case, N, step_bytes)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if _dist is not None:
+        _dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,183 @@
+/*
+ * tbq4.h -- C ABI of libtbq4: attention over a long-context KV cache stored
+ * in the TBQ4 block format, on NVIDIA B200 (sm_100a).
+ *
+ * The format.  TBQ4 stores 128 values in 66 bytes: a 2-byte scale followed
+ * by 64 bytes of 4-bit indices, 4.125 bits per value, in a Hadamard-rotated
+ * domain; attention reads the raw blocks and dequantises them in its inner
+ * loop, with no separate dequantisation pass and no fp16 copy of the cache
+ * (trefon.com, "Kontekst 262K na jednej RTX 4090: co dodalem do
+ * llama.cpp-turboq", section "Od czego zaczalem").  K and V have separate
+ * caches, as the page's "-ctk tbq4_0 -ctv tbq4_0" flags do (section
+ * "Konfiguracja").
+ *
+ * The codebook (the page does not give one; this library fixes it):
+ *   x_rot = R x with R = H * D / sqrt(128), H the 128x128 Sylvester Hadamard
+ *     matrix (H[i][j] = (-1)^popcount(i&j)), D = diag(s), s_i = +-1 from
+ *     SplitMix64(sign_seed): s_i = 1 - 2*bit(i%64) of output number i/64.
+ *     Computed as: sign flip, 7 butterfly stages of stride 1,2,...,64 (lower
+ *     = a+b, upper = a-b, each rounded to binary32), one binary32 multiply
+ *     by fl32(1/sqrt(128)) = 0x3DB504F3.
+ *   scale S = fp16(max_i |x_rot_i|), round to nearest even, saturating at
+ *     65504; stored little endian in bytes 0-1.
+ *   index i = clamp(rne(fl32(fl32(x_rot/S) * 7.5) + 7.5), 0, 15) (index 8
+ *     when S == 0); byte 2+j = index[2j] | index[2j+1] << 4.
+ *   dequantised value = S * (2*index - 15) / 15 (rotated domain).
+ *
+ * Cache layout: [B][Hkv][capacity][66] bytes per cache (K or V); the
+ * blocks of one (sequence, KV head) are contiguous.  capacity must be a
+ * multiple of 8 so that every 8-token group (528 bytes) starts on a 16-byte
+ * boundary, and cache base pointers must be 16-byte aligned.
+ *
+ * Conventions for every call:
+ *   - Pointers marked "device" are CUDA device (or managed) memory on the
+ *     current device; the caller owns all memory.  The library allocates
+ *     nothing and frees nothing; scratch memory is a caller-provided
+ *     workspace whose size the *_workspace_bytes queries return.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every
+ *     compute call is asynchronous on that stream and does not synchronise.
+ *   - Arguments are checked on the host before anything is launched; on a
+ *     non-OK status nothing was launched.  Values that live in device memory
+ *     (positions, lengths) are checked by the kernels, which skip the
+ *     offending work and record an error code that tbq4_get_device_status
+ *     returns.
+ *   - Inputs q, K and V are in the original (unrotated) domain; outputs are
+ *     unrotated.  The rotation is internal and keyed by `sign_seed`, which
+ *     must be the same for the append calls and the attention calls of one
+ *     cache.
+ */
+#ifndef TBQ4_H_
+#define TBQ4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TBQ4_API __attribute__((visibility("default")))
+#else
+#define TBQ4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TBQ4_OK = 0,
+    TBQ4_ERR_NULL = 1,            /* a required pointer is NULL            */
+    TBQ4_ERR_ALIGN = 2,           /* a pointer is not 16-byte aligned      */
+    TBQ4_ERR_SHAPE = 3,           /* bad sizes: Hq % Hkv, G > 8, n <= 0 .. */
+    TBQ4_ERR_CAPACITY = 4,        /* capacity not a multiple of 8, or a
+                                     position/length outside [0, capacity] */
+    TBQ4_ERR_WORKSPACE = 5,       /* workspace smaller than required       */
+    TBQ4_ERR_LAUNCH = 6,          /* a CUDA launch or query failed         */
+    TBQ4_ERR_DEVICE_TIMEOUT = 7   /* a bounded wait inside a kernel gave up */
+} tbq4_status;
+
+/* Bytes of one block (66) and of one cache (B*Hkv*capacity*66). */
+TBQ4_API size_t tbq4_block_bytes(void);
+TBQ4_API size_t tbq4_cache_bytes(int batch, int n_kv_heads, int64_t capacity);
+
+/* Host: the +-1 diagonal for `seed`, written to out[128] (host memory). */
+TBQ4_API void tbq4_signs(uint64_t seed, int8_t out[128]);
+
+/*
+ * Quantise-append: rotate, scale, index and pack new K or V rows into a
+ * cache (the TBQ4 encoding above; page section "Od czego zaczalem").
+ *   src        device, fp32 [B][n_new][Hkv][128], 16-byte aligned
+ *   start_pos  device, int32 [B]: row t of sequence b goes to position
+ *              start_pos[b] + t
+ *   cache      device, uint8 [B][Hkv][capacity][66], 16-byte aligned
+ * Bytes written are bit-exact with the codebook above.  Rows whose position
+ * falls outside [0, capacity) are skipped and flag TBQ4_ERR_CAPACITY in the
+ * device status.
+ */
+TBQ4_API tbq4_status tbq4_quantize_append(const float *src, int B, int n_new, int Hkv,
+                                 const int32_t *start_pos, int64_t capacity,
+                                 uint64_t sign_seed, uint8_t *cache,
+                                 void *stream);
+
+/*
+ * Decode attention (one query token per sequence) over TBQ4 caches, split
+ * over the context and merged by log-sum-exp; grouped-query heads share
+ * one KV stream (q head h reads KV head h / (Hq/Hkv)).
+ *   q          device, fp32 [B][Hq][128], 16-byte aligned
+ *   k_cache,
+ *   v_cache    device, uint8 [B][Hkv][capacity][66], 16-byte aligned
+ *   seq_lens   device, int32 [B]: keys attended per sequence (positions
+ *              0 .. seq_lens[b]-1; the current token is already appended).
+ *              A length of 0 gives a zero output row.
+ *   max_len    host upper bound of seq_lens, sizes the launch; lengths above
+ *              it (or above capacity) are clamped and flag
+ *              TBQ4_ERR_CAPACITY in the device status.
+ *   softmax_scale  multiplies q.k before the softmax (1/sqrt(128) typical).
+ *   workspace  device scratch of at least tbq4_decode_workspace_bytes(...)
+ *              bytes, 256-byte aligned; its contents need no initialisation.
+ *   out        device, fp16 [B][Hq][128] (round to nearest even).
+ * Constraints: Hq % Hkv == 0, Hq/Hkv <= 8, B >= 1.
+ */
+TBQ4_API size_t tbq4_decode_workspace_bytes(int B, int Hq, int Hkv, int32_t max_len);
+TBQ4_API tbq4_status tbq4_attn_decode(const float *q, const uint8_t *k_cache,
+                             const uint8_t *v_cache, const int32_t *seq_lens,
+                             int32_t max_len, int B, int Hq, int Hkv,
+                             int64_t capacity, float softmax_scale,
+                             uint64_t sign_seed, void *workspace,
+                             size_t ws_bytes, uint16_t *out, void *stream);
+
+/* As tbq4_attn_decode, with the context split into pieces of
+ * `split_tokens` keys (a multiple of 32; 0 = automatic).  The result does
+ * not depend on the split beyond fp32 rounding.  Workspace requirement:
+ * tbq4_decode_workspace_bytes_split(). */
+TBQ4_API size_t tbq4_decode_workspace_bytes_split(int B, int Hq, int Hkv,
+                                         int32_t max_len, int32_t split_tokens);
+TBQ4_API tbq4_status tbq4_attn_decode_split(const float *q, const uint8_t *k_cache,
+                                   const uint8_t *v_cache,
+                                   const int32_t *seq_lens, int32_t max_len,
+                                   int B, int Hq, int Hkv, int64_t capacity,
+                                   float softmax_scale, uint64_t sign_seed,
+                                   int32_t split_tokens, void *workspace,
+                                   size_t ws_bytes, uint16_t *out,
+                                   void *stream);
+
+/*
+ * Chunked prefill attention for one sequence: n_new query tokens at
+ * absolute positions n_cached .. n_cached+n_new-1, each attending causally
+ * to keys 0 .. its own position, over TBQ4 caches that already hold the
+ * chunk's K/V (call tbq4_quantize_append on the chunk first).
+ *   q          device, bf16 bits [n_new][Hq][128], 16-byte aligned
+ *   k_cache,
+ *   v_cache    device, uint8 [Hkv][capacity][66] (one sequence), 16-byte
+ *              aligned; n_cached + n_new <= capacity
+ *   workspace  device scratch of tbq4_prefill_workspace_bytes(...) bytes
+ *   out        device, bf16 bits [n_new][Hq][128] (round to nearest even)
+ */
+TBQ4_API size_t tbq4_prefill_workspace_bytes(int n_new, int Hq, int Hkv,
+                                    int64_t n_cached);
+TBQ4_API tbq4_status tbq4_attn_prefill_chunk(const uint16_t *q, int n_new,
+                                    int64_t n_cached, const uint8_t *k_cache,
+                                    const uint8_t *v_cache, int Hq, int Hkv,
+                                    int64_t capacity, float softmax_scale,
+                                    uint64_t sign_seed, void *workspace,
+                                    size_t ws_bytes, uint16_t *out,
+                                    void *stream);
+
+/* Profiling hook: while set, every attention call records `before` on its
+ * stream just before its main (split) kernel and `after` just after it, so
+ * a caller can time that kernel alone with cudaEventElapsedTime.  Both are
+ * cudaEvent_t created by the caller; pass NULLs to stop recording.  Not
+ * thread-safe: meant for benchmarks. */
+TBQ4_API void tbq4_set_timing_events(void *before, void *after);
+
+/* Synchronises `stream`, returns the first error code a kernel of this
+ * library recorded on the current device since the last call (TBQ4_OK if
+ * none) and clears it. */
+TBQ4_API tbq4_status tbq4_get_device_status(void *stream);
+
+/* Static description of a status code. */
+TBQ4_API const char *tbq4_status_string(tbq4_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TBQ4_H_ */

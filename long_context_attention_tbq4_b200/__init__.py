@@ -1,0 +1,157 @@
+"""TBQ4 long-context attention on NVIDIA B200 (sm_100a).
+
+A thin binding over libtbq4.so (include/tbq4.h): every function here only
+checks and marshals torch tensors (device memory, current stream) and calls
+the C ABI of the same name; all arithmetic runs in the library's CUDA
+kernels.  There is no CPU path.
+
+TBQ4 stores 128 values in 66 bytes (2-byte scale + 64 bytes of 4-bit
+indices) in a Hadamard-rotated domain, and attention dequantises the raw
+blocks inside its inner loop (trefon.com, "Kontekst 262K na jednej RTX 4090:
+co dodalem do llama.cpp-turboq", section "Od czego zaczalem").
+"""
+import ctypes as C
+
+import numpy as np
+import torch
+
+from ._lib import LIB_PATH, STATUS_NAMES, Tbq4Error, check, lib
+
+D = 128
+BLOCK_BYTES = 66
+
+__all__ = [
+    "D", "BLOCK_BYTES", "LIB_PATH", "Tbq4Error", "tbq4_block_bytes",
+    "tbq4_cache_bytes", "tbq4_signs", "tbq4_quantize_append",
+    "tbq4_decode_workspace_bytes", "tbq4_attn_decode",
+    "tbq4_prefill_workspace_bytes", "tbq4_attn_prefill_chunk",
+    "tbq4_set_timing_events", "tbq4_get_device_status", "empty_cache",
+]
+
+
+def _ptr(t):
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _need(t, dtype, name, ndim=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+
+
+def tbq4_block_bytes() -> int:
+    return int(lib.tbq4_block_bytes())
+
+
+def tbq4_cache_bytes(batch: int, n_kv_heads: int, capacity: int) -> int:
+    return int(lib.tbq4_cache_bytes(batch, n_kv_heads, capacity))
+
+
+def tbq4_signs(seed: int) -> np.ndarray:
+    out = np.zeros(D, np.int8)
+    lib.tbq4_signs(C.c_uint64(seed), out.ctypes.data_as(C.c_void_p))
+    return out
+
+
+def empty_cache(batch, n_kv_heads, capacity, device="cuda"):
+    """An uninitialised [B][Hkv][capacity][66] uint8 cache (capacity % 8 == 0)."""
+    return torch.empty((batch, n_kv_heads, capacity, BLOCK_BYTES), dtype=torch.uint8,
+                       device=device)
+
+
+def tbq4_quantize_append(src, start_pos, cache, sign_seed=0, stream=None):
+    """src fp32 [B][n_new][Hkv][128]; start_pos int32 [B]; cache uint8
+    [B][Hkv][capacity][66] (written in place)."""
+    _need(src, torch.float32, "src", 4)
+    _need(start_pos, torch.int32, "start_pos", 1)
+    _need(cache, torch.uint8, "cache", 4)
+    B, n_new, Hkv, d = src.shape
+    if d != D or tuple(cache.shape[:2]) != (B, Hkv) or cache.shape[3] != BLOCK_BYTES:
+        raise ValueError("shape mismatch between src and cache")
+    check(lib.tbq4_quantize_append(_ptr(src), B, n_new, Hkv, _ptr(start_pos),
+                                   cache.shape[2], C.c_uint64(sign_seed), _ptr(cache),
+                                   _stream(stream)), "tbq4_quantize_append")
+    return cache
+
+
+def tbq4_decode_workspace_bytes(B, Hq, Hkv, max_len, split_tokens=0) -> int:
+    return int(lib.tbq4_decode_workspace_bytes_split(B, Hq, Hkv, max_len, split_tokens))
+
+
+def tbq4_attn_decode(q, k_cache, v_cache, seq_lens, max_len, softmax_scale,
+                     sign_seed=0, workspace=None, out=None, split_tokens=0,
+                     stream=None):
+    """q fp32 [B][Hq][128]; caches uint8 [B][Hkv][capacity][66]; seq_lens
+    int32 [B] (device); returns fp16 [B][Hq][128]."""
+    _need(q, torch.float32, "q", 3)
+    _need(k_cache, torch.uint8, "k_cache", 4)
+    _need(v_cache, torch.uint8, "v_cache", 4)
+    _need(seq_lens, torch.int32, "seq_lens", 1)
+    B, Hq, d = q.shape
+    _, Hkv, cap, nb = k_cache.shape
+    if d != D or nb != BLOCK_BYTES or v_cache.shape != k_cache.shape or k_cache.shape[0] != B:
+        raise ValueError("shape mismatch between q and caches")
+    need = tbq4_decode_workspace_bytes(B, Hq, Hkv, max_len, split_tokens)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float16, device=q.device)
+    _need(out, torch.float16, "out", 3)
+    check(lib.tbq4_attn_decode_split(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), int(max_len), B, Hq, Hkv,
+        cap, float(softmax_scale), C.c_uint64(sign_seed), int(split_tokens),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out),
+        _stream(stream)), "tbq4_attn_decode")
+    return out
+
+
+def tbq4_prefill_workspace_bytes(n_new, Hq, Hkv, n_cached) -> int:
+    return int(lib.tbq4_prefill_workspace_bytes(n_new, Hq, Hkv, n_cached))
+
+
+def tbq4_attn_prefill_chunk(q, n_cached, k_cache, v_cache, softmax_scale, sign_seed=0,
+                            workspace=None, out=None, stream=None):
+    """q bf16 [n_new][Hq][128]; caches uint8 [Hkv][capacity][66] of one
+    sequence holding the chunk at n_cached ..; returns bf16 [n_new][Hq][128]."""
+    _need(q, torch.bfloat16, "q", 3)
+    _need(k_cache, torch.uint8, "k_cache", 3)
+    _need(v_cache, torch.uint8, "v_cache", 3)
+    n_new, Hq, d = q.shape
+    Hkv, cap, nb = k_cache.shape
+    if d != D or nb != BLOCK_BYTES or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch between q and caches")
+    need = tbq4_prefill_workspace_bytes(n_new, Hq, Hkv, n_cached)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((n_new, Hq, D), dtype=torch.bfloat16, device=q.device)
+    _need(out, torch.bfloat16, "out", 3)
+    check(lib.tbq4_attn_prefill_chunk(
+        _ptr(q), n_new, int(n_cached), _ptr(k_cache), _ptr(v_cache), Hq, Hkv, cap,
+        float(softmax_scale), C.c_uint64(sign_seed), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)),
+        "tbq4_attn_prefill_chunk")
+    return out
+
+
+def tbq4_set_timing_events(before=None, after=None):
+    """Record torch.cuda.Event `before`/`after` around the main attention
+    kernel of every following attention call (None, None to stop)."""
+    lib.tbq4_set_timing_events(C.c_void_p(before.cuda_event if before is not None else 0),
+                               C.c_void_p(after.cuda_event if after is not None else 0))
+
+
+def tbq4_get_device_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device error code."""
+    return int(lib.tbq4_get_device_status(_stream(stream)))

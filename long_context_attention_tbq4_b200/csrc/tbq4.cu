@@ -1,0 +1,270 @@
+// tbq4.cu -- libtbq4: the C ABI declared in include/tbq4.h and its launchers.
+//
+// One translation unit: the kernels live in the headers included below.
+// Host code checks every argument before launching anything and never
+// allocates, frees or synchronises (except tbq4_get_device_status).
+#include "tbq4.h"
+
+#include "common.cuh"
+#include "quantize.cuh"
+#include "decode.cuh"
+
+#include <cmath>
+
+namespace {
+
+using namespace tbq4;
+
+constexpr int kNumSMs = 148;          // B200
+constexpr size_t kWsAlign = 256;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// SplitMix64 (Steele, Lea & Flood 2014): the two words whose bits are the
+// +-1 diagonal (bit set -> -1).
+void sign_words(uint64_t seed, uint64_t *lo, uint64_t *hi) {
+    uint64_t st = seed, w[2];
+    for (int k = 0; k < 2; ++k) {
+        st += 0x9E3779B97F4A7C15ULL;
+        uint64_t z = st;
+        z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+        z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+        w[k] = z ^ (z >> 31);
+    }
+    *lo = w[0];
+    *hi = w[1];
+}
+
+// Keys per split: about four CTAs per SM over the whole launch, a multiple
+// of 32, at least 256.
+int32_t auto_split_tokens(int nseq, int Hkv, int32_t max_len) {
+    const int64_t target = (int64_t)kNumSMs * 4;
+    int64_t per = ceil_div((int64_t)max_len * nseq * Hkv, target);
+    per = ceil_div(per, 32) * 32;
+    if (per < 256) per = 256;
+    return (int32_t)per;
+}
+
+struct WsLayout {
+    size_t part_o, part_ml, total;
+    int n_splits;
+};
+
+WsLayout attn_ws_layout(int nseq, int Hq, int32_t max_len, int32_t split_tokens) {
+    WsLayout w;
+    w.n_splits = max_len > 0 ? (int)ceil_div(max_len, split_tokens) : 1;
+    const size_t rows = (size_t)nseq * Hq * w.n_splits;
+    w.part_o = 0;
+    w.part_ml = align_up(rows * kD * sizeof(float), kWsAlign);
+    w.total = align_up(w.part_ml + rows * sizeof(float2), kWsAlign);
+    return w;
+}
+
+cudaEvent_t g_ev_before = nullptr, g_ev_after = nullptr;
+
+tbq4_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? TBQ4_OK : TBQ4_ERR_LAUNCH;
+}
+
+tbq4_status run_attention(AttnParams p, void *workspace, size_t ws_bytes,
+                          cudaStream_t st) {
+    if (p.split_tokens <= 0 || p.split_tokens % 32 != 0) return TBQ4_ERR_SHAPE;
+    const WsLayout w = attn_ws_layout(p.nseq, p.Hq, p.max_len, p.split_tokens);
+    if (ws_bytes < w.total) return TBQ4_ERR_WORKSPACE;
+    if (w.n_splits > 65535 * 16) return TBQ4_ERR_SHAPE;
+    p.n_splits = w.n_splits;
+    p.part_o = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.part_o);
+    p.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) + w.part_ml);
+    dim3 g1(p.n_splits, p.Hkv, p.nseq);
+    if (g_ev_before) cudaEventRecord(g_ev_before, st);
+    decode_split_kernel<<<g1, kSplitWarps * 32, 0, st>>>(p);
+    if (g_ev_after) cudaEventRecord(g_ev_after, st);
+    dim3 g2(p.Hq, p.nseq);
+    decode_combine_kernel<<<g2, kD, 0, st>>>(p);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t tbq4_block_bytes(void) { return kBlockBytes; }
+
+size_t tbq4_cache_bytes(int batch, int n_kv_heads, int64_t capacity) {
+    if (batch <= 0 || n_kv_heads <= 0 || capacity <= 0) return 0;
+    return (size_t)batch * n_kv_heads * (size_t)capacity * kBlockBytes;
+}
+
+void tbq4_signs(uint64_t seed, int8_t out[128]) {
+    uint64_t lo, hi;
+    sign_words(seed, &lo, &hi);
+    for (int i = 0; i < kD; ++i) {
+        const uint64_t w = i < 64 ? lo : hi;
+        out[i] = ((w >> (i & 63)) & 1u) ? -1 : 1;
+    }
+}
+
+tbq4_status tbq4_quantize_append(const float *src, int B, int n_new, int Hkv,
+                                 const int32_t *start_pos, int64_t capacity,
+                                 uint64_t sign_seed, uint8_t *cache, void *stream) {
+    if (!src || !start_pos || !cache) return TBQ4_ERR_NULL;
+    if (!aligned(src, 16) || !aligned(cache, 16) || !aligned(start_pos, 4))
+        return TBQ4_ERR_ALIGN;
+    if (B <= 0 || n_new < 0 || Hkv <= 0) return TBQ4_ERR_SHAPE;
+    if (capacity <= 0 || capacity % 8 != 0) return TBQ4_ERR_CAPACITY;
+    if (n_new == 0) return TBQ4_OK;
+    uint64_t lo, hi;
+    sign_words(sign_seed, &lo, &hi);
+    const int64_t rows = (int64_t)B * n_new * Hkv;
+    const int threads = 256;
+    int64_t blocks = ceil_div(rows, threads / 32);
+    if (blocks > (int64_t)kNumSMs * 16) blocks = (int64_t)kNumSMs * 16;
+    quantize_append_kernel<<<(unsigned)blocks, threads, 0, (cudaStream_t)stream>>>(
+        src, B, n_new, Hkv, start_pos, capacity, lo, hi, cache);
+    return launch_status();
+}
+
+size_t tbq4_decode_workspace_bytes_split(int B, int Hq, int Hkv, int32_t max_len,
+                                         int32_t split_tokens) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || max_len < 0) return 0;
+    if (split_tokens == 0) split_tokens = auto_split_tokens(B, Hkv, max_len);
+    if (split_tokens <= 0) return 0;
+    return attn_ws_layout(B, Hq, max_len, split_tokens).total;
+}
+
+size_t tbq4_decode_workspace_bytes(int B, int Hq, int Hkv, int32_t max_len) {
+    return tbq4_decode_workspace_bytes_split(B, Hq, Hkv, max_len, 0);
+}
+
+tbq4_status tbq4_attn_decode_split(const float *q, const uint8_t *k_cache,
+                                   const uint8_t *v_cache, const int32_t *seq_lens,
+                                   int32_t max_len, int B, int Hq, int Hkv,
+                                   int64_t capacity, float softmax_scale,
+                                   uint64_t sign_seed, int32_t split_tokens,
+                                   void *workspace, size_t ws_bytes, uint16_t *out,
+                                   void *stream) {
+    if (!q || !k_cache || !v_cache || !seq_lens || !workspace || !out)
+        return TBQ4_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(workspace, kWsAlign) || !aligned(out, 2) || !aligned(seq_lens, 4))
+        return TBQ4_ERR_ALIGN;
+    if (B <= 0 || B > 65535 || Hkv <= 0 || Hkv > 65535 || Hq <= 0 || Hq % Hkv != 0 ||
+        Hq / Hkv > kMaxGroup || max_len < 0 || split_tokens < 0 || split_tokens % 32 != 0)
+        return TBQ4_ERR_SHAPE;
+    if (capacity <= 0 || capacity % 8 != 0 || (int64_t)max_len > capacity)
+        return TBQ4_ERR_CAPACITY;
+    if (!std::isfinite(softmax_scale)) return TBQ4_ERR_SHAPE;
+    AttnParams p = {};
+    p.q = q;
+    p.q_bf16 = 0;
+    p.k = k_cache;
+    p.v = v_cache;
+    p.head_stride = capacity * kBlockBytes;
+    p.seq_stride = (int64_t)Hkv * p.head_stride;
+    p.seq_lens = seq_lens;
+    p.max_len = max_len;
+    p.capacity = capacity;
+    p.nseq = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = Hq / Hkv;
+    p.split_tokens = split_tokens ? split_tokens : auto_split_tokens(B, Hkv, max_len);
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    sign_words(sign_seed, &p.sign_lo, &p.sign_hi);
+    p.out = out;
+    p.out_bf16 = 0;
+    return run_attention(p, workspace, ws_bytes, (cudaStream_t)stream);
+}
+
+tbq4_status tbq4_attn_decode(const float *q, const uint8_t *k_cache,
+                             const uint8_t *v_cache, const int32_t *seq_lens,
+                             int32_t max_len, int B, int Hq, int Hkv, int64_t capacity,
+                             float softmax_scale, uint64_t sign_seed, void *workspace,
+                             size_t ws_bytes, uint16_t *out, void *stream) {
+    return tbq4_attn_decode_split(q, k_cache, v_cache, seq_lens, max_len, B, Hq, Hkv,
+                                  capacity, softmax_scale, sign_seed, 0, workspace,
+                                  ws_bytes, out, stream);
+}
+
+size_t tbq4_prefill_workspace_bytes(int n_new, int Hq, int Hkv, int64_t n_cached) {
+    if (n_new <= 0 || Hq <= 0 || Hkv <= 0 || n_cached < 0) return 0;
+    const int64_t max_len = n_cached + n_new;
+    if (max_len > INT32_MAX) return 0;
+    const int32_t st = auto_split_tokens(n_new, Hkv, (int32_t)max_len);
+    return attn_ws_layout(n_new, Hq, (int32_t)max_len, st).total;
+}
+
+tbq4_status tbq4_attn_prefill_chunk(const uint16_t *q, int n_new, int64_t n_cached,
+                                    const uint8_t *k_cache, const uint8_t *v_cache,
+                                    int Hq, int Hkv, int64_t capacity,
+                                    float softmax_scale, uint64_t sign_seed,
+                                    void *workspace, size_t ws_bytes, uint16_t *out,
+                                    void *stream) {
+    if (!q || !k_cache || !v_cache || !workspace || !out) return TBQ4_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(workspace, kWsAlign) || !aligned(out, 2))
+        return TBQ4_ERR_ALIGN;
+    if (n_new <= 0 || n_new > 65535 || Hkv <= 0 || Hq <= 0 || Hq % Hkv != 0 ||
+        Hq / Hkv > kMaxGroup || n_cached < 0)
+        return TBQ4_ERR_SHAPE;
+    if (capacity <= 0 || capacity % 8 != 0 || n_cached + n_new > capacity ||
+        n_cached + n_new > INT32_MAX)
+        return TBQ4_ERR_CAPACITY;
+    if (!std::isfinite(softmax_scale)) return TBQ4_ERR_SHAPE;
+    AttnParams p = {};
+    p.q = q;
+    p.q_bf16 = 1;
+    p.k = k_cache;
+    p.v = v_cache;
+    p.head_stride = capacity * kBlockBytes;
+    p.seq_stride = 0;                          // every query row reads the same cache
+    p.seq_lens = nullptr;
+    p.len_base = (int32_t)(n_cached + 1);      // row i sees keys 0 .. n_cached + i
+    p.max_len = (int32_t)(n_cached + n_new);
+    p.capacity = capacity;
+    p.nseq = n_new;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = Hq / Hkv;
+    p.split_tokens = auto_split_tokens(n_new, Hkv, p.max_len);
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    sign_words(sign_seed, &p.sign_lo, &p.sign_hi);
+    p.out = out;
+    p.out_bf16 = 1;
+    return run_attention(p, workspace, ws_bytes, (cudaStream_t)stream);
+}
+
+void tbq4_set_timing_events(void *before, void *after) {
+    g_ev_before = (cudaEvent_t)before;
+    g_ev_after = (cudaEvent_t)after;
+}
+
+tbq4_status tbq4_get_device_status(void *stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return TBQ4_ERR_LAUNCH;
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return TBQ4_ERR_LAUNCH;
+    if (v != 0) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess)
+            return TBQ4_ERR_LAUNCH;
+    }
+    return (tbq4_status)v;
+}
+
+const char *tbq4_status_string(tbq4_status s) {
+    switch (s) {
+        case TBQ4_OK: return "ok";
+        case TBQ4_ERR_NULL: return "a required pointer is NULL";
+        case TBQ4_ERR_ALIGN: return "a pointer is not suitably aligned";
+        case TBQ4_ERR_SHAPE: return "unsupported sizes or arguments";
+        case TBQ4_ERR_CAPACITY: return "position or length outside the cache capacity";
+        case TBQ4_ERR_WORKSPACE: return "workspace smaller than required";
+        case TBQ4_ERR_LAUNCH: return "a CUDA launch or query failed";
+        case TBQ4_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel gave up";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+"""Shared test plumbing: building caches on both sides, comparing results.
+
+The CUDA side is driven only through the package binding (the C ABI); the
+oracle side only through ``oracle``.  Both take their inputs from
+``long_context_attention_tbq4_b200.workloads``.
+"""
+import math
+
+import numpy as np
+
+D = 128
+DECODE_MAX_ABS = 2e-3
+DECODE_REL_L2 = 1e-3
+PREFILL_REL_L2 = 1e-2
+
+
+def rel_l2(got, want):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    return float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-300))
+
+
+def max_abs(got, want):
+    return float(np.abs(np.asarray(got, np.float64) - np.asarray(want, np.float64)).max())
+
+
+def oracle_caches(seqs, Hkv, capacity, seed):
+    """Oracle caches [B][Hkv][capacity][66] from per-sequence fp32 rows."""
+    import oracle
+    B = len(seqs)
+    cache = np.zeros((B, Hkv, capacity, 66), np.uint8)
+    for b, x in enumerate(seqs):
+        if len(x) == 0:
+            continue
+        sub = cache[b:b + 1]
+        oracle.quantize_append(x[None], np.zeros(1, np.int32), capacity, seed, sub)
+        cache[b:b + 1] = sub
+    return cache
+
+
+def gpu_caches(seqs, Hkv, capacity, seed, fill=None):
+    """GPU caches built by tbq4_quantize_append, one call per sequence."""
+    import torch
+    import long_context_attention_tbq4_b200 as T
+    B = len(seqs)
+    cache = T.empty_cache(B, Hkv, capacity)
+    if fill is not None:
+        cache.fill_(fill)
+    else:
+        cache.zero_()
+    for b, x in enumerate(seqs):
+        if len(x) == 0:
+            continue
+        src = torch.from_numpy(np.ascontiguousarray(x)[None]).cuda()
+        view = cache[b:b + 1]
+        T.tbq4_quantize_append(src, torch.zeros(1, dtype=torch.int32, device="cuda"), view,
+                               sign_seed=seed)
+    return cache
+
+
+def check_decode(got, want):
+    got = np.asarray(got, np.float64)
+    ma, rl = max_abs(got, want), rel_l2(got, want)
+    assert ma <= DECODE_MAX_ABS and rl <= DECODE_REL_L2, (ma, rl)
+    return ma, rl
+
+
+def capacity_for(n, multiple=8):
+    return max(multiple, int(math.ceil(n / multiple)) * multiple)

@@ -1,0 +1,102 @@
+"""GPU quantise-append against the oracle: packed bytes must be bit-exact."""
+import numpy as np
+import pytest
+
+import oracle
+from long_context_attention_tbq4_b200 import workloads as W
+
+from helpers import gpu_caches, oracle_caches
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def T():
+    import torch
+    import long_context_attention_tbq4_b200 as pkg
+    assert torch.cuda.is_available()
+    return pkg
+
+
+def _gpu_append(T, src, start, capacity, seed, fill=0xAB):
+    import torch
+    B, n_new, Hkv, _ = src.shape
+    cache = T.empty_cache(B, Hkv, capacity)
+    cache.fill_(fill)
+    T.tbq4_quantize_append(torch.from_numpy(src).cuda(),
+                           torch.from_numpy(np.asarray(start, np.int32)).cuda(), cache,
+                           sign_seed=seed)
+    assert T.tbq4_get_device_status() == 0
+    return cache.cpu().numpy()
+
+
+def _oracle_append(src, start, capacity, seed, fill=0xAB):
+    B, n_new, Hkv, _ = src.shape
+    cache = np.full((B, Hkv, capacity, 66), fill, np.uint8)
+    oracle.quantize_append(src, np.asarray(start, np.int32), capacity, seed, cache)
+    return cache
+
+
+@pytest.mark.parametrize("dist,gain", [("normal", 1.0), ("t4", 1.0), ("normal", 1e-3),
+                                       ("t4", 300.0), ("normal", 1e-6), ("normal", 5e3)])
+def test_bytes_bit_exact_small(T, dist, gain):
+    rng = np.random.default_rng(hash((dist, gain)) % 2**32)
+    B, n_new, Hkv, cap = 3, 37, 3, 64
+    if dist == "normal":
+        src = rng.standard_normal((B, n_new, Hkv, 128)).astype(np.float32)
+    else:
+        src = rng.standard_t(4, (B, n_new, Hkv, 128)).astype(np.float32)
+    src *= np.float32(gain)
+    src[0, 3] = 0.0                                   # zero rows -> scale 0, index 8
+    src[1, 5, 0, 17] = 1e9                            # saturating scale
+    start = [3, 16, 27]
+    for seed in [0, 99]:
+        got = _gpu_append(T, src, start, cap, seed)
+        want = _oracle_append(src, start, cap, seed)
+        assert np.array_equal(got, want)
+
+
+def test_ragged_tail_and_single_rows(T):
+    rng = np.random.default_rng(7)
+    for n_new in [1, 2, 7, 8, 9, 31, 33]:
+        src = rng.standard_normal((2, n_new, 1, 128)).astype(np.float32)
+        got = _gpu_append(T, src, [0, 40 - n_new], 40, 0)
+        want = _oracle_append(src, [0, 40 - n_new], 40, 0)
+        assert np.array_equal(got, want)
+
+
+def test_out_of_range_rows_are_skipped_and_flagged(T):
+    import torch
+    rng = np.random.default_rng(8)
+    src = rng.standard_normal((1, 6, 2, 128)).astype(np.float32)
+    cache = T.empty_cache(1, 2, 8)
+    cache.fill_(0xAB)
+    T.tbq4_quantize_append(torch.from_numpy(src).cuda(),
+                           torch.tensor([5], dtype=torch.int32, device="cuda"), cache)
+    assert T.tbq4_get_device_status() == 4           # TBQ4_ERR_CAPACITY
+    assert T.tbq4_get_device_status() == 0           # cleared
+    want = _oracle_append(src, [5], 8, 0)
+    assert np.array_equal(cache.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("case", ["decode_32k", "decode_262k", "ragged", "prefill"])
+def test_bytes_bit_exact_workloads(T, case):
+    if case == "decode_32k":
+        c = W.decode_32k()
+        seqs_k, seqs_v, Hkv = c.k, c.v, c.Hkv
+    elif case == "decode_262k":
+        c = W.decode_262k()
+        seqs_k, seqs_v, Hkv = c.k, c.v, c.Hkv
+    elif case == "ragged":
+        c = W.ragged_decode()
+        seqs_k, seqs_v, Hkv = c.k, c.v, c.Hkv
+    else:
+        c = W.prefill_131k()
+        seqs_k, seqs_v, Hkv = [c.k], [c.v], c.Hkv
+    cap = W.round_capacity(max(len(x) for x in seqs_k))
+    for seqs in (seqs_k, seqs_v):
+        got = gpu_caches(seqs, Hkv, cap, W.SIGN_SEED).cpu().numpy()
+        want = oracle_caches(seqs, Hkv, cap, W.SIGN_SEED)
+        for b, x in enumerate(seqs):
+            n = len(x)
+            assert np.array_equal(got[b, :, :n], want[b, :, :n]), (case, b)
