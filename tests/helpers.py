@@ -58,10 +58,25 @@ def gpu_caches(seqs, Hkv, capacity, seed, fill=None):
     return cache
 
 
+def half_ulp_fp16(x):
+    """Half a unit in the last place of fp16 at |x|: the rounding error the
+    fp16 output format itself allows (2^-25 in the subnormal range)."""
+    a = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -14)))
+    return 2.0 ** (e - 11)
+
+
 def check_decode(got, want):
+    """max-abs <= 2e-3 beyond the fp16 output rounding, rel-L2 <= 1e-3.
+
+    The decode output is fp16, so even an exact kernel is off by up to half
+    an fp16 ulp of the true value (1.95e-3 at |o| in [4, 8)); the absolute
+    bound is applied on top of that allowance."""
     got = np.asarray(got, np.float64)
-    ma, rl = max_abs(got, want), rel_l2(got, want)
-    assert ma <= DECODE_MAX_ABS and rl <= DECODE_REL_L2, (ma, rl)
+    want = np.asarray(want, np.float64)
+    excess = np.abs(got - want) - half_ulp_fp16(want)
+    ma, rl = float(excess.max()), rel_l2(got, want)
+    assert ma <= DECODE_MAX_ABS and rl <= DECODE_REL_L2, (ma, max_abs(got, want), rl)
     return ma, rl
 
 
