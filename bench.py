@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--prefill-steps", type=int, default=5)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["decode", "prefill"], default=None,
+                    help="only run warm-up + steps of one workload's step, untimed, with "
+                         "no flush buffer (a small footprint for ncu captures)")
     return ap.parse_args()
 
 
@@ -294,6 +297,61 @@ def bench_prefill(T, torch, steps, warmup, flush):
             "attn_kernel_tflops": flops / (kern_ms * 1e-3) / 1e12, "steps": steps}
 
 
+def profile_decode(T, torch, case, N, n_steps):
+    """Decode steps at 262K with nothing else on the device (for ncu)."""
+    dev = torch.device("cuda")
+    kc = T.empty_cache(1, case.Hkv, N)
+    vc = T.empty_cache(1, case.Hkv, N)
+    zero = torch.zeros(1, dtype=torch.int32, device=dev)
+    for cache, x in ((kc, case.k[0]), (vc, case.v[0])):
+        src = torch.from_numpy(np.ascontiguousarray(x)[None]).to(dev)
+        T.tbq4_quantize_append(src, zero, cache, case.sign_seed)
+        del src
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    q = torch.from_numpy(case.q).to(dev)
+    lens = torch.tensor([N], dtype=torch.int32, device=dev)
+    ws = torch.empty(T.tbq4_decode_workspace_bytes(1, case.Hq, case.Hkv, N), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty((1, case.Hq, D), dtype=torch.float16, device=dev)
+    for _ in range(n_steps):
+        T.tbq4_attn_decode(q, kc, vc, lens, N, case.softmax_scale, case.sign_seed,
+                           workspace=ws, out=out)
+    torch.cuda.synchronize()
+    assert T.tbq4_get_device_status() == 0
+    print("profile: %d decode steps at %d keys" % (n_steps, N))
+    return 0
+
+
+def profile_prefill(T, torch, n_steps):
+    """Chunked-prefill steps (append the chunk, attend) with nothing else on
+    the device (for ncu)."""
+    from long_context_attention_tbq4_b200 import workloads as W
+    c = W.prefill_131k()
+    dev = torch.device("cuda")
+    cap = W.round_capacity(c.n_cached + c.n_new)
+    kc = T.empty_cache(1, c.Hkv, cap)
+    vc = T.empty_cache(1, c.Hkv, cap)
+    zero = torch.zeros(1, dtype=torch.int32, device=dev)
+    for cache, x in ((kc, c.k), (vc, c.v)):
+        src = torch.from_numpy(np.ascontiguousarray(x)[None]).to(dev)
+        T.tbq4_quantize_append(src, zero, cache, c.sign_seed)
+        del src
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    q = torch.from_numpy(c.q_bf16.view(np.int16)).to(dev).view(torch.bfloat16)
+    ws = torch.empty(T.tbq4_prefill_workspace_bytes(c.n_new, c.Hq, c.Hkv, c.n_cached),
+                     dtype=torch.uint8, device=dev)
+    out = torch.empty((c.n_new, c.Hq, D), dtype=torch.bfloat16, device=dev)
+    for _ in range(n_steps):
+        T.tbq4_attn_prefill_chunk(q, c.n_cached, kc[0], vc[0], c.softmax_scale, c.sign_seed,
+                                  workspace=ws, out=out)
+    torch.cuda.synchronize()
+    assert T.tbq4_get_device_status() == 0
+    print("profile: %d prefill steps, %d new over %d cached" % (n_steps, c.n_new, c.n_cached))
+    return 0
+
+
 # ------------------------------------------------------------ CPU baseline
 def oracle_decode_sample(case, N, rows):
     """Oracle caches (built once, untimed) and a timed call on `rows`."""
@@ -410,6 +468,10 @@ def main():
 
     peaks = measured_peaks()
     case, N, step_bytes, kernel_bytes = decode_workload()
+    if args.profile == "decode":
+        return profile_decode(T, torch, case, N, args.steps + args.warmup)
+    if args.profile == "prefill":
+        return profile_prefill(T, torch, args.steps + args.warmup)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     uuid = str(getattr(torch.cuda.get_device_properties(local), "uuid", "") or "")
     with Clocks(uuid) as clk:

@@ -1,10 +1,10 @@
-// decode.cuh -- split-K flash-decode over TBQ4 caches, and the log-sum-exp
-// combine that applies the inverse rotation.
+// decode.cuh -- parameters shared by the attention kernels, and the
+// log-sum-exp combine of split partials that applies the inverse rotation.
 //
 // The attention runs in the rotated domain (trefon.com, "Kontekst 262K na
 // jednej RTX 4090", section "Od czego zaczalem"): q is rotated once per
 // CTA, every K/V block is dequantised in the inner loop straight from the
-// raw bytes, and the output row is rotated back once, in the combine.
+// raw bytes, and each output row is rotated back once, here.
 //
 // Level arithmetic.  A block dequantises to (S/15) * L with L = 2*index-15,
 // an odd integer in [-15, 15].  The per-token factor S/15 is applied to the
@@ -33,6 +33,7 @@ struct AttnParams {
     float2 *part_ml;            // [nseq][Hq][n_splits]  (max in log2 units, sum)
     void *out;                  // [nseq][Hq][128], fp16 or bf16
     int out_bf16;
+    int all_splits;             // combine every split (prefill) instead of ceil(len/split)
 };
 
 __device__ __forceinline__ int32_t seq_length(const AttnParams &p, int s) {
@@ -52,159 +53,79 @@ __device__ __forceinline__ float load_q(const AttnParams &p, int64_t idx) {
     return reinterpret_cast<const float *>(p.q)[idx];
 }
 
-// One CTA = one (sequence, KV head, split).  Four warps take interleaved
-// tokens of the split; each lane owns four dimensions; the G query heads of
-// the KV head share every dequantised block.
-constexpr int kSplitWarps = 4;
+// One CTA per (sequence, query head): merge the split partials by
+// log-sum-exp, then o = D H o_rot / sqrt(128) (H is symmetric, so R^T = D H
+// c) and round to fp16 or bf16.  Eight warps take interleaved splits with a
+// running max each (independent loads, no dependent chain over the splits);
+// each lane owns four dimensions (one float4).  Warp 0 merges the warps and
+// applies the inverse rotation with the same shuffle transform as q.
+constexpr int kCombineWarps = 8;
 
-__global__ void __launch_bounds__(kSplitWarps * 32)
-decode_split_kernel(const AttnParams p) {
-    __shared__ float q_s[kMaxGroup][kD];
-    __shared__ float m_w[kSplitWarps][kMaxGroup], l_w[kSplitWarps][kMaxGroup];
-    __shared__ float o_w[kSplitWarps][kMaxGroup][kD];
-
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int split = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
-    const int G = p.G;
-    const int32_t len = seq_length(p, s);
-    const int32_t t0 = split * p.split_tokens;
-    const int32_t t1 = min(len, t0 + p.split_tokens);
-
-    // q_rot * softmax_scale * log2(e) / 15, one head per warp.
-    const uint32_t sbits = lane_sign_bits(p.sign_lo, p.sign_hi, lane);
-    for (int hh = warp; hh < G; hh += kSplitWarps) {
-        const int64_t base = ((int64_t)s * p.Hq + g * G + hh) * kD + 4 * lane;
-        float v[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) v[k] = load_q(p, base + k);
-        warp_rotate128(v, sbits, lane);
-        const float f = p.scale_log2 * (1.0f / 15.0f);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) q_s[hh][4 * lane + k] = v[k] * f;
-    }
-    __syncthreads();
-
-    float qr[kMaxGroup][4], m[kMaxGroup], l[kMaxGroup], o[kMaxGroup][4];
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-        m[h] = -INFINITY;
-        l[h] = 0.f;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            qr[h][k] = h < G ? q_s[h][4 * lane + k] : 0.f;
-            o[h][k] = 0.f;
-        }
-    }
-
-    const uint8_t *kb = p.k + s * p.seq_stride + g * p.head_stride;
-    const uint8_t *vb = p.v + s * p.seq_stride + g * p.head_stride;
-    for (int32_t t = t0 + warp; t < t1; t += kSplitWarps) {
-        const uint8_t *kr = kb + (int64_t)t * kBlockBytes;
-        const uint8_t *vr = vb + (int64_t)t * kBlockBytes;
-        const uint32_t kn = __ldg(reinterpret_cast<const uint16_t *>(kr + 2) + lane);
-        const uint32_t vn = __ldg(reinterpret_cast<const uint16_t *>(vr + 2) + lane);
-        const float sk = half_bits_to_float(__ldg(reinterpret_cast<const uint16_t *>(kr)));
-        const float sv = half_bits_to_float(__ldg(reinterpret_cast<const uint16_t *>(vr)))
-                         * (1.0f / 15.0f);
-        float lk[4], lv[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            lk[k] = (float)(2 * (int)((kn >> (4 * k)) & 15u) - 15);
-            lv[k] = (float)(2 * (int)((vn >> (4 * k)) & 15u) - 15);
-        }
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) {
-            if (h >= G) break;
-            float d = qr[h][0] * lk[0] + qr[h][1] * lk[1] + qr[h][2] * lk[2] + qr[h][3] * lk[3];
-            d = warp_sum(d) * sk;
-            const float mn = fmaxf(m[h], d);
-            const float corr = exp2f(m[h] - mn);
-            const float pr = exp2f(d - mn);
-            l[h] = l[h] * corr + pr;
-            const float pv = pr * sv;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) o[h][k] = o[h][k] * corr + pv * lv[k];
-            m[h] = mn;
-        }
-    }
-
-    // Merge the four warps, then write this split's partial.
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-        if (h >= G) break;
-        if (lane == 0) { m_w[warp][h] = m[h]; l_w[warp][h] = l[h]; }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) o_w[warp][h][4 * lane + k] = o[h][k];
-    }
-    __syncthreads();
-    const int d = threadIdx.x;
-    for (int h = 0; h < G; ++h) {
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kSplitWarps; ++w) M = fmaxf(M, m_w[w][h]);
-        float O = 0.f, L = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < kSplitWarps; ++w) {
-                const float mw = m_w[w][h];
-                const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
-                O += f * o_w[w][h][d];
-                L += f * l_w[w][h];
-            }
-        }
-        const int64_t row = ((int64_t)s * p.Hq + g * G + h) * p.n_splits + split;
-        p.part_o[row * kD + d] = O;
-        if (d == 0) p.part_ml[row] = make_float2(M, L);
-    }
-}
-
-// One CTA of 128 threads per (sequence, query head): merge the splits by
-// log-sum-exp, then o = D H o_rot / sqrt(128) (H symmetric, so R^T = D H c)
-// and round to fp16 or bf16.
-__global__ void __launch_bounds__(kD)
+__global__ void __launch_bounds__(kCombineWarps * 32)
 decode_combine_kernel(const AttnParams p) {
-    __shared__ float x_s[kD];
-    const int d = threadIdx.x, lane = d & 31;
+    __shared__ float4 o_s[kCombineWarps][32];
+    __shared__ float m_s[kCombineWarps], l_s[kCombineWarps];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int h = blockIdx.x, s = blockIdx.y;
     const int32_t len = seq_length(p, s);
-    const int used = (len + p.split_tokens - 1) / p.split_tokens;
+    const int used = p.all_splits ? p.n_splits : (len + p.split_tokens - 1) / p.split_tokens;
     const int64_t row0 = ((int64_t)s * p.Hq + h) * p.n_splits;
 
-    float M = -INFINITY;
-    for (int i = 0; i < used; ++i) M = fmaxf(M, p.part_ml[row0 + i].x);
-    float O = 0.f, L = 0.f;
-    if (M != -INFINITY) {
-        for (int i = 0; i < used; ++i) {
-            const float2 ml = p.part_ml[row0 + i];
-            const float f = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
-            O += f * p.part_o[(row0 + i) * kD + d];
-            L += f * ml.y;
+    float M = -INFINITY, L = 0.f;
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int i = warp; i < used; i += kCombineWarps) {
+        const float2 ml = p.part_ml[row0 + i];
+        const float4 oi = reinterpret_cast<const float4 *>(p.part_o + (row0 + i) * kD)[lane];
+        if (ml.x == -INFINITY) continue;                  // empty split
+        const float Mn = fmaxf(M, ml.x);
+        const float a = M == -INFINITY ? 0.f : exp2f(M - Mn);
+        const float b = exp2f(ml.x - Mn);
+        O.x = O.x * a + oi.x * b;
+        O.y = O.y * a + oi.y * b;
+        O.z = O.z * a + oi.z * b;
+        O.w = O.w * a + oi.w * b;
+        L = L * a + ml.y * b;
+        M = Mn;
+    }
+    o_s[warp][lane] = O;
+    if (lane == 0) { m_s[warp] = M; l_s[warp] = L; }
+    __syncthreads();
+    if (warp != 0) return;
+
+    float Mt = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) Mt = fmaxf(Mt, m_s[w]);
+    float v[4] = {0.f, 0.f, 0.f, 0.f}, Lt = 0.f;
+    if (Mt != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < kCombineWarps; ++w) {
+            const float f = m_s[w] == -INFINITY ? 0.f : exp2f(m_s[w] - Mt);
+            const float4 ow = o_s[w][lane];
+            v[0] += f * ow.x;
+            v[1] += f * ow.y;
+            v[2] += f * ow.z;
+            v[3] += f * ow.w;
+            Lt += f * l_s[w];
         }
     }
-    float x = L > 0.f ? O / L : 0.f;
-
-    // Walsh-Hadamard transform across the 128 threads.
+    const float inv = Lt > 0.f ? 1.0f / Lt : 0.f;
 #pragma unroll
-    for (int m = 1; m < 32; m <<= 1) {
-        const float o = __shfl_xor_sync(kFull, x, m);
-        x = (lane & m) ? o - x : x + o;
-    }
+    for (int k = 0; k < 4; ++k) v[k] *= inv;
+    // inverse rotation: transform, scale, then the sign diagonal
+    warp_fwht128(v, lane);
+    const uint32_t sbits = lane_sign_bits(p.sign_lo, p.sign_hi, lane);
+    const float c = rot_c();
+    const int64_t oi = ((int64_t)s * p.Hq + h) * kD + 4 * lane;
 #pragma unroll
-    for (int m = 32; m < kD; m <<= 1) {
-        x_s[d] = x;
-        __syncthreads();
-        const float o = x_s[d ^ m];
-        __syncthreads();
-        x = (d & m) ? o - x : x + o;
+    for (int k = 0; k < 4; ++k) {
+        float x = v[k] * c;
+        if ((sbits >> k) & 1u) x = -x;
+        if (p.out_bf16)
+            reinterpret_cast<__nv_bfloat16 *>(p.out)[oi + k] = __float2bfloat16_rn(x);
+        else
+            reinterpret_cast<__half *>(p.out)[oi + k] = __float2half_rn(x);
     }
-    const uint64_t w = d < 64 ? p.sign_lo : p.sign_hi;
-    x *= rot_c();
-    if ((w >> (d & 63)) & 1u) x = -x;
-    const int64_t oi = ((int64_t)s * p.Hq + h) * kD + d;
-    if (p.out_bf16)
-        reinterpret_cast<__nv_bfloat16 *>(p.out)[oi] = __float2bfloat16_rn(x);
-    else
-        reinterpret_cast<__half *>(p.out)[oi] = __float2half_rn(x);
 }
 
 }  // namespace tbq4

@@ -1,0 +1,458 @@
+// decode_tc.cuh -- split-K flash-decode over TBQ4 caches on the tensor cores.
+//
+// One CTA = one (sequence, KV head, split of the context).  Each warp
+// streams its own 32-token chunks of raw K and V blocks (32 x 66 bytes each)
+// from HBM into a private shared-memory ring with cp.async.bulk and an
+// mbarrier per stage; the blocks are dequantised in registers inside the
+// inner loop (no dequantisation pass, no fp16 copy of the cache: trefon.com,
+// "Kontekst 262K na jednej RTX 4090", section "Od czego zaczalem") and the
+// G query heads of the KV head share every block through the tensor cores:
+//
+//   S^T (32 tokens x 8 heads) = K (tokens x 128) . Q_rot^T   mma m16n8k32 u8 x s8
+//   O^T (128 dims x 8 heads) += V^T (dims x tokens) . P'^T    mma m16n8k16 f16
+//
+// K operand: the nibbles themselves, as unsigned bytes (two LOP3 and a
+// shift per 8 values).  q_rot is normalised by a power of two and held as a
+// 22-bit fixed-point integer split into three signed bytes, so the integer
+// MMAs give sum_d n_d q_d exactly; the level map is applied afterwards,
+// sum_d q_d (2n_d - 15) = 2 sum_d n_d q_d - 15 sum_d q_d.  (fp16 q was not
+// enough: heavy-tailed keys turn a 2^-12 error in q into output errors of a
+// few 1e-3 where one token dominates.)
+// V operand: pairs of tokens are interleaved with PRMT so that one register
+// holds the same dimension of two tokens; the levels enter as n - 8 and the
+// odd level 2n - 15 is restored at the end (see lvl_lo).  P' = p * S_v (the
+// block scale of V), so O = sum_t p_t S_v,t (2n-15) / 15.
+// Softmax runs in fp32 in the log2 domain; the running max is per head and
+// the accumulators are only rescaled when some head's max grows.
+#pragma once
+#include "common.cuh"
+#include "decode.cuh"
+
+namespace tbq4 {
+
+constexpr int kTcWarps = 8;
+constexpr int kTcStages = 3;
+constexpr int kChunk = 32;                                 // tokens per chunk
+constexpr int kChunkBytes = kChunk * kBlockBytes;          // 2112
+constexpr int kStageBytes = 2 * kChunkBytes + 16;          // K | V | pad
+constexpr int kWarpRing = kTcStages * kStageBytes;
+constexpr int kRingBytes = kTcWarps * kWarpRing;
+constexpr int kTcSmemBytes = kRingBytes + kTcWarps * kTcStages * 8 + 128;
+constexpr uint32_t kSpinLimit = 1u << 22;                  // bounded mbarrier wait
+
+static_assert(kStageBytes % 16 == 0, "stage must keep 16-byte alignment");
+static_assert(kRingBytes >= kTcWarps * kMaxGroup * kD * 4 + 2 * kTcWarps * kMaxGroup * 4,
+              "merge buffers reuse the ring");
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase with the given parity; gives up after kSpinLimit
+// polls and returns false (warp-uniform).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+    bool ok = false;
+    for (uint32_t i = 0; i < kSpinLimit && !ok; ++i) ok = mbar_try_wait(bar, parity);
+    return __all_sync(kFull, ok);
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                         uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D (s32) += A (u8, 16x32 row) * B (s8, 32x8 col)
+__device__ __forceinline__ void imma16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float lds_half(uint32_t addr) {
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return __half2float(__ushort_as_half(v));
+}
+
+// V levels enter the tensor cores as n - 8 (exact in fp16), built from a
+// magic-exponent fp16 and one HADD2: nibble in mantissa bits 0-3 under the
+// exponent of 1024 gives 1024 + n, in bits 4-7 under 64 gives 64 + n.  Since
+// 2n - 15 = 2 (n - 8) + 1, O = 2 sum_t P'_t (n_t - 8) + sum_t P'_t; the second
+// sum (R) comes from one extra MMA per k-step with an all-ones A operand.
+constexpr uint32_t kH2Neg1032 = 0xE408E408u;   // {-1032, -1032}
+constexpr uint32_t kH2Neg72 = 0xD480D480u;     // {-72, -72}
+constexpr uint32_t kH2Ones = 0x3C003C00u;      // {1, 1}
+
+__device__ __forceinline__ uint32_t hadd2_u32(uint32_t x, uint32_t a) {
+    __half2 r = __hadd2(*reinterpret_cast<__half2 *>(&x), *reinterpret_cast<__half2 *>(&a));
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+// low nibbles of bytes 0 and 2 -> {n - 8, n - 8}
+__device__ __forceinline__ uint32_t lvl_lo(uint32_t v) {
+    return hadd2_u32((v & 0x000F000Fu) | 0x64006400u, kH2Neg1032);
+}
+// high nibbles of bytes 0 and 2 -> {n - 8, n - 8}
+__device__ __forceinline__ uint32_t lvl_hi(uint32_t v) {
+    return hadd2_u32((v & 0x00F000F0u) | 0x54005400u, kH2Neg72);
+}
+
+// 32-bit word of nibble bytes at an arbitrary 2-byte-aligned shared address:
+// two aligned loads and a funnel shift by 0 or 16 bits.
+struct Funnel {
+    uint32_t base, sh;
+    __device__ __forceinline__ Funnel(uint32_t addr) : base(addr & ~3u), sh((addr & 3u) * 8u) {}
+};
+
+__global__ void __launch_bounds__(kTcWarps * 32, 2)
+decode_tc_kernel(const AttnParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint8_t *ring = smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kRingBytes);
+    // prologue scratch inside the ring (before any copy is issued)
+    float *qpar = reinterpret_cast<float *>(ring + 3 * kMaxGroup * kD);    // [8][2]
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int r = lane >> 2, c = lane & 3;
+    const int split = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+    const int G = p.G;
+    const int32_t len = seq_length(p, s);
+    const int32_t t0 = split * p.split_tokens;
+    const int32_t t1 = min(len, t0 + p.split_tokens);
+    const int n_chunks = t1 > t0 ? (t1 - t0 + kChunk - 1) / kChunk : 0;
+
+    // ---- q: rotate, normalise by a power of two, split into three bytes ----
+    // q_int = rint(q_rot * 2^(22-e)) with 2^e > max|q_rot|, so |q_int| <= 2^22;
+    // q_int = 65536 c2 + 256 c1 + c0 with c0, c1 in [-128, 127], |c2| <= 64.
+    int8_t *q8 = reinterpret_cast<int8_t *>(ring);                       // [3][8][128]
+    if (warp < G) {
+        const uint32_t sbits = lane_sign_bits(p.sign_lo, p.sign_hi, lane);
+        const int64_t base = ((int64_t)s * p.Hq + g * G + warp) * kD + 4 * lane;
+        float v[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) v[k] = load_q(p, base + k);
+        warp_rotate128(v, sbits, lane);
+        float mx = warp_max(fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
+        int e = 0;
+        if (mx > 0.f) frexpf(mx, &e);                 // mx = f * 2^e, f in [0.5, 1)
+        int qsum = 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int qi = __float2int_rn(ldexpf(v[k], 22 - e));
+            const int c0 = ((qi + 128) & 255) - 128;
+            const int q1 = (qi - c0) >> 8;
+            const int c1 = ((q1 + 128) & 255) - 128;
+            const int c2 = (q1 - c1) >> 8;
+            q8[(0 * kMaxGroup + warp) * kD + 4 * lane + k] = (int8_t)c0;
+            q8[(1 * kMaxGroup + warp) * kD + 4 * lane + k] = (int8_t)c1;
+            q8[(2 * kMaxGroup + warp) * kD + 4 * lane + k] = (int8_t)c2;
+            qsum += qi;
+        }
+        qsum = __reduce_add_sync(kFull, qsum);
+        if (lane == 0) {
+            // log2 logit = (2 S - 15 sum q) * S_k * scale * log2(e) / 15 * 2^(e-22)
+            const float fh = p.scale_log2 * (1.0f / 15.0f) * ldexpf(1.0f, e - 22);
+            qpar[2 * warp + 0] = 2.0f * fh;
+            qpar[2 * warp + 1] = -15.0f * (float)qsum * fh;
+        }
+    } else if (warp < kMaxGroup) {
+        for (int k = lane; k < kD; k += 32)
+            for (int pc = 0; pc < 3; ++pc) q8[(pc * kMaxGroup + warp) * kD + k] = 0;
+        if (lane == 0) { qpar[2 * warp] = 0.f; qpar[2 * warp + 1] = 0.f; }
+    }
+    __syncthreads();
+
+    // B fragments of the q pieces (k = dims, n = heads), thread (n = r, c):
+    // k-step i covers dims 32c+8i .. +7; b0 = bytes of dims +0,+2,+4,+6,
+    // b1 = dims +1,+3,+5,+7 (matching the lo/hi nibble split of the word).
+    uint32_t qb[4][3][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int pc = 0; pc < 3; ++pc) {
+            const uint8_t *row =
+                reinterpret_cast<const uint8_t *>(q8) + (pc * kMaxGroup + r) * kD + 32 * c + 8 * i;
+            qb[i][pc][0] = (uint32_t)row[0] | ((uint32_t)row[2] << 8) | ((uint32_t)row[4] << 16) |
+                           ((uint32_t)row[6] << 24);
+            qb[i][pc][1] = (uint32_t)row[1] | ((uint32_t)row[3] << 8) | ((uint32_t)row[5] << 16) |
+                           ((uint32_t)row[7] << 24);
+        }
+    }
+    // per-head constants for this thread's score columns (heads 2c, 2c+1)
+    const float f2a = qpar[4 * c + 0], bha = qpar[4 * c + 1];
+    const float f2b = qpar[4 * c + 2], bhb = qpar[4 * c + 3];
+    __syncthreads();   // the ring is about to be overwritten by copies
+
+    // ---- per-warp ring --------------------------------------------------
+    const uint32_t ring_w = smem_u32(ring) + warp * kWarpRing;
+    const uint32_t bar_w = smem_u32(bars) + warp * kTcStages * 8;
+    const uint8_t *kb = p.k + s * p.seq_stride + g * p.head_stride;
+    const uint8_t *vb = p.v + s * p.seq_stride + g * p.head_stride;
+    const int my_chunks = warp < n_chunks ? (n_chunks - warp + kTcWarps - 1) / kTcWarps : 0;
+
+    if (lane == 0) {
+        for (int st = 0; st < kTcStages; ++st) mbar_init(bar_w + 8 * st, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+
+    auto issue = [&](int k) {   // lane 0: copy the warp's k-th chunk
+        const int ci = warp + k * kTcWarps;
+        const int32_t start = t0 + ci * kChunk;
+        const int32_t valid = min(kChunk, t1 - start);
+        const uint32_t bytes = (uint32_t)((valid + 7) & ~7) * kBlockBytes;
+        const int st = k % kTcStages;
+        const uint32_t bar = bar_w + 8 * st;
+        const uint32_t dst = ring_w + st * kStageBytes;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_expect_tx(bar, 2 * bytes);
+        bulk_g2s(dst, kb + (int64_t)start * kBlockBytes, bytes, bar);
+        bulk_g2s(dst + kChunkBytes, vb + (int64_t)start * kBlockBytes, bytes, bar);
+    };
+    if (lane == 0)
+        for (int k = 0; k < min(kTcStages, my_chunks); ++k) issue(k);
+
+    float o[8][4];
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) o[mt][k] = 0.f;
+    float rr[4] = {0.f, 0.f, 0.f, 0.f};        // sum_t P'_t for heads 2c, 2c+1
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+    const uint32_t hsel = (r & 1) ? 0x7632u : 0x5410u;          // half of head n = r
+    const int src0 = 4 * (2 * c) + (r >> 1), src1 = 4 * (2 * c + 1) + (r >> 1);
+    bool aborted = false;
+
+    for (int k = 0; k < my_chunks; ++k) {
+        const int st = k % kTcStages;
+        if (!mbar_wait_bounded(bar_w + 8 * st, (uint32_t)(k / kTcStages) & 1u)) {
+            if (lane == 0) record_status(7u /* TBQ4_ERR_DEVICE_TIMEOUT */);
+            aborted = true;
+            break;
+        }
+        const int ci = warp + k * kTcWarps;
+        const int32_t valid = min(kChunk, t1 - (t0 + ci * kChunk));
+        const uint32_t kst = ring_w + st * kStageBytes;
+        const uint32_t vst = kst + kChunkBytes;
+
+        // ---- S^T = K Q^T for two 16-token tiles (exact, integer) ---------
+        float sc[2][4];
+#pragma unroll
+        for (int tile = 0; tile < 2; ++tile) {
+            int acc[3][4];
+#pragma unroll
+            for (int pc = 0; pc < 3; ++pc) acc[pc][0] = acc[pc][1] = acc[pc][2] = acc[pc][3] = 0;
+            const Funnel f0(kst + (16 * tile + r) * kBlockBytes + 2 + 16 * c);
+            const Funnel f1(kst + (16 * tile + r + 8) * kBlockBytes + 2 + 16 * c);
+            uint32_t w0[5], w1[5];
+#pragma unroll
+            for (int i = 0; i < 5; ++i) { w0[i] = lds32(f0.base + 4 * i); w1[i] = lds32(f1.base + 4 * i); }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t x0 = __funnelshift_r(w0[i], w0[i + 1], f0.sh);
+                const uint32_t x1 = __funnelshift_r(w1[i], w1[i + 1], f1.sh);
+                // bytes of dims +0,+2,+4,+6 (lo) and +1,+3,+5,+7 (hi) of the word
+                const uint32_t lo0 = x0 & 0x0F0F0F0Fu, hi0 = (x0 >> 4) & 0x0F0F0F0Fu;
+                const uint32_t lo1 = x1 & 0x0F0F0F0Fu, hi1 = (x1 >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+                for (int pc = 0; pc < 3; ++pc)
+                    imma16832(acc[pc], lo0, lo1, hi0, hi1, qb[i][pc][0], qb[i][pc][1]);
+            }
+            // sum_d n_d q_int_d = 65536 acc2 + 256 acc1 + acc0
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                sc[tile][e] = fmaf((float)acc[2][e], 65536.0f, (float)(acc[1][e] * 256 + acc[0][e]));
+        }
+
+        // ---- scores -> log2 logits, masked beyond `valid` -----------------
+        // thread's tokens: u = 0..3 -> token 8u + r (tile u>>1, row half u&1)
+        float lg[4][2], sv[4];
+        if (valid == kChunk) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = 8 * u + r;
+                const float sk = lds_half(kst + j * kBlockBytes);
+                sv[u] = lds_half(vst + j * kBlockBytes);
+                lg[u][0] = fmaf(sc[u >> 1][2 * (u & 1) + 0], f2a, bha) * sk;
+                lg[u][1] = fmaf(sc[u >> 1][2 * (u & 1) + 1], f2b, bhb) * sk;
+            }
+        } else {                                  // tail chunk: mask tokens >= valid
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = 8 * u + r;
+                const float sk = lds_half(kst + j * kBlockBytes);
+                const float svj = lds_half(vst + j * kBlockBytes);
+                const bool ok = j < valid;
+                lg[u][0] = ok ? fmaf(sc[u >> 1][2 * (u & 1) + 0], f2a, bha) * sk : -INFINITY;
+                lg[u][1] = ok ? fmaf(sc[u >> 1][2 * (u & 1) + 1], f2b, bhb) * sk : -INFINITY;
+                sv[u] = ok ? svj : 0.f;
+            }
+        }
+        float mxa = fmaxf(fmaxf(lg[0][0], lg[1][0]), fmaxf(lg[2][0], lg[3][0]));
+        float mxb = fmaxf(fmaxf(lg[0][1], lg[1][1]), fmaxf(lg[2][1], lg[3][1]));
+#pragma unroll
+        for (int msk = 4; msk < 32; msk <<= 1) {
+            mxa = fmaxf(mxa, __shfl_xor_sync(kFull, mxa, msk));
+            mxb = fmaxf(mxb, __shfl_xor_sync(kFull, mxb, msk));
+        }
+        if (__any_sync(kFull, mxa > m_a || mxb > m_b)) {
+            const float na = fmaxf(m_a, mxa), nb = fmaxf(m_b, mxb);
+            const float ca = exp2f(m_a - na), cb = exp2f(m_b - nb);
+            m_a = na;
+            m_b = nb;
+            l_a *= ca;
+            l_b *= cb;
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                o[mt][0] *= ca; o[mt][1] *= cb; o[mt][2] *= ca; o[mt][3] *= cb;
+            }
+            rr[0] *= ca; rr[1] *= cb; rr[2] *= ca; rr[3] *= cb;
+        }
+        uint32_t p2[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float pa = exp2f(lg[u][0] - m_a), pb = exp2f(lg[u][1] - m_b);
+            l_a += pa;
+            l_b += pb;
+            __half2 h = __floats2half2_rn(pa * sv[u], pb * sv[u]);
+            p2[u] = *reinterpret_cast<uint32_t *>(&h);
+        }
+        // P'^T B fragments: thread (n = r, c) needs head n, tokens
+        // 16ks + {2c, 2c+1} (b0) and 16ks + 8 + {2c, 2c+1} (b1).
+        uint32_t pb[2][2];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const uint32_t x = __shfl_sync(kFull, p2[u], src0);
+            const uint32_t y = __shfl_sync(kFull, p2[u], src1);
+            pb[u >> 1][u & 1] = __byte_perm(x, y, hsel);
+        }
+
+        // ---- O^T += V^T P'^T ---------------------------------------------
+        // thread (r, c): dims 16r .. 16r+15 (m-tile mt: rows r -> dim
+        // 16r+2mt, r+8 -> dim 16r+2mt+1), tokens 16ks + {2c,2c+1,2c+8,2c+9}.
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            uint32_t xw[4][2];   // [token 2c, 2c+1, 2c+8, 2c+9][word]
+#pragma unroll
+            for (int tt = 0; tt < 4; ++tt) {
+                const int j = 16 * ks + 2 * c + (tt & 1) + 8 * (tt >> 1);
+                const uint32_t a = vst + j * kBlockBytes + 2 + 8 * r;
+                if (tt & 1) {            // odd token: its nibbles are 4-byte aligned
+                    xw[tt][0] = lds32(a);
+                    xw[tt][1] = lds32(a + 4);
+                } else {                 // even token: 2 bytes past a 4-byte boundary
+                    const uint32_t w0 = lds32(a - 2), w1 = lds32(a + 2), w2 = lds32(a + 6);
+                    xw[tt][0] = __byte_perm(w0, w1, 0x5432);
+                    xw[tt][1] = __byte_perm(w1, w2, 0x5432);
+                }
+            }
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {        // byte pairs -> dims 16r + 4q4 .. +3
+                const uint32_t sel = (q4 & 1) ? 0x7632u : 0x5410u;
+                const int w = q4 >> 1;
+                const uint32_t X = __byte_perm(xw[0][w], xw[1][w], sel);   // pair (2c, 2c+1)
+                const uint32_t Y = __byte_perm(xw[2][w], xw[3][w], sel);   // pair (2c+8, 2c+9)
+                const uint32_t Xs = X >> 8, Ys = Y >> 8;
+                // dims 16r+4q4+{0,1} -> m-tile 2q4, rows r / r+8;
+                // dims 16r+4q4+{2,3} -> m-tile 2q4+1
+                mma16816(o[2 * q4], lvl_lo(X), lvl_hi(X), lvl_lo(Y), lvl_hi(Y), pb[ks][0], pb[ks][1]);
+                mma16816(o[2 * q4 + 1], lvl_lo(Xs), lvl_hi(Xs), lvl_lo(Ys), lvl_hi(Ys), pb[ks][0],
+                         pb[ks][1]);
+            }
+            mma16816(rr, kH2Ones, kH2Ones, kH2Ones, kH2Ones, pb[ks][0], pb[ks][1]);
+        }
+
+        __syncwarp();
+        if (lane == 0 && k + kTcStages < my_chunks) issue(k + kTcStages);
+    }
+
+    // ---- warp totals, CTA merge, partial write ----------------------------
+#pragma unroll
+    for (int msk = 4; msk < 32; msk <<= 1) {
+        l_a += __shfl_xor_sync(kFull, l_a, msk);
+        l_b += __shfl_xor_sync(kFull, l_b, msk);
+    }
+    if (aborted) { m_a = m_b = -INFINITY; }
+    __syncthreads();     // every warp is done with its ring
+    float *o_w = reinterpret_cast<float *>(ring);                       // [W][8][128]
+    float *m_w = o_w + kTcWarps * kMaxGroup * kD;                        // [W][8]
+    float *l_w = m_w + kTcWarps * kMaxGroup;                             // [W][8]
+    // sum_t P'_t (2n - 15) = 2 sum_t P'_t (n - 8) + sum_t P'_t
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+        const int d0 = 16 * r + 2 * mt;
+        o_w[(warp * kMaxGroup + 2 * c) * kD + d0] = fmaf(2.f, o[mt][0], rr[0]);
+        o_w[(warp * kMaxGroup + 2 * c + 1) * kD + d0] = fmaf(2.f, o[mt][1], rr[1]);
+        o_w[(warp * kMaxGroup + 2 * c) * kD + d0 + 1] = fmaf(2.f, o[mt][2], rr[2]);
+        o_w[(warp * kMaxGroup + 2 * c + 1) * kD + d0 + 1] = fmaf(2.f, o[mt][3], rr[3]);
+    }
+    if (r == 0) {
+        m_w[warp * kMaxGroup + 2 * c] = m_a;
+        m_w[warp * kMaxGroup + 2 * c + 1] = m_b;
+        l_w[warp * kMaxGroup + 2 * c] = l_a;
+        l_w[warp * kMaxGroup + 2 * c + 1] = l_b;
+    }
+    __syncthreads();
+    // 256 threads: thread = (head half, dim); levels carry a factor 15
+    const int d = threadIdx.x & (kD - 1);
+    for (int h = threadIdx.x >> 7; h < G; h += 2) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kTcWarps; ++w) M = fmaxf(M, m_w[w * kMaxGroup + h]);
+        float O = 0.f, L = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kTcWarps; ++w) {
+                const float mw = m_w[w * kMaxGroup + h];
+                const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
+                O += f * o_w[(w * kMaxGroup + h) * kD + d];
+                L += f * l_w[w * kMaxGroup + h];
+            }
+        }
+        const int64_t row = ((int64_t)s * p.Hq + g * G + h) * p.n_splits + split;
+        p.part_o[row * kD + d] = O * (1.0f / 15.0f);
+        if (d == 0) p.part_ml[row] = make_float2(M, L);
+    }
+}
+
+}  // namespace tbq4

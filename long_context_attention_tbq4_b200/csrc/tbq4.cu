@@ -8,7 +8,10 @@
 #include "common.cuh"
 #include "quantize.cuh"
 #include "decode.cuh"
+#include "decode_tc.cuh"
+#include "prefill_tc.cuh"
 
+#include <algorithm>
 #include <cmath>
 
 namespace {
@@ -37,10 +40,10 @@ void sign_words(uint64_t seed, uint64_t *lo, uint64_t *hi) {
     *hi = w[1];
 }
 
-// Keys per split: about four CTAs per SM over the whole launch, a multiple
-// of 32, at least 256.
+// Keys per split: one wave of the decode kernel (two CTAs per SM) over the
+// whole launch, a multiple of 32, at least 256.
 int32_t auto_split_tokens(int nseq, int Hkv, int32_t max_len) {
-    const int64_t target = (int64_t)kNumSMs * 4;
+    const int64_t target = (int64_t)kNumSMs * 2;
     int64_t per = ceil_div((int64_t)max_len * nseq * Hkv, target);
     per = ceil_div(per, 32) * 32;
     if (per < 256) per = 256;
@@ -64,6 +67,44 @@ WsLayout attn_ws_layout(int nseq, int Hq, int32_t max_len, int32_t split_tokens)
 
 cudaEvent_t g_ev_before = nullptr, g_ev_after = nullptr;
 
+// Prefill work: one CTA per (M-pair, key split); M-pair = two query heads of
+// a KV group x 128 query positions.  Key splits fill the 148 SMs (one CTA
+// per SM: the kernel takes all of tensor memory).
+struct PrefillPlan {
+    int pairs, iblocks, mpairs, n_splits;
+    size_t part_o, part_ml, total;
+};
+
+PrefillPlan prefill_ws_layout(int n_new, int Hq, int Hkv, int64_t n_cached) {
+    PrefillPlan w;
+    const int G = Hq / Hkv;
+    w.pairs = (G + 1) / 2;
+    w.iblocks = (n_new + pre::kTile - 1) / pre::kTile;
+    w.mpairs = Hkv * w.pairs * w.iblocks;
+    const int64_t tiles0 = (n_cached + std::min(n_new, pre::kTile) + pre::kTile - 1) / pre::kTile;
+    int64_t ns = kNumSMs / w.mpairs;
+    if (ns > tiles0) ns = tiles0;
+    if (ns < 1) ns = 1;
+    w.n_splits = (int)ns;
+    const size_t rows = (size_t)n_new * Hq * w.n_splits;
+    w.part_o = 0;
+    w.part_ml = align_up(rows * kD * sizeof(float), kWsAlign);
+    w.total = align_up(w.part_ml + rows * sizeof(float2), kWsAlign);
+    return w;
+}
+
+bool ensure_smem_attr(const void *fn, int bytes, bool *done_per_device) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    if (!done_per_device[dev]) {
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+            cudaSuccess)
+            return false;
+        done_per_device[dev] = true;
+    }
+    return true;
+}
+
 tbq4_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? TBQ4_OK : TBQ4_ERR_LAUNCH;
 }
@@ -77,12 +118,15 @@ tbq4_status run_attention(AttnParams p, void *workspace, size_t ws_bytes,
     p.n_splits = w.n_splits;
     p.part_o = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.part_o);
     p.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) + w.part_ml);
+    static bool attr_set[64] = {};    // the attribute is set once per device
+    if (!ensure_smem_attr((const void *)decode_tc_kernel, kTcSmemBytes, attr_set))
+        return TBQ4_ERR_LAUNCH;
     dim3 g1(p.n_splits, p.Hkv, p.nseq);
     if (g_ev_before) cudaEventRecord(g_ev_before, st);
-    decode_split_kernel<<<g1, kSplitWarps * 32, 0, st>>>(p);
+    decode_tc_kernel<<<g1, kTcWarps * 32, kTcSmemBytes, st>>>(p);
     if (g_ev_after) cudaEventRecord(g_ev_after, st);
     dim3 g2(p.Hq, p.nseq);
-    decode_combine_kernel<<<g2, kD, 0, st>>>(p);
+    decode_combine_kernel<<<g2, kCombineWarps * 32, 0, st>>>(p);
     return launch_status();
 }
 
@@ -189,11 +233,8 @@ tbq4_status tbq4_attn_decode(const float *q, const uint8_t *k_cache,
 }
 
 size_t tbq4_prefill_workspace_bytes(int n_new, int Hq, int Hkv, int64_t n_cached) {
-    if (n_new <= 0 || Hq <= 0 || Hkv <= 0 || n_cached < 0) return 0;
-    const int64_t max_len = n_cached + n_new;
-    if (max_len > INT32_MAX) return 0;
-    const int32_t st = auto_split_tokens(n_new, Hkv, (int32_t)max_len);
-    return attn_ws_layout(n_new, Hq, (int32_t)max_len, st).total;
+    if (n_new <= 0 || Hq <= 0 || Hkv <= 0 || n_cached < 0 || Hq % Hkv != 0) return 0;
+    return prefill_ws_layout(n_new, Hq, Hkv, n_cached).total;
 }
 
 tbq4_status tbq4_attn_prefill_chunk(const uint16_t *q, int n_new, int64_t n_cached,
@@ -213,27 +254,56 @@ tbq4_status tbq4_attn_prefill_chunk(const uint16_t *q, int n_new, int64_t n_cach
         n_cached + n_new > INT32_MAX)
         return TBQ4_ERR_CAPACITY;
     if (!std::isfinite(softmax_scale)) return TBQ4_ERR_SHAPE;
-    AttnParams p = {};
-    p.q = q;
-    p.q_bf16 = 1;
-    p.k = k_cache;
-    p.v = v_cache;
-    p.head_stride = capacity * kBlockBytes;
-    p.seq_stride = 0;                          // every query row reads the same cache
-    p.seq_lens = nullptr;
-    p.len_base = (int32_t)(n_cached + 1);      // row i sees keys 0 .. n_cached + i
-    p.max_len = (int32_t)(n_cached + n_new);
-    p.capacity = capacity;
-    p.nseq = n_new;
-    p.Hq = Hq;
-    p.Hkv = Hkv;
-    p.G = Hq / Hkv;
-    p.split_tokens = auto_split_tokens(n_new, Hkv, p.max_len);
-    p.scale_log2 = softmax_scale * 1.4426950408889634f;
-    sign_words(sign_seed, &p.sign_lo, &p.sign_hi);
-    p.out = out;
-    p.out_bf16 = 1;
-    return run_attention(p, workspace, ws_bytes, (cudaStream_t)stream);
+    const PrefillPlan w = prefill_ws_layout(n_new, Hq, Hkv, n_cached);
+    if (ws_bytes < w.total) return TBQ4_ERR_WORKSPACE;
+    static bool attr_set[64] = {};
+    if (!ensure_smem_attr((const void *)pre::prefill_tc_kernel, pre::kSmemBytes, attr_set))
+        return TBQ4_ERR_LAUNCH;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint64_t lo, hi;
+    sign_words(sign_seed, &lo, &hi);
+    pre::PrefillParams pp = {};
+    pp.q = q;
+    pp.k = k_cache;
+    pp.v = v_cache;
+    pp.head_stride = capacity * kBlockBytes;
+    pp.n_new = n_new;
+    pp.n_cached = n_cached;
+    pp.Hq = Hq;
+    pp.Hkv = Hkv;
+    pp.G = Hq / Hkv;
+    pp.pairs = w.pairs;
+    pp.iblocks = w.iblocks;
+    pp.n_splits = w.n_splits;
+    pp.scale_log2_15 = softmax_scale * 1.4426950408889634f / 15.0f;
+    pp.sign_lo = lo;
+    pp.sign_hi = hi;
+    pp.part_o = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.part_o);
+    pp.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) + w.part_ml);
+    if (g_ev_before) cudaEventRecord(g_ev_before, st);
+    pre::prefill_tc_kernel<<<dim3(w.n_splits, w.mpairs), pre::kThreads, pre::kSmemBytes, st>>>(pp);
+    if (g_ev_after) cudaEventRecord(g_ev_after, st);
+
+    AttnParams c = {};
+    c.seq_lens = nullptr;
+    c.len_base = (int32_t)(n_cached + 1);
+    c.max_len = (int32_t)(n_cached + n_new);
+    c.capacity = capacity;
+    c.nseq = n_new;
+    c.Hq = Hq;
+    c.Hkv = Hkv;
+    c.G = Hq / Hkv;
+    c.split_tokens = 1;
+    c.n_splits = w.n_splits;
+    c.all_splits = 1;
+    c.sign_lo = lo;
+    c.sign_hi = hi;
+    c.part_o = pp.part_o;
+    c.part_ml = pp.part_ml;
+    c.out = out;
+    c.out_bf16 = 1;
+    decode_combine_kernel<<<dim3(Hq, n_new), kCombineWarps * 32, 0, st>>>(c);
+    return launch_status();
 }
 
 void tbq4_set_timing_events(void *before, void *after) {
