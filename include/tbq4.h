@@ -140,6 +140,39 @@ TBQ4_API tbq4_status tbq4_attn_decode_split(const float *q, const uint8_t *k_cac
                                    void *stream);
 
 /*
+ * Decode attention for callers that cannot allocate device memory.  It
+ * computes exactly what tbq4_attn_decode computes, with the same arguments
+ * minus the workspace.  The scratch for the split partials is a fixed array
+ * of 8 MiB (8,388,608 bytes) compiled into this library as a static device
+ * variable, so every GPU that loads the library holds those 8 MiB until the
+ * process exits.
+ *
+ * Who needs it: code that is handed its inputs and outputs but has no way
+ * to obtain device memory where it calls attention, such as a plugin that
+ * runs inside another framework that owns all device memory, or a serving
+ * loop whose memory is fixed before it starts.  The source pages describe
+ * no counterpart of this entry point.
+ *
+ *   - If the scratch the call needs, tbq4_decode_workspace_bytes(B, Hq,
+ *     Hkv, max_len), exceeds 8 MiB, it returns TBQ4_ERR_WORKSPACE and
+ *     launches nothing.
+ *   - The first call on a device looks up the device address of the array
+ *     (cudaGetSymbolAddress, with that device current) and keeps it; make
+ *     that first call before any stream capture.
+ *   - All calls share the one array, which keeps what the previous call
+ *     wrote.  Nothing in it needs clearing (each partial is written before
+ *     it is read), but calls whose kernels overlap on the GPU, for example
+ *     on two streams at once, race on it: serialise them.
+ *   - It allocates and frees nothing.
+ */
+TBQ4_API tbq4_status tbq4_attn_decode_noalloc(const float *q, const uint8_t *k_cache,
+                                              const uint8_t *v_cache,
+                                              const int32_t *seq_lens, int32_t max_len,
+                                              int B, int Hq, int Hkv, int64_t capacity,
+                                              float softmax_scale, uint64_t sign_seed,
+                                              uint16_t *out, void *stream);
+
+/*
  * Chunked prefill attention for one sequence: n_new query tokens at
  * absolute positions n_cached .. n_cached+n_new-1, each attending causally
  * to keys 0 .. its own position, over TBQ4 caches that already hold the

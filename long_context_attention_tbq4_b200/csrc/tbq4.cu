@@ -13,6 +13,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 
 namespace {
 
@@ -130,6 +131,29 @@ tbq4_status run_attention(AttnParams p, void *workspace, size_t ws_bytes,
     return launch_status();
 }
 
+// Scratch of tbq4_attn_decode_noalloc: a fixed array in this library, for
+// callers that cannot allocate.  Host code only ever passes its device
+// address, looked up once per device (the host-side name is not an address
+// the GPU can use).
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+tbq4_status noalloc_scratch(void **ptr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TBQ4_ERR_LAUNCH;
+    static void *addr[64] = {};
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return TBQ4_ERR_LAUNCH;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    return TBQ4_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -230,6 +254,21 @@ tbq4_status tbq4_attn_decode(const float *q, const uint8_t *k_cache,
     return tbq4_attn_decode_split(q, k_cache, v_cache, seq_lens, max_len, B, Hq, Hkv,
                                   capacity, softmax_scale, sign_seed, 0, workspace,
                                   ws_bytes, out, stream);
+}
+
+tbq4_status tbq4_attn_decode_noalloc(const float *q, const uint8_t *k_cache,
+                                     const uint8_t *v_cache, const int32_t *seq_lens,
+                                     int32_t max_len, int B, int Hq, int Hkv, int64_t capacity,
+                                     float softmax_scale, uint64_t sign_seed, uint16_t *out,
+                                     void *stream) {
+    const size_t need = tbq4_decode_workspace_bytes(B, Hq, Hkv, max_len);
+    if (need > kNoAllocScratchBytes) return TBQ4_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    const tbq4_status st = noalloc_scratch(&scratch);
+    if (st != TBQ4_OK) return st;
+    return tbq4_attn_decode(q, k_cache, v_cache, seq_lens, max_len, B, Hq, Hkv, capacity,
+                            softmax_scale, sign_seed, scratch, kNoAllocScratchBytes, out,
+                            stream);
 }
 
 size_t tbq4_prefill_workspace_bytes(int n_new, int Hq, int Hkv, int64_t n_cached) {
