@@ -68,10 +68,18 @@ def measured_peaks():
             "source": "fallback"}
 
 
-def kernel_source_hash():
+# Source files each profiled kernel is built from: a recorded ncu traffic
+# figure is only reported while these files are unchanged.
+KERNEL_SOURCES = {
+    "decode_tc_kernel": ["common.cuh", "decode.cuh", "decode_tc.cuh"],
+    "prefill_tc_kernel": ["common.cuh", "decode.cuh", "tcgen05.cuh", "prefill_tc.cuh"],
+}
+
+
+def kernel_source_hash(kernel):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "long_context_attention_tbq4_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         h.update(name.encode())
         h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()[:16]
@@ -79,12 +87,12 @@ def kernel_source_hash():
 
 def recorded_traffic(kernel):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+    the kernel's current sources (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     rec = json.load(open(path)).get(kernel)
-    if not rec or rec.get("source_sha256") != kernel_source_hash():
+    if not rec or rec.get("source_sha256") != kernel_source_hash(kernel):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -487,7 +495,7 @@ def main():
     e2e_ms = max_over_ranks(torch, float(np.mean(dec["e2e_ms"])))
     kern_ms = float(np.mean(dec["kern_ms"]))
     achieved = kernel_bytes / (kern_ms * 1e-3) / 1e9
-    traffic = recorded_traffic("decode_split_kernel")
+    traffic = recorded_traffic("decode_tc_kernel")
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -499,7 +507,7 @@ def main():
                    "parallelism": "replicas" if world > 1 else "single"},
         "step_bytes": step_bytes,
         "pct_hbm_peak": value / world / peaks["hbm_gbs"],
-        "roofline": {"kernel": "decode_split_kernel", "bound": "hbm", "achieved": achieved,
+        "roofline": {"kernel": "decode_tc_kernel", "bound": "hbm", "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                      "algorithmic_bytes": kernel_bytes, "kernel_ms": kern_ms,
