@@ -396,20 +396,32 @@ prefill_tc_kernel(const PrefillParams p) {
             const float *sv = sig + (sr * 2 + 1) * kTile;
             const int64_t kt = (int64_t)(tile_begin + j) * kTile;
             const bool diag = kt + kTile - 1 > p.n_cached + i0;
-            // pass 1: row max of the masked log2 logits
-            float mx = -INFINITY;
+            // Causal mask only on tiles that reach past the block's first row:
+            // column col is masked when kt + col > lim, i.e. col > rel.
+            const int rel = diag ? (int)(lim - kt) : kTile;
+            // pass 1: row max of the log2 logits, two 32-column loads per wait
+            // and four independent max chains
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
-            for (int ch = 0; ch < 4; ++ch) {
-                float v[32];
-                tc::tmem_ld32(t_s + 32 * ch, v);
+            for (int ch = 0; ch < 4; ch += 2) {
+                float v0[32], v1[32];
+                tc::tmem_ld32(t_s + 32 * ch, v0);
+                tc::tmem_ld32(t_s + 32 * ch + 32, v1);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    float z = v[e] * sk[32 * ch + e];
-                    if (diag && kt + 32 * ch + e > lim) z = -INFINITY;
-                    mx = fmaxf(mx, z);
+                for (int e = 0; e < 64; e += 2) {
+                    const float2 skv = *reinterpret_cast<const float2 *>(sk + 32 * ch + e);
+                    const float2 sv2 = e < 32 ? make_float2(v0[e], v0[e + 1])
+                                              : make_float2(v1[e - 32], v1[e - 31]);
+                    float2 z = __fmul2_rn(sv2, skv);
+                    if (diag) {
+                        if (32 * ch + e > rel) z.x = -INFINITY;
+                        if (32 * ch + e + 1 > rel) z.y = -INFINITY;
+                    }
+                    mx4[(e >> 1) & 3] = fmaxf(mx4[(e >> 1) & 3], fmaxf(z.x, z.y));
                 }
             }
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
             const float m_new = fmaxf(m, mx);
             const bool need = (m == -INFINITY && m_new != -INFINITY) || m_new > m + kRescaleThreshold;
             if (__any_sync(kFull, need)) {
@@ -432,7 +444,10 @@ prefill_tc_kernel(const PrefillParams p) {
                 m = m_new;
             }
             const float m_use = (m == -INFINITY) ? 0.f : m;
-            // pass 2: P' = exp2(z - m) * S_v / 15 as bf16 over S's first 64 columns
+            const float2 negm = make_float2(-m_use, -m_use);
+            // pass 2: P' = exp2(z - m) * S_v / 15 as bf16 over S's first 64
+            // columns (each 32-column chunk of P lands on S columns already read)
+            float2 lacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll 1
             for (int ch = 0; ch < 4; ++ch) {
                 float v[32];
@@ -441,17 +456,23 @@ prefill_tc_kernel(const PrefillParams p) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    float z0 = v[e] * sk[32 * ch + e], z1 = v[e + 1] * sk[32 * ch + e + 1];
-                    if (diag && kt + 32 * ch + e > lim) z0 = -INFINITY;
-                    if (diag && kt + 32 * ch + e + 1 > lim) z1 = -INFINITY;
-                    const float p0 = tc::ex2(z0 - m_use), p1 = tc::ex2(z1 - m_use);
-                    l += p0 + p1;
-                    __nv_bfloat162 b = __floats2bfloat162_rn(p0 * sv[32 * ch + e],
-                                                             p1 * sv[32 * ch + e + 1]);
+                    const int col = 32 * ch + e;
+                    const float2 skv = *reinterpret_cast<const float2 *>(sk + col);
+                    const float2 svv = *reinterpret_cast<const float2 *>(sv + col);
+                    float2 z = __fadd2_rn(__fmul2_rn(make_float2(v[e], v[e + 1]), skv), negm);
+                    if (diag) {
+                        if (col > rel) z.x = -INFINITY;
+                        if (col + 1 > rel) z.y = -INFINITY;
+                    }
+                    const float2 pr = make_float2(tc::ex2(z.x), tc::ex2(z.y));
+                    lacc[(e >> 1) & 1] = __fadd2_rn(lacc[(e >> 1) & 1], pr);
+                    const float2 pw = __fmul2_rn(pr, svv);
+                    __nv_bfloat162 b = __floats2bfloat162_rn(pw.x, pw.y);
                     pk[e >> 1] = *reinterpret_cast<uint32_t *>(&b);
                 }
                 tc::tmem_st16(t_s + 16 * ch, pk);
             }
+            l += (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y);
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
