@@ -399,6 +399,50 @@ prefill_tc_kernel(const PrefillParams p) {
             // Causal mask only on tiles that reach past the block's first row:
             // column col is masked when kt + col > lim, i.e. col > rel.
             const int rel = diag ? (int)(lim - kt) : kTile;
+            // Fast path (every row of the warp already has a finite running
+            // max): one pass with the stale max m, P held in registers.  It is
+            // kept only if no logit exceeds m by more than the threshold (so
+            // every P <= 2^8); otherwise the two-pass path below recomputes the
+            // tile from S, which is still intact in tensor memory.
+            bool done = false;
+            if (!__any_sync(kFull, m == -INFINITY)) {
+                const float2 negm = make_float2(-m, -m);
+                uint32_t pk[64];
+                float dmx[2] = {-INFINITY, -INFINITY};
+                float2 lf[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    float v[16];
+                    tc::tmem_ld16(t_s + 16 * ch, v);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; e += 2) {
+                        const int col = 16 * ch + e;
+                        const float2 skv = *reinterpret_cast<const float2 *>(sk + col);
+                        const float2 svv = *reinterpret_cast<const float2 *>(sv + col);
+                        float2 d = __ffma2_rn(make_float2(v[e], v[e + 1]), skv, negm);
+                        if (diag) {
+                            if (col > rel) d.x = -INFINITY;
+                            if (col + 1 > rel) d.y = -INFINITY;
+                        }
+                        dmx[(e >> 1) & 1] = fmaxf(dmx[(e >> 1) & 1], fmaxf(d.x, d.y));
+                        const float2 pr = make_float2(tc::ex2(d.x), tc::ex2(d.y));
+                        lf[(e >> 1) & 1] = __fadd2_rn(lf[(e >> 1) & 1], pr);
+                        const float2 pw = __fmul2_rn(pr, svv);
+                        __nv_bfloat162 b = __floats2bfloat162_rn(pw.x, pw.y);
+                        pk[col >> 1] = *reinterpret_cast<uint32_t *>(&b);
+                    }
+                }
+                if (!__any_sync(kFull, fmaxf(dmx[0], dmx[1]) > kRescaleThreshold)) {
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch)
+                        tc::tmem_st16(t_s + 16 * ch,
+                                      *reinterpret_cast<const uint32_t(*)[16]>(pk + 16 * ch));
+                    l += (lf[0].x + lf[0].y) + (lf[1].x + lf[1].y);
+                    done = true;
+                }
+            }
+            if (!done) {
             // pass 1: row max of the log2 logits, two 32-column loads per wait
             // and four independent max chains
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -473,6 +517,7 @@ prefill_tc_kernel(const PrefillParams p) {
                 tc::tmem_st16(t_s + 16 * ch, pk);
             }
             l += (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y);
+            }   // two-pass path
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
