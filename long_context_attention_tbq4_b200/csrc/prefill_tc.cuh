@@ -12,10 +12,11 @@
 //   warp 0      producer: cp.async.bulk of raw K and V blocks (128 tokens,
 //               8,448 bytes each) into a 2-stage raw ring
 //   warp 1      tensor-memory allocation; lane 0 issues every tcgen05.mma
-//   warps 4-7   dequantisation: raw nibbles -> exact bf16 levels 2n-15 in a
-//               3-slot ring of 32 KB operand tiles (K tile: keys x dims, V^T
-//               tile: dims x keys, both K-major with the 128-byte swizzle),
-//               plus the per-token factors S_k * c and S_v / 15
+//   warps 4-7   dequantisation: raw nibbles -> bf16 operand tiles in a
+//               3-slot ring of 32 KB (K tile: keys x dims, exact levels
+//               2n-15; V^T tile: dims x keys, (2n-15) S_v/15 rounded once;
+//               both K-major with the 128-byte swizzle), plus the per-token
+//               factor S_k * scale * log2(e) / 15 for the softmax
 //   warps 8-11  softmax of M-tile 0 (thread = query row = TMEM lane)
 //   warps 12-15 softmax of M-tile 1
 // Tensor memory (512 columns): M-tile a has S at [256a, 256a+128) (P, bf16,
@@ -42,6 +43,7 @@ constexpr int kSlots = 3;
 constexpr int kOpBytes = kTile * kD * 2;                // 32 KB bf16 operand tile
 constexpr int kSigRing = 4;
 constexpr float kRescaleThreshold = 8.0f;               // log2 units
+constexpr float kFastSumLimit = 256.0f;                 // 2^kRescaleThreshold
 constexpr uint32_t kSpin = 1u << 22;
 
 // shared-memory layout (offsets from a 1024-aligned base)
@@ -63,12 +65,28 @@ constexpr uint32_t kIdesc = tc::idesc_bf16(128, 128);
 constexpr uint32_t kB2Two = 0x40004000u;
 constexpr uint32_t kB2Neg143 = 0xC30FC30Fu;
 constexpr uint32_t kB2Magic64 = 0x42804280u;
+// {128 + n} from a nibble in mantissa bits 0-3, and {-136}: 128 + n - 136 = n - 8.
+constexpr uint32_t kB2Magic128 = 0x43004300u;
+constexpr uint32_t kB2Neg136 = 0xC308C308u;
 
 __device__ __forceinline__ uint32_t bfma2(uint32_t x, uint32_t m, uint32_t a) {
     __nv_bfloat162 r = __hfma2(*reinterpret_cast<__nv_bfloat162 *>(&x),
                                *reinterpret_cast<__nv_bfloat162 *>(&m),
                                *reinterpret_cast<__nv_bfloat162 *>(&a));
     return *reinterpret_cast<uint32_t *>(&r);
+}
+
+__device__ __forceinline__ uint32_t badd2(uint32_t x, uint32_t a) {
+    __nv_bfloat162 r = __hadd2(*reinterpret_cast<__nv_bfloat162 *>(&x),
+                               *reinterpret_cast<__nv_bfloat162 *>(&a));
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
+// V level times the token's factor S_v/15, in one rounding: with n - 8
+// exact, (n - 8) * 2 s + s = (2n - 15) s.  v holds nibbles in bits 0-3 and
+// 16-19; s2 = {2 s_a, 2 s_b}, s1 = {s_a, s_b}.
+__device__ __forceinline__ uint32_t v_scaled(uint32_t v, uint32_t s2, uint32_t s1) {
+    return bfma2(badd2((v & 0x000F000Fu) | kB2Magic128, kB2Neg136), s2, s1);
 }
 
 // Nibbles at bit offset `sh` of both 16-bit halves of v -> bf16 64+n.
@@ -214,8 +232,8 @@ prefill_tc_kernel(const PrefillParams p) {
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_ptr;
     const int64_t head_off = (int64_t)g * p.head_stride;
-
-    if (warp == 0) {
+    if (warp < 4) {
+      if (warp == 0) {
         // ======================= producer ====================================
         if (lane == 0) {
             for (int j = 0; j < n_tiles; ++j) {
@@ -236,7 +254,7 @@ prefill_tc_kernel(const PrefillParams p) {
                              raw_full(st));
             }
         }
-    } else if (warp == 1) {
+      } else if (warp == 1) {
         // ======================= MMA issuer ==================================
         if (lane == 0 && n_tiles > 0) {
             bool ok = true;
@@ -292,7 +310,8 @@ prefill_tc_kernel(const PrefillParams p) {
                 }
             }
         }
-    } else if (warp >= 4 && warp < 8) {
+      }
+    } else if (warp < 8) {
         // ======================= dequantisation ==============================
         const int t = threadIdx.x - 128;              // 0..127
         for (int j = 0; j < n_tiles; ++j) {
@@ -307,9 +326,7 @@ prefill_tc_kernel(const PrefillParams p) {
             {
                 const bool in = t0 + t < keys_total;
                 const float sk = __half2float(__ushort_as_half(lds16(raw + t * kBlockBytes)));
-                const float sv = __half2float(__ushort_as_half(lds16(raw + kRawBytes + t * kBlockBytes)));
                 sig[(sr * 2 + 0) * kTile + t] = in ? sk * p.scale_log2_15 : 0.f;
-                sig[(sr * 2 + 1) * kTile + t] = in ? sv * (1.0f / 15.0f) : 0.f;
             }
             __syncwarp();
             if (lane == 0) tc::bar_arrive(sig_full(sr));
@@ -351,6 +368,16 @@ prefill_tc_kernel(const PrefillParams p) {
                 const int ta = 2 * pp;
                 const uint32_t srca = raw + kRawBytes + ta * kBlockBytes + 2 + 32 * hf;
                 const uint32_t srcb = srca + kBlockBytes;
+                // S_v / 15 of the two tokens; 0 past the cache end, where the
+                // raw bytes are stale (their P is 0, and 0 * level must not be NaN)
+                const float sva = t0 + ta < keys_total
+                    ? __half2float(__ushort_as_half(lds16(srca - 2 - 32 * hf))) * (1.0f / 15.0f) : 0.f;
+                const float svb = t0 + ta + 1 < keys_total
+                    ? __half2float(__ushort_as_half(lds16(srcb - 2 - 32 * hf))) * (1.0f / 15.0f) : 0.f;
+                __nv_bfloat162 s1b = __floats2bfloat162_rn(sva, svb);
+                __nv_bfloat162 s2b = __hmul2(s1b, __floats2bfloat162_rn(2.f, 2.f));
+                const uint32_t s1 = *reinterpret_cast<uint32_t *>(&s1b);
+                const uint32_t s2 = *reinterpret_cast<uint32_t *>(&s2b);
 #pragma unroll 2
                 for (int w = 0; w < 8; ++w) {
                     const uint32_t wa = funnel_word(srca + 4 * w), wb = funnel_word(srcb + 4 * w);
@@ -359,10 +386,10 @@ prefill_tc_kernel(const PrefillParams p) {
                     for (int half = 0; half < 2; ++half) {
                         const uint32_t X = __byte_perm(wa, wb, half ? 0x7632 : 0x5410);
                         const int d = d0 + 4 * half;
-                        sts32(dst + sw128_off(d + 0, ta), bfma2(nib_pair(X, -1), kB2Two, kB2Neg143));
-                        sts32(dst + sw128_off(d + 1, ta), bfma2(nib_pair(X, 3), kB2Two, kB2Neg143));
-                        sts32(dst + sw128_off(d + 2, ta), bfma2(nib_pair(X, 7), kB2Two, kB2Neg143));
-                        sts32(dst + sw128_off(d + 3, ta), bfma2(nib_pair(X, 11), kB2Two, kB2Neg143));
+                        sts32(dst + sw128_off(d + 0, ta), v_scaled(X, s2, s1));
+                        sts32(dst + sw128_off(d + 1, ta), v_scaled(X >> 4, s2, s1));
+                        sts32(dst + sw128_off(d + 2, ta), v_scaled(X >> 8, s2, s1));
+                        sts32(dst + sw128_off(d + 3, ta), v_scaled(X >> 12, s2, s1));
                     }
                 }
                 tc::fence_proxy_async();
@@ -372,7 +399,7 @@ prefill_tc_kernel(const PrefillParams p) {
             __syncwarp();
             if (lane == 0) tc::bar_arrive(raw_empty(st));
         }
-    } else if (warp >= 8) {
+    } else {
         // ======================= softmax =====================================
         const int a = (warp - 8) >> 2;
         const int row = 32 * (warp & 3) + lane;           // TMEM lane = query row
@@ -393,7 +420,6 @@ prefill_tc_kernel(const PrefillParams p) {
             }
             tc::fence_after_sync();
             const float *sk = sig + (sr * 2 + 0) * kTile;
-            const float *sv = sig + (sr * 2 + 1) * kTile;
             const int64_t kt = (int64_t)(tile_begin + j) * kTile;
             const bool diag = kt + kTile - 1 > p.n_cached + i0;
             // Causal mask only on tiles that reach past the block's first row:
@@ -401,14 +427,13 @@ prefill_tc_kernel(const PrefillParams p) {
             const int rel = diag ? (int)(lim - kt) : kTile;
             // Fast path (every row of the warp already has a finite running
             // max): one pass with the stale max m, P held in registers.  It is
-            // kept only if no logit exceeds m by more than the threshold (so
-            // every P <= 2^8); otherwise the two-pass path below recomputes the
-            // tile from S, which is still intact in tensor memory.
+            // kept if each row's sum of P over the tile stays <= 2^8, which
+            // bounds every P by 2^8; otherwise the two-pass path below
+            // recomputes the tile from S, still intact in tensor memory.
             bool done = false;
             if (!__any_sync(kFull, m == -INFINITY)) {
                 const float2 negm = make_float2(-m, -m);
                 uint32_t pk[64];
-                float dmx[2] = {-INFINITY, -INFINITY};
                 float2 lf[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
@@ -419,45 +444,39 @@ prefill_tc_kernel(const PrefillParams p) {
                     for (int e = 0; e < 16; e += 2) {
                         const int col = 16 * ch + e;
                         const float2 skv = *reinterpret_cast<const float2 *>(sk + col);
-                        const float2 svv = *reinterpret_cast<const float2 *>(sv + col);
                         float2 d = __ffma2_rn(make_float2(v[e], v[e + 1]), skv, negm);
                         if (diag) {
                             if (col > rel) d.x = -INFINITY;
                             if (col + 1 > rel) d.y = -INFINITY;
                         }
-                        dmx[(e >> 1) & 1] = fmaxf(dmx[(e >> 1) & 1], fmaxf(d.x, d.y));
                         const float2 pr = make_float2(tc::ex2(d.x), tc::ex2(d.y));
                         lf[(e >> 1) & 1] = __fadd2_rn(lf[(e >> 1) & 1], pr);
-                        const float2 pw = __fmul2_rn(pr, svv);
-                        __nv_bfloat162 b = __floats2bfloat162_rn(pw.x, pw.y);
+                        __nv_bfloat162 b = __floats2bfloat162_rn(pr.x, pr.y);
                         pk[col >> 1] = *reinterpret_cast<uint32_t *>(&b);
                     }
                 }
-                if (!__any_sync(kFull, fmaxf(dmx[0], dmx[1]) > kRescaleThreshold)) {
+                const float lt = (lf[0].x + lf[0].y) + (lf[1].x + lf[1].y);
+                if (!__any_sync(kFull, !(lt <= kFastSumLimit))) {
 #pragma unroll
                     for (int ch = 0; ch < 4; ++ch)
                         tc::tmem_st16(t_s + 16 * ch,
                                       *reinterpret_cast<const uint32_t(*)[16]>(pk + 16 * ch));
-                    l += (lf[0].x + lf[0].y) + (lf[1].x + lf[1].y);
+                    l += lt;
                     done = true;
                 }
             }
             if (!done) {
-            // pass 1: row max of the log2 logits, two 32-column loads per wait
-            // and four independent max chains
+            // pass 1: row max of the log2 logits, four independent max chains
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
-            for (int ch = 0; ch < 4; ch += 2) {
-                float v0[32], v1[32];
+            for (int ch = 0; ch < 4; ++ch) {
+                float v0[32];
                 tc::tmem_ld32(t_s + 32 * ch, v0);
-                tc::tmem_ld32(t_s + 32 * ch + 32, v1);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 64; e += 2) {
+                for (int e = 0; e < 32; e += 2) {
                     const float2 skv = *reinterpret_cast<const float2 *>(sk + 32 * ch + e);
-                    const float2 sv2 = e < 32 ? make_float2(v0[e], v0[e + 1])
-                                              : make_float2(v1[e - 32], v1[e - 31]);
-                    float2 z = __fmul2_rn(sv2, skv);
+                    float2 z = __fmul2_rn(make_float2(v0[e], v0[e + 1]), skv);
                     if (diag) {
                         if (32 * ch + e > rel) z.x = -INFINITY;
                         if (32 * ch + e + 1 > rel) z.y = -INFINITY;
@@ -489,7 +508,7 @@ prefill_tc_kernel(const PrefillParams p) {
             }
             const float m_use = (m == -INFINITY) ? 0.f : m;
             const float2 negm = make_float2(-m_use, -m_use);
-            // pass 2: P' = exp2(z - m) * S_v / 15 as bf16 over S's first 64
+            // pass 2: P = exp2(z - m) as bf16 over S's first 64
             // columns (each 32-column chunk of P lands on S columns already read)
             float2 lacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll 1
@@ -502,16 +521,14 @@ prefill_tc_kernel(const PrefillParams p) {
                 for (int e = 0; e < 32; e += 2) {
                     const int col = 32 * ch + e;
                     const float2 skv = *reinterpret_cast<const float2 *>(sk + col);
-                    const float2 svv = *reinterpret_cast<const float2 *>(sv + col);
-                    float2 z = __fadd2_rn(__fmul2_rn(make_float2(v[e], v[e + 1]), skv), negm);
+                    float2 z = __ffma2_rn(make_float2(v[e], v[e + 1]), skv, negm);
                     if (diag) {
                         if (col > rel) z.x = -INFINITY;
                         if (col + 1 > rel) z.y = -INFINITY;
                     }
                     const float2 pr = make_float2(tc::ex2(z.x), tc::ex2(z.y));
                     lacc[(e >> 1) & 1] = __fadd2_rn(lacc[(e >> 1) & 1], pr);
-                    const float2 pw = __fmul2_rn(pr, svv);
-                    __nv_bfloat162 b = __floats2bfloat162_rn(pw.x, pw.y);
+                    __nv_bfloat162 b = __floats2bfloat162_rn(pr.x, pr.y);
                     pk[e >> 1] = *reinterpret_cast<uint32_t *>(&b);
                 }
                 tc::tmem_st16(t_s + 16 * ch, pk);
