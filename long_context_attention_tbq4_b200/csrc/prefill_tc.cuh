@@ -436,13 +436,13 @@ prefill_tc_kernel(const PrefillParams p) {
                 uint32_t pk[64];
                 float2 lf[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    float v[16];
-                    tc::tmem_ld16(t_s + 16 * ch, v);
+                for (int ch = 0; ch < 4; ++ch) {
+                    float v[32];
+                    tc::tmem_ld32(t_s + 32 * ch, v);
                     tc::tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; e += 2) {
-                        const int col = 16 * ch + e;
+                    for (int e = 0; e < 32; e += 2) {
+                        const int col = 32 * ch + e;
                         const float2 skv = *reinterpret_cast<const float2 *>(sk + col);
                         float2 d = __ffma2_rn(make_float2(v[e], v[e + 1]), skv, negm);
                         if (diag) {
