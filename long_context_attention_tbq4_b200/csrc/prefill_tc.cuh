@@ -45,6 +45,15 @@ constexpr int kSigRing = 4;
 constexpr float kRescaleThreshold = 8.0f;               // log2 units
 constexpr float kFastSumLimit = 256.0f;                 // 2^kRescaleThreshold
 constexpr uint32_t kSpin = 1u << 22;
+// Registers per thread after the prologue, per warpgroup: producer/MMA,
+// dequantisation, and each softmax warpgroup (which holds a full S row of 128
+// floats).  Their sum x 128 threads must fit in what the CTA was launched
+// with, 512 threads x the compiled count; the host refuses to launch if the
+// compiled count is below kMinLaunchRegs.
+constexpr uint32_t kRegsCtl = 40, kRegsDeq = 88, kRegsSoft = 192;
+constexpr int kMinLaunchRegs = 128;
+static_assert((kRegsCtl + kRegsDeq + 2 * kRegsSoft) * 128 <= kMinLaunchRegs * kThreads,
+              "register split exceeds the launch budget");
 
 // shared-memory layout (offsets from a 1024-aligned base)
 constexpr int kOffQ = 0;                                        // 2 x 32 KB
@@ -233,6 +242,7 @@ prefill_tc_kernel(const PrefillParams p) {
     const uint32_t tmem = *tmem_ptr;
     const int64_t head_off = (int64_t)g * p.head_stride;
     if (warp < 4) {
+      tc::regs_dec<kRegsCtl>();
       if (warp == 0) {
         // ======================= producer ====================================
         if (lane == 0) {
@@ -312,6 +322,7 @@ prefill_tc_kernel(const PrefillParams p) {
         }
       }
     } else if (warp < 8) {
+        tc::regs_dec<kRegsDeq>();
         // ======================= dequantisation ==============================
         const int t = threadIdx.x - 128;              // 0..127
         for (int j = 0; j < n_tiles; ++j) {
@@ -400,6 +411,7 @@ prefill_tc_kernel(const PrefillParams p) {
             if (lane == 0) tc::bar_arrive(raw_empty(st));
         }
     } else {
+        tc::regs_inc<kRegsSoft>();
         // ======================= softmax =====================================
         const int a = (warp - 8) >> 2;
         const int row = 32 * (warp & 3) + lane;           // TMEM lane = query row
@@ -425,116 +437,110 @@ prefill_tc_kernel(const PrefillParams p) {
             // Causal mask only on tiles that reach past the block's first row:
             // column col is masked when kt + col > lim, i.e. col > rel.
             const int rel = diag ? (int)(lim - kt) : kTile;
-            // Fast path (every row of the warp already has a finite running
-            // max): one pass with the stale max m, P held in registers.  It is
-            // kept if each row's sum of P over the tile stays <= 2^8, which
-            // bounds every P by 2^8; otherwise the two-pass path below
-            // recomputes the tile from S, still intact in tensor memory.
+            // The whole S row of this thread goes to registers with one wait;
+            // from then on P may overwrite S in tensor memory.
+            float sr_[kTile];
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch)
+                tc::tmem_ld32(t_s + 32 * ch, *reinterpret_cast<float(*)[32]>(sr_ + 32 * ch));
+            tc::tmem_wait_ld();
+            // Fast path (every row of the warp has a finite running max): P =
+            // exp2(S*sk - m) with the stale m, kept if each row's sum of P over
+            // the tile stays <= 2^8 (which bounds every P by 2^8).
             bool done = false;
             if (!__any_sync(kFull, m == -INFINITY)) {
                 const float2 negm = make_float2(-m, -m);
-                uint32_t pk[64];
                 float2 lf[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) {
-                    float v[32];
-                    tc::tmem_ld32(t_s + 32 * ch, v);
-                    tc::tmem_wait_ld();
+                    uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
                         const int col = 32 * ch + e;
                         const float2 skv = *reinterpret_cast<const float2 *>(sk + col);
-                        float2 d = __ffma2_rn(make_float2(v[e], v[e + 1]), skv, negm);
+                        float2 d = __ffma2_rn(make_float2(sr_[col], sr_[col + 1]), skv, negm);
                         if (diag) {
                             if (col > rel) d.x = -INFINITY;
                             if (col + 1 > rel) d.y = -INFINITY;
                         }
                         const float2 pr = make_float2(tc::ex2(d.x), tc::ex2(d.y));
                         lf[(e >> 1) & 1] = __fadd2_rn(lf[(e >> 1) & 1], pr);
-                        __nv_bfloat162 b = __floats2bfloat162_rn(pr.x, pr.y);
-                        pk[col >> 1] = *reinterpret_cast<uint32_t *>(&b);
+                        __nv_bfloat162 bb = __floats2bfloat162_rn(pr.x, pr.y);
+                        pk[e >> 1] = *reinterpret_cast<uint32_t *>(&bb);
                     }
+                    tc::tmem_st16(t_s + 16 * ch, pk);
                 }
                 const float lt = (lf[0].x + lf[0].y) + (lf[1].x + lf[1].y);
                 if (!__any_sync(kFull, !(lt <= kFastSumLimit))) {
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch)
-                        tc::tmem_st16(t_s + 16 * ch,
-                                      *reinterpret_cast<const uint32_t(*)[16]>(pk + 16 * ch));
                     l += lt;
                     done = true;
                 }
             }
             if (!done) {
-            // pass 1: row max of the log2 logits, four independent max chains
-            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-            for (int ch = 0; ch < 4; ++ch) {
-                float v0[32];
-                tc::tmem_ld32(t_s + 32 * ch, v0);
-                tc::tmem_wait_ld();
+                // exact row max, O rescale when it grows past the threshold,
+                // then P again from the registers (over whatever the fast path
+                // wrote)
+                float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float2 skv = *reinterpret_cast<const float2 *>(sk + 32 * ch + e);
-                    float2 z = __fmul2_rn(make_float2(v0[e], v0[e + 1]), skv);
+                for (int e = 0; e < kTile; e += 2) {
+                    const float2 skv = *reinterpret_cast<const float2 *>(sk + e);
+                    float2 z = __fmul2_rn(make_float2(sr_[e], sr_[e + 1]), skv);
                     if (diag) {
-                        if (32 * ch + e > rel) z.x = -INFINITY;
-                        if (32 * ch + e + 1 > rel) z.y = -INFINITY;
+                        if (e > rel) z.x = -INFINITY;
+                        if (e + 1 > rel) z.y = -INFINITY;
                     }
                     mx4[(e >> 1) & 3] = fmaxf(mx4[(e >> 1) & 3], fmaxf(z.x, z.y));
                 }
-            }
-            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-            const float m_new = fmaxf(m, mx);
-            const bool need = (m == -INFINITY && m_new != -INFINITY) || m_new > m + kRescaleThreshold;
-            if (__any_sync(kFull, need)) {
-                const float corr = (m == -INFINITY) ? 0.f : tc::ex2(m - m_new);
-                if (j > 0) {
-                    if (!tc::bar_wait_warp(o_done(a), (j - 1) & 1, kSpin)) { record_status(7u); ok = false; break; }
-                    tc::fence_after_sync();
+                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+                const float m_new = fmaxf(m, mx);
+                const bool need =
+                    (m == -INFINITY && m_new != -INFINITY) || m_new > m + kRescaleThreshold;
+                if (__any_sync(kFull, need)) {
+                    const float corr = (m == -INFINITY) ? 0.f : tc::ex2(m - m_new);
+                    if (j > 0) {
+                        if (!tc::bar_wait_warp(o_done(a), (j - 1) & 1, kSpin)) {
+                            record_status(7u);
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after_sync();
 #pragma unroll 1
-                    for (int ch = 0; ch < 4; ++ch) {
-                        float o[32];
-                        tc::tmem_ld32(t_o + 32 * ch, o);
-                        tc::tmem_wait_ld();
+                        for (int ch = 0; ch < 4; ++ch) {
+                            float o[32];
+                            tc::tmem_ld32(t_o + 32 * ch, o);
+                            tc::tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] *= corr;
-                        tc::tmem_st32(t_o + 32 * ch, o);
+                            for (int e = 0; e < 32; ++e) o[e] *= corr;
+                            tc::tmem_st32(t_o + 32 * ch, o);
+                        }
                     }
-                    tc::tmem_wait_st();
+                    l *= corr;
+                    m = m_new;
                 }
-                l *= corr;
-                m = m_new;
-            }
-            const float m_use = (m == -INFINITY) ? 0.f : m;
-            const float2 negm = make_float2(-m_use, -m_use);
-            // pass 2: P = exp2(z - m) as bf16 over S's first 64
-            // columns (each 32-column chunk of P lands on S columns already read)
-            float2 lacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll 1
-            for (int ch = 0; ch < 4; ++ch) {
-                float v[32];
-                tc::tmem_ld32(t_s + 32 * ch, v);
-                tc::tmem_wait_ld();
-                uint32_t pk[16];
+                const float m_use = (m == -INFINITY) ? 0.f : m;
+                const float2 negm = make_float2(-m_use, -m_use);
+                float2 lacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int col = 32 * ch + e;
-                    const float2 skv = *reinterpret_cast<const float2 *>(sk + col);
-                    float2 z = __ffma2_rn(make_float2(v[e], v[e + 1]), skv, negm);
-                    if (diag) {
-                        if (col > rel) z.x = -INFINITY;
-                        if (col + 1 > rel) z.y = -INFINITY;
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const int col = 32 * ch + e;
+                        const float2 skv = *reinterpret_cast<const float2 *>(sk + col);
+                        float2 z = __ffma2_rn(make_float2(sr_[col], sr_[col + 1]), skv, negm);
+                        if (diag) {
+                            if (col > rel) z.x = -INFINITY;
+                            if (col + 1 > rel) z.y = -INFINITY;
+                        }
+                        const float2 pr = make_float2(tc::ex2(z.x), tc::ex2(z.y));
+                        lacc[(e >> 1) & 1] = __fadd2_rn(lacc[(e >> 1) & 1], pr);
+                        __nv_bfloat162 bb = __floats2bfloat162_rn(pr.x, pr.y);
+                        pk[e >> 1] = *reinterpret_cast<uint32_t *>(&bb);
                     }
-                    const float2 pr = make_float2(tc::ex2(z.x), tc::ex2(z.y));
-                    lacc[(e >> 1) & 1] = __fadd2_rn(lacc[(e >> 1) & 1], pr);
-                    __nv_bfloat162 b = __floats2bfloat162_rn(pr.x, pr.y);
-                    pk[e >> 1] = *reinterpret_cast<uint32_t *>(&b);
+                    tc::tmem_st16(t_s + 16 * ch, pk);
                 }
-                tc::tmem_st16(t_s + 16 * ch, pk);
+                l += (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y);
             }
-            l += (lacc[0].x + lacc[0].y) + (lacc[1].x + lacc[1].y);
-            }   // two-pass path
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();

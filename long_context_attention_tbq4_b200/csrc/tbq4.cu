@@ -298,6 +298,15 @@ tbq4_status tbq4_attn_prefill_chunk(const uint16_t *q, int n_new, int64_t n_cach
     static bool attr_set[64] = {};
     if (!ensure_smem_attr((const void *)pre::prefill_tc_kernel, pre::kSmemBytes, attr_set))
         return TBQ4_ERR_LAUNCH;
+    // The kernel moves registers between its warpgroups (setmaxnreg); that is
+    // only safe when it was compiled with at least pre::kMinLaunchRegs.
+    static int regs_ok = -1;
+    if (regs_ok < 0) {
+        cudaFuncAttributes fa;
+        regs_ok = cudaFuncGetAttributes(&fa, pre::prefill_tc_kernel) == cudaSuccess &&
+                  fa.numRegs >= pre::kMinLaunchRegs && fa.numRegs * pre::kThreads <= 65536;
+    }
+    if (!regs_ok) return TBQ4_ERR_LAUNCH;
     cudaStream_t st = (cudaStream_t)stream;
     uint64_t lo, hi;
     sign_words(sign_seed, &lo, &hi);

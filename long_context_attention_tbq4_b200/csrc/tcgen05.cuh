@@ -156,6 +156,19 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ---- register budget per warpgroup ----------------------------------------
+// setmaxnreg: every warp of a warpgroup executes the same one.  Increases
+// draw on the registers the CTA was launched with, so the decreases of the
+// other warpgroups must free enough for them.
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---- UMMA -------------------------------------------------------------------
 // K-major operand tile with 128-byte swizzle: rows of 128 bytes (64 bf16 of
 // K), 8-row groups 1024 bytes apart (stride byte offset).
