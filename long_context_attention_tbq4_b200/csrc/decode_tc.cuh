@@ -41,6 +41,7 @@ constexpr int kTcSmemBytes = kRingBytes + kTcWarps * kTcStages * 8 + 128;
 constexpr uint32_t kSpinLimit = 1u << 22;                  // bounded mbarrier wait
 
 static_assert(kStageBytes % 16 == 0, "stage must keep 16-byte alignment");
+constexpr float kLazyRescale = 8.0f;                       // log2 units
 static_assert(kRingBytes >= kTcWarps * kMaxGroup * kD * 4 + 2 * kTcWarps * kMaxGroup * 4,
               "merge buffers reuse the ring");
 
@@ -101,6 +102,16 @@ __device__ __forceinline__ void imma16832(int (&d)[4], uint32_t a0, uint32_t a1,
         "{%8,%9}, {%0,%1,%2,%3};\n"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D (s32) = A (u8) * B (s8), accumulator starting from zero
+__device__ __forceinline__ void imma16832_z(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                            uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%10,%10,%10};\n"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
 
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
@@ -280,8 +291,6 @@ decode_tc_kernel(const AttnParams p) {
 #pragma unroll
         for (int tile = 0; tile < 2; ++tile) {
             int acc[3][4];
-#pragma unroll
-            for (int pc = 0; pc < 3; ++pc) acc[pc][0] = acc[pc][1] = acc[pc][2] = acc[pc][3] = 0;
             const Funnel f0(kst + (16 * tile + r) * kBlockBytes + 2 + 16 * c);
             const Funnel f1(kst + (16 * tile + r + 8) * kBlockBytes + 2 + 16 * c);
             uint32_t w0[5], w1[5];
@@ -295,8 +304,12 @@ decode_tc_kernel(const AttnParams p) {
                 const uint32_t lo0 = x0 & 0x0F0F0F0Fu, hi0 = (x0 >> 4) & 0x0F0F0F0Fu;
                 const uint32_t lo1 = x1 & 0x0F0F0F0Fu, hi1 = (x1 >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
-                for (int pc = 0; pc < 3; ++pc)
-                    imma16832(acc[pc], lo0, lo1, hi0, hi1, qb[i][pc][0], qb[i][pc][1]);
+                for (int pc = 0; pc < 3; ++pc) {
+                    if (i == 0)
+                        imma16832_z(acc[pc], lo0, lo1, hi0, hi1, qb[i][pc][0], qb[i][pc][1]);
+                    else
+                        imma16832(acc[pc], lo0, lo1, hi0, hi1, qb[i][pc][0], qb[i][pc][1]);
+                }
             }
             // sum_d n_d q_int_d = 65536 acc2 + 256 acc1 + acc0
 #pragma unroll
@@ -335,7 +348,11 @@ decode_tc_kernel(const AttnParams p) {
             mxa = fmaxf(mxa, __shfl_xor_sync(kFull, mxa, msk));
             mxb = fmaxf(mxb, __shfl_xor_sync(kFull, mxb, msk));
         }
-        if (__any_sync(kFull, mxa > m_a || mxb > m_b)) {
+        // The running max is only moved (and the accumulators rescaled)
+        // when some head's chunk max exceeds it by more than 2^8; otherwise
+        // p = exp2(logit - m) <= 2^8, and P' carries a factor 2^-8 so that
+        // fp16 P' = p * S_v * 2^-8 stays <= S_v <= 65504.
+        if (__any_sync(kFull, mxa > m_a + kLazyRescale || mxb > m_b + kLazyRescale)) {
             const float na = fmaxf(m_a, mxa), nb = fmaxf(m_b, mxb);
             const float ca = exp2f(m_a - na), cb = exp2f(m_b - nb);
             m_a = na;
@@ -354,7 +371,8 @@ decode_tc_kernel(const AttnParams p) {
             const float pa = exp2f(lg[u][0] - m_a), pb = exp2f(lg[u][1] - m_b);
             l_a += pa;
             l_b += pb;
-            __half2 h = __floats2half2_rn(pa * sv[u], pb * sv[u]);
+            const float svs = sv[u] * (1.0f / 256.0f);
+            __half2 h = __floats2half2_rn(pa * svs, pb * svs);
             p2[u] = *reinterpret_cast<uint32_t *>(&h);
         }
         // P'^T B fragments: thread (n = r, c) needs head n, tokens
@@ -450,7 +468,7 @@ decode_tc_kernel(const AttnParams p) {
             }
         }
         const int64_t row = ((int64_t)s * p.Hq + g * G + h) * p.n_splits + split;
-        p.part_o[row * kD + d] = O * (1.0f / 15.0f);
+        p.part_o[row * kD + d] = O * (256.0f / 15.0f);     // 2^8 undoes the scale of P-prime
         if (d == 0) p.part_ml[row] = make_float2(M, L);
     }
 }
