@@ -153,7 +153,8 @@ def decode_workload():
     bytes_q = case.B * case.Hq * D * 4
     bytes_out = case.B * case.Hq * D * 2
     bytes_append = 2 * case.Hkv * (D * 4 + BLOCK)          # new token: read fp32, write block
-    return case, N, bytes_kv + bytes_q + bytes_out + bytes_append, bytes_kv + bytes_q
+    # the attention kernel also encodes the new token, so its bytes include the append
+    return case, N, bytes_kv + bytes_q + bytes_out + bytes_append, bytes_kv + bytes_q + bytes_append
 
 
 def prefill_flops(n_cached, n_new, Hq):
@@ -187,7 +188,6 @@ def bench_decode(T, torch, case, N, step_bytes, kernel_bytes, steps, warmup, flu
         del src
     k_new = torch.from_numpy(np.ascontiguousarray(K[N - 1:N])[None]).to(dev)
     v_new = torch.from_numpy(np.ascontiguousarray(V[N - 1:N])[None]).to(dev)
-    pos = torch.tensor([N - 1], dtype=torch.int32, device=dev)
     q = torch.from_numpy(case.q).to(dev)
     lens = torch.tensor([N], dtype=torch.int32, device=dev)
     ws = torch.empty(T.tbq4_decode_workspace_bytes(1, case.Hq, case.Hkv, N), dtype=torch.uint8,
@@ -195,10 +195,11 @@ def bench_decode(T, torch, case, N, step_bytes, kernel_bytes, steps, warmup, flu
     out = torch.empty((1, case.Hq, D), dtype=torch.float16, device=dev)
 
     def step(qq=q, kn=k_new, vn=v_new, o=out):
-        T.tbq4_quantize_append(kn, pos, kc, case.sign_seed)
-        T.tbq4_quantize_append(vn, pos, vc, case.sign_seed)
-        T.tbq4_attn_decode(qq, kc, vc, lens, N, case.softmax_scale, case.sign_seed,
-                           workspace=ws, out=o)
+        # one decode step: the new token's K/V rows are encoded into the caches
+        # at position N-1 by the attention kernel itself
+        T.tbq4_attn_decode_append(qq, kn.view(1, case.Hkv, D), vn.view(1, case.Hkv, D), kc, vc,
+                                  lens, N, case.softmax_scale, case.sign_seed, workspace=ws,
+                                  out=o)
 
     for _ in range(warmup):
         step()
@@ -252,7 +253,7 @@ def bench_decode(T, torch, case, N, step_bytes, kernel_bytes, steps, warmup, flu
     h2d = q_h.numel() * 4 + kn_h.numel() * 4 + vn_h.numel() * 4
     d2h = out_h.numel() * 2
     return {"step_ms": step_ms, "kern_ms": kern_ms, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
-            "launches_per_step": 4, "out": out.float().cpu().numpy()}
+            "launches_per_step": 2, "out": out.float().cpu().numpy()}
 
 
 def bench_prefill(T, torch, steps, warmup, flush):
@@ -312,19 +313,21 @@ def profile_decode(T, torch, case, N, n_steps):
     vc = T.empty_cache(1, case.Hkv, N)
     zero = torch.zeros(1, dtype=torch.int32, device=dev)
     for cache, x in ((kc, case.k[0]), (vc, case.v[0])):
-        src = torch.from_numpy(np.ascontiguousarray(x)[None]).to(dev)
+        src = torch.from_numpy(np.ascontiguousarray(x[:N - 1])[None]).to(dev)
         T.tbq4_quantize_append(src, zero, cache, case.sign_seed)
         del src
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
+    k_new = torch.from_numpy(np.ascontiguousarray(case.k[0][N - 1])[None]).to(dev)
+    v_new = torch.from_numpy(np.ascontiguousarray(case.v[0][N - 1])[None]).to(dev)
     q = torch.from_numpy(case.q).to(dev)
     lens = torch.tensor([N], dtype=torch.int32, device=dev)
     ws = torch.empty(T.tbq4_decode_workspace_bytes(1, case.Hq, case.Hkv, N), dtype=torch.uint8,
                      device=dev)
     out = torch.empty((1, case.Hq, D), dtype=torch.float16, device=dev)
     for _ in range(n_steps):
-        T.tbq4_attn_decode(q, kc, vc, lens, N, case.softmax_scale, case.sign_seed,
-                           workspace=ws, out=out)
+        T.tbq4_attn_decode_append(q, k_new, v_new, kc, vc, lens, N, case.softmax_scale,
+                                  case.sign_seed, workspace=ws, out=out)
     torch.cuda.synchronize()
     assert T.tbq4_get_device_status() == 0
     print("profile: %d decode steps at %d keys" % (n_steps, N))

@@ -124,6 +124,29 @@ TBQ4_API tbq4_status tbq4_attn_decode(const float *q, const uint8_t *k_cache,
                              uint64_t sign_seed, void *workspace,
                              size_t ws_bytes, uint16_t *out, void *stream);
 
+/*
+ * One decode step: append the current token's K and V rows to the caches and
+ * attend, in one attention launch.  The result equals tbq4_quantize_append of
+ * k_new / v_new at position seq_lens[b]-1 followed by tbq4_attn_decode (same
+ * bytes in the caches, same output); the rows are encoded inside the
+ * attention kernel by the CTA that streams that position, which saves the two
+ * append launches of a decode step.  This fuses the page's two per-token
+ * operations, writing the new token into the TBQ4 cache and reading the cache
+ * in the flash-attention kernel (trefon.com, "Kontekst 262K na jednej RTX
+ * 4090", sections "Konfiguracja" and "Od czego zaczalem").
+ *   k_new, v_new  device, fp32 [B][Hkv][128], 16-byte aligned
+ *   seq_lens      device, int32 [B], counting the appended token; a length
+ *                 of 0 appends nothing and gives a zero output row.
+ * Other arguments as tbq4_attn_decode; the caches are written.
+ */
+TBQ4_API tbq4_status tbq4_attn_decode_append(const float *q, const float *k_new,
+                                             const float *v_new, uint8_t *k_cache,
+                                             uint8_t *v_cache, const int32_t *seq_lens,
+                                             int32_t max_len, int B, int Hq, int Hkv,
+                                             int64_t capacity, float softmax_scale,
+                                             uint64_t sign_seed, void *workspace,
+                                             size_t ws_bytes, uint16_t *out, void *stream);
+
 /* As tbq4_attn_decode, with the context split into pieces of
  * `split_tokens` keys (a multiple of 32; 0 = automatic).  The result does
  * not depend on the split beyond fp32 rounding.  Workspace requirement:

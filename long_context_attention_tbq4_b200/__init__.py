@@ -23,7 +23,7 @@ BLOCK_BYTES = 66
 __all__ = [
     "D", "BLOCK_BYTES", "LIB_PATH", "Tbq4Error", "tbq4_block_bytes",
     "tbq4_cache_bytes", "tbq4_signs", "tbq4_quantize_append",
-    "tbq4_decode_workspace_bytes", "tbq4_attn_decode",
+    "tbq4_decode_workspace_bytes", "tbq4_attn_decode", "tbq4_attn_decode_append",
     "tbq4_prefill_workspace_bytes", "tbq4_attn_prefill_chunk",
     "tbq4_set_timing_events", "tbq4_get_device_status", "empty_cache",
 ]
@@ -113,6 +113,36 @@ def tbq4_attn_decode(q, k_cache, v_cache, seq_lens, max_len, softmax_scale,
         cap, float(softmax_scale), C.c_uint64(sign_seed), int(split_tokens),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out),
         _stream(stream)), "tbq4_attn_decode")
+    return out
+
+
+def tbq4_attn_decode_append(q, k_new, v_new, k_cache, v_cache, seq_lens, max_len,
+                            softmax_scale, sign_seed=0, workspace=None, out=None, stream=None):
+    """One decode step: k_new / v_new fp32 [B][Hkv][128] are encoded into the
+    caches at position seq_lens[b]-1, then decode attention over seq_lens[b]
+    keys; returns fp16 [B][Hq][128]."""
+    _need(q, torch.float32, "q", 3)
+    _need(k_new, torch.float32, "k_new", 3)
+    _need(v_new, torch.float32, "v_new", 3)
+    _need(k_cache, torch.uint8, "k_cache", 4)
+    _need(v_cache, torch.uint8, "v_cache", 4)
+    _need(seq_lens, torch.int32, "seq_lens", 1)
+    B, Hq, d = q.shape
+    _, Hkv, cap, nb = k_cache.shape
+    if (d != D or nb != BLOCK_BYTES or v_cache.shape != k_cache.shape or k_cache.shape[0] != B
+            or tuple(k_new.shape) != (B, Hkv, D) or tuple(v_new.shape) != (B, Hkv, D)):
+        raise ValueError("shape mismatch between q, new rows and caches")
+    need = tbq4_decode_workspace_bytes(B, Hq, Hkv, max_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float16, device=q.device)
+    _need(out, torch.float16, "out", 3)
+    check(lib.tbq4_attn_decode_append(
+        _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
+        int(max_len), B, Hq, Hkv, cap, float(softmax_scale), C.c_uint64(sign_seed),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out),
+        _stream(stream)), "tbq4_attn_decode_append")
     return out
 
 

@@ -34,6 +34,13 @@ struct AttnParams {
     void *out;                  // [nseq][Hq][128], fp16 or bf16
     int out_bf16;
     int all_splits;             // combine every split (prefill) instead of ceil(len/split)
+    // Fused append (decode step): the current token's K and V rows, fp32
+    // [nseq][Hkv][128], encoded into the caches at position len - 1 by the
+    // CTA that streams that position.  nullptr: no append.
+    const float *k_new;
+    const float *v_new;
+    uint8_t *k_wr;              // the same caches as k / v, written
+    uint8_t *v_wr;
 };
 
 __device__ __forceinline__ int32_t seq_length(const AttnParams &p, int s) {

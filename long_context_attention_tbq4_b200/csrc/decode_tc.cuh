@@ -27,6 +27,7 @@
 #pragma once
 #include "common.cuh"
 #include "decode.cuh"
+#include "quantize.cuh"
 
 namespace tbq4 {
 
@@ -282,9 +283,37 @@ decode_tc_kernel(const AttnParams p) {
             break;
         }
         const int ci = warp + k * kTcWarps;
-        const int32_t valid = min(kChunk, t1 - (t0 + ci * kChunk));
+        const int32_t cstart = t0 + ci * kChunk;
+        const int32_t valid = min(kChunk, t1 - cstart);
         const uint32_t kst = ring_w + st * kStageBytes;
         const uint32_t vst = kst + kChunkBytes;
+        // Fused append: if this chunk holds the current token (len - 1),
+        // encode its K and V rows here, exactly as quantize-append does,
+        // patch them into the staged blocks and store them in the caches.
+        // A length that was clamped (flagged as a capacity error) appends nothing.
+        if (p.k_new != nullptr && len - 1 >= cstart && len - 1 < cstart + valid &&
+            __ldg(p.seq_lens + s) == len) {
+            const int jn = len - 1 - cstart;
+            const uint32_t sbits = lane_sign_bits(p.sign_lo, p.sign_hi, lane);
+            const int64_t row = ((int64_t)s * p.Hkv + g) * kD;
+            const int64_t gofs = s * p.seq_stride + g * p.head_stride + (int64_t)(len - 1) * kBlockBytes;
+#pragma unroll
+            for (int kv = 0; kv < 2; ++kv) {
+                const float4 x4 = reinterpret_cast<const float4 *>((kv ? p.v_new : p.k_new) + row)[lane];
+                float xv[4] = {x4.x, x4.y, x4.z, x4.w};
+                uint16_t sb;
+                const uint32_t packed = encode_row(xv, sbits, lane, &sb);
+                const uint32_t sa = (kv ? vst : kst) + jn * kBlockBytes;
+                uint8_t *ga = (kv ? p.v_wr : p.k_wr) + gofs;
+                asm volatile("st.shared.u16 [%0], %1;" ::"r"(sa + 2 + 2 * lane), "h"((uint16_t)packed) : "memory");
+                reinterpret_cast<uint16_t *>(ga + 2)[lane] = (uint16_t)packed;
+                if (lane == 0) {
+                    asm volatile("st.shared.u16 [%0], %1;" ::"r"(sa), "h"(sb) : "memory");
+                    *reinterpret_cast<uint16_t *>(ga) = sb;
+                }
+            }
+            __syncwarp();
+        }
 
         // ---- S^T = K Q^T for two 16-token tiles (exact, integer) ---------
         float sc[2][4];

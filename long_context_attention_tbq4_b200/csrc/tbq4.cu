@@ -206,13 +206,15 @@ size_t tbq4_decode_workspace_bytes(int B, int Hq, int Hkv, int32_t max_len) {
     return tbq4_decode_workspace_bytes_split(B, Hq, Hkv, max_len, 0);
 }
 
-tbq4_status tbq4_attn_decode_split(const float *q, const uint8_t *k_cache,
-                                   const uint8_t *v_cache, const int32_t *seq_lens,
-                                   int32_t max_len, int B, int Hq, int Hkv,
-                                   int64_t capacity, float softmax_scale,
-                                   uint64_t sign_seed, int32_t split_tokens,
-                                   void *workspace, size_t ws_bytes, uint16_t *out,
-                                   void *stream) {
+}  // extern "C"
+
+namespace {
+
+tbq4_status decode_impl(const float *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                        const int32_t *seq_lens, int32_t max_len, int B, int Hq, int Hkv,
+                        int64_t capacity, float softmax_scale, uint64_t sign_seed,
+                        int32_t split_tokens, void *workspace, size_t ws_bytes, uint16_t *out,
+                        void *stream, const float *k_new, const float *v_new) {
     if (!q || !k_cache || !v_cache || !seq_lens || !workspace || !out)
         return TBQ4_ERR_NULL;
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
@@ -243,7 +245,41 @@ tbq4_status tbq4_attn_decode_split(const float *q, const uint8_t *k_cache,
     sign_words(sign_seed, &p.sign_lo, &p.sign_hi);
     p.out = out;
     p.out_bf16 = 0;
+    if (k_new) {
+        p.k_new = k_new;
+        p.v_new = v_new;
+        p.k_wr = const_cast<uint8_t *>(k_cache);
+        p.v_wr = const_cast<uint8_t *>(v_cache);
+    }
     return run_attention(p, workspace, ws_bytes, (cudaStream_t)stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+tbq4_status tbq4_attn_decode_split(const float *q, const uint8_t *k_cache,
+                                   const uint8_t *v_cache, const int32_t *seq_lens,
+                                   int32_t max_len, int B, int Hq, int Hkv,
+                                   int64_t capacity, float softmax_scale,
+                                   uint64_t sign_seed, int32_t split_tokens,
+                                   void *workspace, size_t ws_bytes, uint16_t *out,
+                                   void *stream) {
+    return decode_impl(q, k_cache, v_cache, seq_lens, max_len, B, Hq, Hkv, capacity,
+                       softmax_scale, sign_seed, split_tokens, workspace, ws_bytes, out, stream,
+                       nullptr, nullptr);
+}
+
+tbq4_status tbq4_attn_decode_append(const float *q, const float *k_new, const float *v_new,
+                                    uint8_t *k_cache, uint8_t *v_cache, const int32_t *seq_lens,
+                                    int32_t max_len, int B, int Hq, int Hkv, int64_t capacity,
+                                    float softmax_scale, uint64_t sign_seed, void *workspace,
+                                    size_t ws_bytes, uint16_t *out, void *stream) {
+    if (!k_new || !v_new) return TBQ4_ERR_NULL;
+    if (!aligned(k_new, 16) || !aligned(v_new, 16)) return TBQ4_ERR_ALIGN;
+    return decode_impl(q, k_cache, v_cache, seq_lens, max_len, B, Hq, Hkv, capacity,
+                       softmax_scale, sign_seed, 0, workspace, ws_bytes, out, stream, k_new,
+                       v_new);
 }
 
 tbq4_status tbq4_attn_decode(const float *q, const uint8_t *k_cache,

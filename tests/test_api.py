@@ -136,3 +136,24 @@ def test_status_strings(T):
     from long_context_attention_tbq4_b200._lib import lib as L
     for code in range(8):
         assert len(L.tbq4_status_string(code)) > 0
+
+
+def test_decode_append_rejects_bad_arguments(T):
+    from long_context_attention_tbq4_b200._lib import lib as L
+
+    def d(**kw):
+        a = dict(q=A, kn=A, vn=A, k=A, v=A, lens=A, max_len=64, B=1, Hq=8, Hkv=2, cap=64,
+                 scale=0.1, seed=0, ws=A2, ws_bytes=1 << 30, out=A, stream=None)
+        a.update(kw)
+        return L.tbq4_attn_decode_append(a["q"], a["kn"], a["vn"], a["k"], a["v"], a["lens"],
+                                         a["max_len"], a["B"], a["Hq"], a["Hkv"], a["cap"],
+                                         a["scale"], a["seed"], a["ws"], a["ws_bytes"],
+                                         a["out"], a["stream"])
+    assert d(kn=None) == 1
+    assert d(vn=None) == 1
+    assert d(q=None) == 1
+    assert d(kn=C.c_void_p(0x10008)) == 2            # new rows must be 16-B aligned
+    assert d(v=MIS) == 2
+    assert d(Hq=7) == 3
+    assert d(cap=60) == 4
+    assert d(ws_bytes=16) == 5
