@@ -500,6 +500,36 @@ decode_tc_kernel(const AttnParams p) {
         p.part_o[row * kD + d] = O * (256.0f / 15.0f);     // 2^8 undoes the scale of P-prime
         if (d == 0) p.part_ml[row] = make_float2(M, L);
     }
+    if (p.arrive == nullptr) return;
+
+    // ---- the last CTA of this (sequence, KV head) merges its splits --------
+    __shared__ int s_last;
+    __threadfence();                 // this CTA's partials, before its arrival
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = arrive_last(p, s, g);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();                 // every other CTA's partials, after the count
+    if (merge_group<kTcWarps>(p, s, g, used_splits(p, len), reinterpret_cast<float2 *>(ring),
+                              kRingBytes / (int)sizeof(float2)))
+        return;
+    // more splits than shared memory holds: running merge, 8 / G warps a head
+    const int wph = kTcWarps / G;
+    const int h = warp / wph, sub = warp - h * wph;
+    float4 *o_s = reinterpret_cast<float4 *>(ring);                    // [8][32]
+    float *m_s = reinterpret_cast<float *>(o_s + kTcWarps * 32);        // [8]
+    float *l_s = m_s + kTcWarps;                                        // [8]
+    if (h < G) {
+        float4 O;
+        float M, L;
+        merge_split_run(p, ((int64_t)s * p.Hq + g * G + h) * p.n_splits, used_splits(p, len),
+                        sub, wph, lane, O, M, L);
+        o_s[32 * warp + lane] = O;
+        if (lane == 0) { m_s[warp] = M; l_s[warp] = L; }
+    }
+    __syncthreads();
+    if (h < G && sub == 0)
+        finish_row(p, s, g * G + h, o_s + 32 * warp, m_s + warp, l_s + warp, wph, lane);
 }
 
 }  // namespace tbq4

@@ -92,6 +92,16 @@ def test_split_counts_agree(T):
         assert rel_l2(r, results[0]) < 1e-3
 
 
+def test_many_splits_running_merge(T):
+    # 8 heads a group and 1,875 splits of 32 keys: more (m, l) pairs than the
+    # merging CTA stages in shared memory, so it takes the running merge
+    case = W.decode_case("many_splits", 33, 1, 8, 1, [60000])
+    got, want, _ = run_case(T, case, split_tokens=32)
+    check_decode(got, want)
+    got2, _, _ = run_case(T, case)
+    assert rel_l2(got, got2) < 1e-3
+
+
 def test_zero_length_gives_zero_row(T):
     case = W.decode_case("zero", 41, 3, 4, 1, [0, 5, 0])
     got, want, _ = run_case(T, case, capacity=8)
@@ -119,3 +129,48 @@ def test_deterministic(T):
     a = T.tbq4_attn_decode(q, kg, vg, lt, int(lens.max()), case.softmax_scale, 0)
     b = T.tbq4_attn_decode(q, kg, vg, lt, int(lens.max()), case.softmax_scale, 0)
     assert torch.equal(a, b)
+
+
+def test_merge_with_garbage_workspace_and_graph_replay(T):
+    """The splits are merged by the last CTA of each (sequence, KV head),
+    counted in arrival words inside the workspace (zeroed on the stream by
+    each call).  A workspace holding arbitrary bytes, and replays of a
+    captured call, must give the same output as a fresh call."""
+    import torch
+    case = W.decode_case("merge", 91, 2, 16, 4, [5000, 12000])
+    cap = 12000
+    kg = gpu_caches(case.k, case.Hkv, cap, case.sign_seed)
+    vg = gpu_caches(case.v, case.Hkv, cap, case.sign_seed)
+    q = torch.from_numpy(case.q).cuda()
+    lens = torch.from_numpy(np.asarray(case.seq_lens, np.int32)).cuda()
+    max_len = int(case.seq_lens.max())
+    ref = T.tbq4_attn_decode(q, kg, vg, lens, max_len, case.softmax_scale, case.sign_seed)
+    torch.cuda.synchronize()
+    for fill in (0xFF, 0x00, 0x5A):
+        ws = torch.full((T.tbq4_decode_workspace_bytes(2, 16, 4, max_len),), fill,
+                        dtype=torch.uint8, device="cuda")
+        out = T.tbq4_attn_decode(q, kg, vg, lens, max_len, case.softmax_scale, case.sign_seed,
+                                 workspace=ws)
+        assert T.tbq4_get_device_status() == 0
+        assert torch.equal(out, ref)
+    ws = torch.empty(T.tbq4_decode_workspace_bytes(2, 16, 4, max_len), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty_like(ref)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        T.tbq4_attn_decode(q, kg, vg, lens, max_len, case.softmax_scale, case.sign_seed,
+                           workspace=ws, out=out)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        T.tbq4_attn_decode(q, kg, vg, lens, max_len, case.softmax_scale, case.sign_seed,
+                           workspace=ws, out=out)
+    for _ in range(3):
+        out.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    del g
+    assert T.tbq4_get_device_status() == 0
