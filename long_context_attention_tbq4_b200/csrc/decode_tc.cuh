@@ -11,19 +11,23 @@
 //   S^T (32 tokens x 8 heads) = K (tokens x 128) . Q_rot^T   mma m16n8k32 u8 x s8
 //   O^T (128 dims x 8 heads) += V^T (dims x tokens) . P'^T    mma m16n8k16 f16
 //
-// K operand: the nibbles themselves, as unsigned bytes (two LOP3 and a
-// shift per 8 values).  q_rot is normalised by a power of two and held as a
-// 22-bit fixed-point integer split into three signed bytes, so the integer
-// MMAs give sum_d n_d q_d exactly; the level map is applied afterwards,
-// sum_d q_d (2n_d - 15) = 2 sum_d n_d q_d - 15 sum_d q_d.  (fp16 q was not
-// enough: heavy-tailed keys turn a 2^-12 error in q into output errors of a
-// few 1e-3 where one token dominates.)
+// K operand: each nibble byte enters twice, raw (lo + 16 hi, no unpacking)
+// and masked to its low nibble (one LOP3 per four bytes).  With the weights
+//   raw byte  : u = q_odd,           low nibble : w = 16 q_even - q_odd
+// the products sum to 16 (lo q_even + hi q_odd): 16 sum_d n_d q_d, exactly,
+// in integers.  q_rot is normalised by a power of two and held as an 18-bit
+// integer; u and w are split into three signed bytes.  The level map is
+// applied afterwards, sum_d q_d (2n_d - 15) = 2 sum_d n_d q_d - 15 sum_d q_d.
+// (fp16 q was not enough: heavy-tailed keys turn a 2^-12 error in q into
+// output errors of a few 1e-3 where one token dominates; 18 bits keep the
+// logit error below 1e-3 of a log2 unit even in the worst case.)
 // V operand: pairs of tokens are interleaved with PRMT so that one register
-// holds the same dimension of two tokens; the levels enter as n - 8 and the
-// odd level 2n - 15 is restored at the end (see lvl_lo).  P' = p * S_v (the
+// holds the same dimension of two tokens; the levels enter as (n - 8) 2^-10
+// and the odd level 2n - 15 is restored at the end (see lvl_lo).  P' = p * S_v (the
 // block scale of V), so O = sum_t p_t S_v,t (2n-15) / 15.
 // Softmax runs in fp32 in the log2 domain; the running max is per head and
-// the accumulators are only rescaled when some head's max grows.
+// the accumulators are only rescaled when some logit exceeds it by 2^3
+// (tested with one vote per chunk; the chunk max is only formed then).
 #pragma once
 #include "common.cuh"
 #include "decode.cuh"
@@ -40,6 +44,7 @@ constexpr int kWarpRing = kTcStages * kStageBytes;
 constexpr int kRingBytes = kTcWarps * kWarpRing;
 constexpr int kTcSmemBytes = kRingBytes + kTcWarps * kTcStages * 8 + 128;
 constexpr uint32_t kSpinLimit = 1u << 22;                  // bounded mbarrier wait
+constexpr int kQBits = 18;                                 // |q_int| <= 2^18
 
 static_assert(kStageBytes % 16 == 0, "stage must keep 16-byte alignment");
 constexpr float kLazyRescale = 8.0f;                       // log2 units
@@ -86,10 +91,11 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         : "memory");
 }
 
+// The MMA wrappers are pure register operations (not volatile), so the
+// compiler may interleave them with the unpacking of the next operands.
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};\n"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -98,8 +104,7 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 // D (s32) += A (u8, 16x32 row) * B (s8, 32x8 col)
 __device__ __forceinline__ void imma16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                           uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};\n"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -108,61 +113,71 @@ __device__ __forceinline__ void imma16832(int (&d)[4], uint32_t a0, uint32_t a1,
 // D (s32) = A (u8) * B (s8), accumulator starting from zero
 __device__ __forceinline__ void imma16832_z(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                             uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%10,%10,%10,%10};\n"
         : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
 
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
+// 2^x with the MUFU approximation (relative error about 2^-22; results
+// below 2^-126 flush to zero, which only drops weights that no sum can see).
+__device__ __forceinline__ float fast_ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
-__device__ __forceinline__ float lds_half(uint32_t addr) {
-    uint16_t v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-    return __half2float(__ushort_as_half(v));
+__device__ __forceinline__ uint32_t ld_u32(const uint8_t *p) {
+    return *reinterpret_cast<const uint32_t *>(p);
 }
 
-// V levels enter the tensor cores as n - 8 (exact in fp16), built from a
-// magic-exponent fp16 and one HADD2: nibble in mantissa bits 0-3 under the
-// exponent of 1024 gives 1024 + n, in bits 4-7 under 64 gives 64 + n.  Since
-// 2n - 15 = 2 (n - 8) + 1, O = 2 sum_t P'_t (n_t - 8) + sum_t P'_t; the second
-// sum (R) comes from one extra MMA per k-step with an all-ones A operand.
-constexpr uint32_t kH2Neg1032 = 0xE408E408u;   // {-1032, -1032}
-constexpr uint32_t kH2Neg72 = 0xD480D480u;     // {-72, -72}
+__device__ __forceinline__ float ld_half(const uint8_t *p) {
+    return __half2float(*reinterpret_cast<const __half *>(p));
+}
+
+// V levels enter the tensor cores as (n - 8) 2^-10, exact in fp16, from one
+// LOP3 and one HFMA2 per register: masking a nibble into the low mantissa
+// bits of an fp16 with a zero exponent field gives the subnormal n 2^-24
+// (bits 0-3) or 16 n 2^-24 (bits 4-7); fp16 arithmetic keeps subnormals, so
+// x 2^14 - 2^-7 (resp. x 2^10 - 2^-7) is (n - 8) 2^-10 with no rounding.
+// Since 2n - 15 = 2 (n - 8) + 1, O = 2^11 sum_t P'_t (n_t - 8) 2^-10 +
+// sum_t P'_t; the second sum (R) comes from one extra MMA per k-step with an
+// all-ones A operand.
+constexpr uint32_t kH2Pow14 = 0x74007400u;     // {2^14, 2^14}
+constexpr uint32_t kH2Pow10 = 0x64006400u;     // {2^10, 2^10}
+constexpr uint32_t kH2NegBias = 0xA000A000u;   // {-2^-7, -2^-7}
 constexpr uint32_t kH2Ones = 0x3C003C00u;      // {1, 1}
+constexpr float kVLevelScale = 2048.0f;        // 2 * 2^10
 
-__device__ __forceinline__ uint32_t hadd2_u32(uint32_t x, uint32_t a) {
-    __half2 r = __hadd2(*reinterpret_cast<__half2 *>(&x), *reinterpret_cast<__half2 *>(&a));
+__device__ __forceinline__ uint32_t hfma2_u32(uint32_t x, uint32_t a, uint32_t b) {
+    __half2 r = __hfma2(*reinterpret_cast<__half2 *>(&x), *reinterpret_cast<__half2 *>(&a),
+                        *reinterpret_cast<__half2 *>(&b));
     return *reinterpret_cast<uint32_t *>(&r);
 }
-// low nibbles of bytes 0 and 2 -> {n - 8, n - 8}
+// low nibbles of bytes 0 and 2 -> {(n - 8) 2^-10, (n - 8) 2^-10}
 __device__ __forceinline__ uint32_t lvl_lo(uint32_t v) {
-    return hadd2_u32((v & 0x000F000Fu) | 0x64006400u, kH2Neg1032);
+    return hfma2_u32(v & 0x000F000Fu, kH2Pow14, kH2NegBias);
 }
-// high nibbles of bytes 0 and 2 -> {n - 8, n - 8}
+// high nibbles of bytes 0 and 2 -> {(n - 8) 2^-10, (n - 8) 2^-10}
 __device__ __forceinline__ uint32_t lvl_hi(uint32_t v) {
-    return hadd2_u32((v & 0x00F000F0u) | 0x54005400u, kH2Neg72);
+    return hfma2_u32(v & 0x00F000F0u, kH2Pow10, kH2NegBias);
 }
 
-// 32-bit word of nibble bytes at an arbitrary 2-byte-aligned shared address:
-// two aligned loads and a funnel shift by 0 or 16 bits.
-struct Funnel {
-    uint32_t base, sh;
-    __device__ __forceinline__ Funnel(uint32_t addr) : base(addr & ~3u), sh((addr & 3u) * 8u) {}
-};
+// x = c0 + 256 c1 + 65536 c2 with c0, c1 in [-128, 127]
+__device__ __forceinline__ void split3(int x, int8_t &c0, int8_t &c1, int8_t &c2) {
+    const int b0 = ((x + 128) & 255) - 128;
+    const int x1 = (x - b0) >> 8;
+    const int b1 = ((x1 + 128) & 255) - 128;
+    c0 = (int8_t)b0;
+    c1 = (int8_t)b1;
+    c2 = (int8_t)((x1 - b1) >> 8);
+}
 
 __global__ void __launch_bounds__(kTcWarps * 32, 2)
 decode_tc_kernel(const AttnParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *ring = smem;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kRingBytes);
-    // prologue scratch inside the ring (before any copy is issued)
-    float *qpar = reinterpret_cast<float *>(ring + 3 * kMaxGroup * kD);    // [8][2]
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int r = lane >> 2, c = lane & 3;
@@ -173,10 +188,14 @@ decode_tc_kernel(const AttnParams p) {
     const int32_t t1 = min(len, t0 + p.split_tokens);
     const int n_chunks = t1 > t0 ? (t1 - t0 + kChunk - 1) / kChunk : 0;
 
-    // ---- q: rotate, normalise by a power of two, split into three bytes ----
-    // q_int = rint(q_rot * 2^(22-e)) with 2^e > max|q_rot|, so |q_int| <= 2^22;
-    // q_int = 65536 c2 + 256 c1 + c0 with c0, c1 in [-128, 127], |c2| <= 64.
-    int8_t *q8 = reinterpret_cast<int8_t *>(ring);                       // [3][8][128]
+    // ---- q: rotate, normalise by a power of two, 18-bit integer ----------
+    // q_int = rint(q_rot * 2^(18-e)) with 2^e > max|q_rot|, so |q_int| <= 2^18.
+    // Per dimension pair j = (2j, 2j+1): u_j = q_int[2j+1] (weight of the raw
+    // byte) and w_j = 16 q_int[2j] - q_int[2j+1] (weight of its low nibble),
+    // each split into three signed bytes, pieces [3][head][pair].
+    int8_t *qu8 = reinterpret_cast<int8_t *>(ring);                     // [3][8][64]
+    int8_t *qw8 = qu8 + 3 * kMaxGroup * 64;                              // [3][8][64]
+    float *qpar = reinterpret_cast<float *>(qw8 + 3 * kMaxGroup * 64);   // [8][2]
     if (warp < G) {
         const uint32_t sbits = lane_sign_bits(p.sign_lo, p.sign_hi, lane);
         const int64_t base = ((int64_t)s * p.Hq + g * G + warp) * kD + 4 * lane;
@@ -187,47 +206,49 @@ decode_tc_kernel(const AttnParams p) {
         float mx = warp_max(fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
         int e = 0;
         if (mx > 0.f) frexpf(mx, &e);                 // mx = f * 2^e, f in [0.5, 1)
-        int qsum = 0;
+        int qi[4], qsum = 0;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const int qi = __float2int_rn(ldexpf(v[k], 22 - e));
-            const int c0 = ((qi + 128) & 255) - 128;
-            const int q1 = (qi - c0) >> 8;
-            const int c1 = ((q1 + 128) & 255) - 128;
-            const int c2 = (q1 - c1) >> 8;
-            q8[(0 * kMaxGroup + warp) * kD + 4 * lane + k] = (int8_t)c0;
-            q8[(1 * kMaxGroup + warp) * kD + 4 * lane + k] = (int8_t)c1;
-            q8[(2 * kMaxGroup + warp) * kD + 4 * lane + k] = (int8_t)c2;
-            qsum += qi;
+            qi[k] = __float2int_rn(ldexpf(v[k], kQBits - e));
+            qsum += qi[k];
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {                 // pairs 2 lane + j
+            const int pair = 2 * lane + j;
+            const int u = qi[2 * j + 1], w = 16 * qi[2 * j] - qi[2 * j + 1];
+            split3(u, qu8[(0 * kMaxGroup + warp) * 64 + pair], qu8[(1 * kMaxGroup + warp) * 64 + pair],
+                   qu8[(2 * kMaxGroup + warp) * 64 + pair]);
+            split3(w, qw8[(0 * kMaxGroup + warp) * 64 + pair], qw8[(1 * kMaxGroup + warp) * 64 + pair],
+                   qw8[(2 * kMaxGroup + warp) * 64 + pair]);
         }
         qsum = __reduce_add_sync(kFull, qsum);
         if (lane == 0) {
-            // log2 logit = (2 S - 15 sum q) * S_k * scale * log2(e) / 15 * 2^(e-22)
-            const float fh = p.scale_log2 * (1.0f / 15.0f) * ldexpf(1.0f, e - 22);
-            qpar[2 * warp + 0] = 2.0f * fh;
+            // log2 logit = (2 S - 15 sum q) * S_k * scale * log2(e) / 15 * 2^(e-18),
+            // and the integer MMAs return 16 S
+            const float fh = p.scale_log2 * (1.0f / 15.0f) * ldexpf(1.0f, e - kQBits);
+            qpar[2 * warp + 0] = 0.125f * fh;
             qpar[2 * warp + 1] = -15.0f * (float)qsum * fh;
         }
     } else if (warp < kMaxGroup) {
-        for (int k = lane; k < kD; k += 32)
-            for (int pc = 0; pc < 3; ++pc) q8[(pc * kMaxGroup + warp) * kD + k] = 0;
+        for (int k = lane; k < 3 * 64; k += 32) {
+            qu8[((k >> 6) * kMaxGroup + warp) * 64 + (k & 63)] = 0;
+            qw8[((k >> 6) * kMaxGroup + warp) * 64 + (k & 63)] = 0;
+        }
         if (lane == 0) { qpar[2 * warp] = 0.f; qpar[2 * warp + 1] = 0.f; }
     }
     __syncthreads();
 
-    // B fragments of the q pieces (k = dims, n = heads), thread (n = r, c):
-    // k-step i covers dims 32c+8i .. +7; b0 = bytes of dims +0,+2,+4,+6,
-    // b1 = dims +1,+3,+5,+7 (matching the lo/hi nibble split of the word).
+    // B fragments (k = byte positions, n = heads), thread (n = r, c): k-step
+    // i covers the nibble bytes 16c + 4i .. +3 of a row (pairs of dims);
+    // b0 weighs the raw bytes, b1 their low nibbles.
     uint32_t qb[4][3][2];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
 #pragma unroll
         for (int pc = 0; pc < 3; ++pc) {
-            const uint8_t *row =
-                reinterpret_cast<const uint8_t *>(q8) + (pc * kMaxGroup + r) * kD + 32 * c + 8 * i;
-            qb[i][pc][0] = (uint32_t)row[0] | ((uint32_t)row[2] << 8) | ((uint32_t)row[4] << 16) |
-                           ((uint32_t)row[6] << 24);
-            qb[i][pc][1] = (uint32_t)row[1] | ((uint32_t)row[3] << 8) | ((uint32_t)row[5] << 16) |
-                           ((uint32_t)row[7] << 24);
+            const int o = (pc * kMaxGroup + r) * 64 + 16 * c + 4 * i;
+            qb[i][pc][0] = *reinterpret_cast<const uint32_t *>(qu8 + o);
+            qb[i][pc][1] = *reinterpret_cast<const uint32_t *>(qw8 + o);
         }
     }
     // per-head constants for this thread's score columns (heads 2c, 2c+1)
@@ -237,6 +258,7 @@ decode_tc_kernel(const AttnParams p) {
 
     // ---- per-warp ring --------------------------------------------------
     const uint32_t ring_w = smem_u32(ring) + warp * kWarpRing;
+    uint8_t *ring_p = ring + warp * kWarpRing;
     const uint32_t bar_w = smem_u32(bars) + warp * kTcStages * 8;
     const uint8_t *kb = p.k + s * p.seq_stride + g * p.head_stride;
     const uint8_t *vb = p.v + s * p.seq_stride + g * p.head_stride;
@@ -248,12 +270,10 @@ decode_tc_kernel(const AttnParams p) {
     }
     __syncwarp();
 
-    auto issue = [&](int k) {   // lane 0: copy the warp's k-th chunk
-        const int ci = warp + k * kTcWarps;
-        const int32_t start = t0 + ci * kChunk;
+    auto issue = [&](int k, int st) {   // lane 0: copy the warp's k-th chunk into stage st
+        const int32_t start = t0 + (warp + k * kTcWarps) * kChunk;
         const int32_t valid = min(kChunk, t1 - start);
         const uint32_t bytes = (uint32_t)((valid + 7) & ~7) * kBlockBytes;
-        const int st = k % kTcStages;
         const uint32_t bar = bar_w + 8 * st;
         const uint32_t dst = ring_w + st * kStageBytes;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -262,7 +282,18 @@ decode_tc_kernel(const AttnParams p) {
         bulk_g2s(dst + kChunkBytes, vb + (int64_t)start * kBlockBytes, bytes, bar);
     };
     if (lane == 0)
-        for (int k = 0; k < min(kTcStages, my_chunks); ++k) issue(k);
+        for (int k = 0; k < min(kTcStages, my_chunks); ++k) issue(k, k);
+
+    // Loop-invariant byte offsets inside a stage.  K: rows r (+8, +16, +24)
+    // of the chunk, 16 bytes from nibble byte 16c; every such row starts at
+    // the same offset mod 4 (16-row and 8-row steps are multiples of 4 bytes),
+    // so one aligned base and one funnel shift serve all four rows.
+    const int koff = r * kBlockBytes + 2 + 16 * c;
+    const int kbase = koff & ~3;
+    const uint32_t ksh = (uint32_t)(koff & 3) * 8u;
+    // V: tokens 2c + {0, 1, 8, 9} (+16 for the second k-step), nibble
+    // bytes 8r .. 8r+7; even tokens sit 2 bytes past a 4-byte boundary.
+    const int voff = 2 * c * kBlockBytes + 2 + 8 * r;
 
     float o[8][4];
 #pragma unroll
@@ -274,19 +305,19 @@ decode_tc_kernel(const AttnParams p) {
     const uint32_t hsel = (r & 1) ? 0x7632u : 0x5410u;          // half of head n = r
     const int src0 = 4 * (2 * c) + (r >> 1), src1 = 4 * (2 * c + 1) + (r >> 1);
     bool aborted = false;
+    int st = 0;
+    uint32_t phase = 0;
 
     for (int k = 0; k < my_chunks; ++k) {
-        const int st = k % kTcStages;
-        if (!mbar_wait_bounded(bar_w + 8 * st, (uint32_t)(k / kTcStages) & 1u)) {
+        if (!mbar_wait_bounded(bar_w + 8 * st, phase)) {
             if (lane == 0) record_status(7u /* TBQ4_ERR_DEVICE_TIMEOUT */);
             aborted = true;
             break;
         }
-        const int ci = warp + k * kTcWarps;
-        const int32_t cstart = t0 + ci * kChunk;
+        const int32_t cstart = t0 + (warp + k * kTcWarps) * kChunk;
         const int32_t valid = min(kChunk, t1 - cstart);
-        const uint32_t kst = ring_w + st * kStageBytes;
-        const uint32_t vst = kst + kChunkBytes;
+        uint8_t *kst = ring_p + st * kStageBytes;
+        uint8_t *vst = kst + kChunkBytes;
         // Fused append: if this chunk holds the current token (len - 1),
         // encode its K and V rows here, exactly as quantize-append does,
         // patch them into the staged blocks and store them in the caches.
@@ -303,87 +334,88 @@ decode_tc_kernel(const AttnParams p) {
                 float xv[4] = {x4.x, x4.y, x4.z, x4.w};
                 uint16_t sb;
                 const uint32_t packed = encode_row(xv, sbits, lane, &sb);
-                const uint32_t sa = (kv ? vst : kst) + jn * kBlockBytes;
+                uint8_t *sa = (kv ? vst : kst) + jn * kBlockBytes;
                 uint8_t *ga = (kv ? p.v_wr : p.k_wr) + gofs;
-                asm volatile("st.shared.u16 [%0], %1;" ::"r"(sa + 2 + 2 * lane), "h"((uint16_t)packed) : "memory");
+                reinterpret_cast<uint16_t *>(sa + 2)[lane] = (uint16_t)packed;
                 reinterpret_cast<uint16_t *>(ga + 2)[lane] = (uint16_t)packed;
                 if (lane == 0) {
-                    asm volatile("st.shared.u16 [%0], %1;" ::"r"(sa), "h"(sb) : "memory");
+                    *reinterpret_cast<uint16_t *>(sa) = sb;
                     *reinterpret_cast<uint16_t *>(ga) = sb;
                 }
             }
             __syncwarp();
         }
 
-        // ---- S^T = K Q^T for two 16-token tiles (exact, integer) ---------
+        // ---- 16 S^T = K Q^T for two 16-token tiles (exact, integer) ------
         float sc[2][4];
 #pragma unroll
         for (int tile = 0; tile < 2; ++tile) {
             int acc[3][4];
-            const Funnel f0(kst + (16 * tile + r) * kBlockBytes + 2 + 16 * c);
-            const Funnel f1(kst + (16 * tile + r + 8) * kBlockBytes + 2 + 16 * c);
+            const uint8_t *k0 = kst + kbase + tile * 16 * kBlockBytes;   // row r
+            const uint8_t *k1 = k0 + 8 * kBlockBytes;                     // row r + 8
             uint32_t w0[5], w1[5];
 #pragma unroll
-            for (int i = 0; i < 5; ++i) { w0[i] = lds32(f0.base + 4 * i); w1[i] = lds32(f1.base + 4 * i); }
+            for (int i = 0; i < 5; ++i) { w0[i] = ld_u32(k0 + 4 * i); w1[i] = ld_u32(k1 + 4 * i); }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const uint32_t x0 = __funnelshift_r(w0[i], w0[i + 1], f0.sh);
-                const uint32_t x1 = __funnelshift_r(w1[i], w1[i + 1], f1.sh);
-                // bytes of dims +0,+2,+4,+6 (lo) and +1,+3,+5,+7 (hi) of the word
-                const uint32_t lo0 = x0 & 0x0F0F0F0Fu, hi0 = (x0 >> 4) & 0x0F0F0F0Fu;
-                const uint32_t lo1 = x1 & 0x0F0F0F0Fu, hi1 = (x1 >> 4) & 0x0F0F0F0Fu;
+                const uint32_t x0 = __funnelshift_r(w0[i], w0[i + 1], ksh);   // raw bytes
+                const uint32_t x1 = __funnelshift_r(w1[i], w1[i + 1], ksh);
+                const uint32_t lo0 = x0 & 0x0F0F0F0Fu, lo1 = x1 & 0x0F0F0F0Fu;
 #pragma unroll
                 for (int pc = 0; pc < 3; ++pc) {
                     if (i == 0)
-                        imma16832_z(acc[pc], lo0, lo1, hi0, hi1, qb[i][pc][0], qb[i][pc][1]);
+                        imma16832_z(acc[pc], x0, x1, lo0, lo1, qb[i][pc][0], qb[i][pc][1]);
                     else
-                        imma16832(acc[pc], lo0, lo1, hi0, hi1, qb[i][pc][0], qb[i][pc][1]);
+                        imma16832(acc[pc], x0, x1, lo0, lo1, qb[i][pc][0], qb[i][pc][1]);
                 }
             }
-            // sum_d n_d q_int_d = 65536 acc2 + 256 acc1 + acc0
+            // 16 sum_d n_d q_int_d = 65536 acc2 + 256 acc1 + acc0
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 sc[tile][e] = fmaf((float)acc[2][e], 65536.0f, (float)(acc[1][e] * 256 + acc[0][e]));
         }
 
-        // ---- scores -> log2 logits, masked beyond `valid` -----------------
+        // ---- log2 logits relative to the running max ----------------------
         // thread's tokens: u = 0..3 -> token 8u + r (tile u>>1, row half u&1)
-        float lg[4][2], sv[4];
-        if (valid == kChunk) {
+        float sk[4], sv[4], ta[4], tb[4], xa[4], xb[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int j = 8 * u + r;
-                const float sk = lds_half(kst + j * kBlockBytes);
-                sv[u] = lds_half(vst + j * kBlockBytes);
-                lg[u][0] = fmaf(sc[u >> 1][2 * (u & 1) + 0], f2a, bha) * sk;
-                lg[u][1] = fmaf(sc[u >> 1][2 * (u & 1) + 1], f2b, bhb) * sk;
-            }
-        } else {                                  // tail chunk: mask tokens >= valid
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int j = 8 * u + r;
-                const float sk = lds_half(kst + j * kBlockBytes);
-                const float svj = lds_half(vst + j * kBlockBytes);
-                const bool ok = j < valid;
-                lg[u][0] = ok ? fmaf(sc[u >> 1][2 * (u & 1) + 0], f2a, bha) * sk : -INFINITY;
-                lg[u][1] = ok ? fmaf(sc[u >> 1][2 * (u & 1) + 1], f2b, bhb) * sk : -INFINITY;
-                sv[u] = ok ? svj : 0.f;
-            }
+        for (int u = 0; u < 4; ++u) {
+            const int j = 8 * u + r;
+            sk[u] = ld_half(kst + j * kBlockBytes);
+            sv[u] = ld_half(vst + j * kBlockBytes);
+            ta[u] = fmaf(sc[u >> 1][2 * (u & 1) + 0], f2a, bha);   // logit / S_k
+            tb[u] = fmaf(sc[u >> 1][2 * (u & 1) + 1], f2b, bhb);
+            xa[u] = fmaf(ta[u], sk[u], -m_a);                       // logit - m
+            xb[u] = fmaf(tb[u], sk[u], -m_b);
         }
-        float mxa = fmaxf(fmaxf(lg[0][0], lg[1][0]), fmaxf(lg[2][0], lg[3][0]));
-        float mxb = fmaxf(fmaxf(lg[0][1], lg[1][1]), fmaxf(lg[2][1], lg[3][1]));
+        if (valid != kChunk) {                    // tail chunk: tokens >= valid
 #pragma unroll
-        for (int msk = 4; msk < 32; msk <<= 1) {
-            mxa = fmaxf(mxa, __shfl_xor_sync(kFull, mxa, msk));
-            mxb = fmaxf(mxb, __shfl_xor_sync(kFull, mxb, msk));
+            for (int u = 0; u < 4; ++u)
+                if (8 * u + r >= valid) { xa[u] = -INFINITY; xb[u] = -INFINITY; sv[u] = 0.f; }
         }
+        bool grow = false;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) grow |= (xa[u] > kLazyRescale) | (xb[u] > kLazyRescale);
         // The running max is only moved (and the accumulators rescaled)
-        // when some head's chunk max exceeds it by more than 2^8; otherwise
-        // p = exp2(logit - m) <= 2^8, and P' carries a factor 2^-8 so that
+        // when some logit exceeds it by more than 2^3; otherwise
+        // p = 2^(logit - m) <= 2^8, and P' carries a factor 2^-8 so that
         // fp16 P' = p * S_v * 2^-8 stays <= S_v <= 65504.
-        if (__any_sync(kFull, mxa > m_a + kLazyRescale || mxb > m_b + kLazyRescale)) {
-            const float na = fmaxf(m_a, mxa), nb = fmaxf(m_b, mxb);
-            const float ca = exp2f(m_a - na), cb = exp2f(m_b - nb);
+        if (__any_sync(kFull, grow)) {
+            float mxa = -INFINITY, mxb = -INFINITY;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                xa[u] = xa[u] == -INFINITY ? -INFINITY : ta[u] * sk[u];     // the logits
+                xb[u] = xb[u] == -INFINITY ? -INFINITY : tb[u] * sk[u];
+                mxa = fmaxf(mxa, xa[u]);
+                mxb = fmaxf(mxb, xb[u]);
+            }
+#pragma unroll
+            for (int msk = 4; msk < 32; msk <<= 1) {
+                mxa = fmaxf(mxa, __shfl_xor_sync(kFull, mxa, msk));
+                mxb = fmaxf(mxb, __shfl_xor_sync(kFull, mxb, msk));
+            }
+            const float na = fmaxf(m_a, mxa), nb = fmaxf(m_b, mxb);   // finite: valid >= 1
+            const float ca = fast_ex2(m_a - na), cb = fast_ex2(m_b - nb);
             m_a = na;
             m_b = nb;
             l_a *= ca;
@@ -393,11 +425,13 @@ decode_tc_kernel(const AttnParams p) {
                 o[mt][0] *= ca; o[mt][1] *= cb; o[mt][2] *= ca; o[mt][3] *= cb;
             }
             rr[0] *= ca; rr[1] *= cb; rr[2] *= ca; rr[3] *= cb;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) { xa[u] -= m_a; xb[u] -= m_b; }
         }
         uint32_t p2[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const float pa = exp2f(lg[u][0] - m_a), pb = exp2f(lg[u][1] - m_b);
+            const float pa = fast_ex2(xa[u]), pb = fast_ex2(xb[u]);
             l_a += pa;
             l_b += pb;
             const float svs = sv[u] * (1.0f / 256.0f);
@@ -422,13 +456,12 @@ decode_tc_kernel(const AttnParams p) {
             uint32_t xw[4][2];   // [token 2c, 2c+1, 2c+8, 2c+9][word]
 #pragma unroll
             for (int tt = 0; tt < 4; ++tt) {
-                const int j = 16 * ks + 2 * c + (tt & 1) + 8 * (tt >> 1);
-                const uint32_t a = vst + j * kBlockBytes + 2 + 8 * r;
+                const uint8_t *a = vst + voff + (16 * ks + (tt & 1) + 8 * (tt >> 1)) * kBlockBytes;
                 if (tt & 1) {            // odd token: its nibbles are 4-byte aligned
-                    xw[tt][0] = lds32(a);
-                    xw[tt][1] = lds32(a + 4);
+                    xw[tt][0] = ld_u32(a);
+                    xw[tt][1] = ld_u32(a + 4);
                 } else {                 // even token: 2 bytes past a 4-byte boundary
-                    const uint32_t w0 = lds32(a - 2), w1 = lds32(a + 2), w2 = lds32(a + 6);
+                    const uint32_t w0 = ld_u32(a - 2), w1 = ld_u32(a + 2), w2 = ld_u32(a + 6);
                     xw[tt][0] = __byte_perm(w0, w1, 0x5432);
                     xw[tt][1] = __byte_perm(w1, w2, 0x5432);
                 }
@@ -450,7 +483,8 @@ decode_tc_kernel(const AttnParams p) {
         }
 
         __syncwarp();
-        if (lane == 0 && k + kTcStages < my_chunks) issue(k + kTcStages);
+        if (lane == 0 && k + kTcStages < my_chunks) issue(k + kTcStages, st);
+        if (++st == kTcStages) { st = 0; phase ^= 1u; }
     }
 
     // ---- warp totals, CTA merge, partial write ----------------------------
@@ -464,14 +498,14 @@ decode_tc_kernel(const AttnParams p) {
     float *o_w = reinterpret_cast<float *>(ring);                       // [W][8][128]
     float *m_w = o_w + kTcWarps * kMaxGroup * kD;                        // [W][8]
     float *l_w = m_w + kTcWarps * kMaxGroup;                             // [W][8]
-    // sum_t P'_t (2n - 15) = 2 sum_t P'_t (n - 8) + sum_t P'_t
+    // sum_t P'_t (2n - 15) = 2^11 sum_t P'_t (n - 8) 2^-10 + sum_t P'_t
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
         const int d0 = 16 * r + 2 * mt;
-        o_w[(warp * kMaxGroup + 2 * c) * kD + d0] = fmaf(2.f, o[mt][0], rr[0]);
-        o_w[(warp * kMaxGroup + 2 * c + 1) * kD + d0] = fmaf(2.f, o[mt][1], rr[1]);
-        o_w[(warp * kMaxGroup + 2 * c) * kD + d0 + 1] = fmaf(2.f, o[mt][2], rr[2]);
-        o_w[(warp * kMaxGroup + 2 * c + 1) * kD + d0 + 1] = fmaf(2.f, o[mt][3], rr[3]);
+        o_w[(warp * kMaxGroup + 2 * c) * kD + d0] = fmaf(kVLevelScale, o[mt][0], rr[0]);
+        o_w[(warp * kMaxGroup + 2 * c + 1) * kD + d0] = fmaf(kVLevelScale, o[mt][1], rr[1]);
+        o_w[(warp * kMaxGroup + 2 * c) * kD + d0 + 1] = fmaf(kVLevelScale, o[mt][2], rr[2]);
+        o_w[(warp * kMaxGroup + 2 * c + 1) * kD + d0 + 1] = fmaf(kVLevelScale, o[mt][3], rr[3]);
     }
     if (r == 0) {
         m_w[warp * kMaxGroup + 2 * c] = m_a;
