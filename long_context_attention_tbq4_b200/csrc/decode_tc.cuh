@@ -35,14 +35,16 @@
 
 namespace tbq4 {
 
-constexpr int kTcWarps = 8;
+constexpr int kTcWarps = 16;                              // one CTA per SM
 constexpr int kTcStages = 3;
 constexpr int kChunk = 32;                                 // tokens per chunk
 constexpr int kChunkBytes = kChunk * kBlockBytes;          // 2112
 constexpr int kStageBytes = 2 * kChunkBytes + 16;          // K | V | pad
 constexpr int kWarpRing = kTcStages * kStageBytes;
 constexpr int kRingBytes = kTcWarps * kWarpRing;
-constexpr int kTcSmemBytes = kRingBytes + kTcWarps * kTcStages * 8 + 128;
+constexpr int kBarBytes = (kTcWarps * kTcStages + 1) * 8;   // + the merge barrier
+constexpr int kQScratchBytes = 2 * 3 * kMaxGroup * 64 + 2 * kMaxGroup * 4;   // q pieces + constants
+constexpr int kTcSmemBytes = kRingBytes + kBarBytes + kQScratchBytes + 128;
 constexpr uint32_t kSpinLimit = 1u << 22;                  // bounded mbarrier wait
 constexpr int kQBits = 18;                                 // |q_int| <= 2^18
 
@@ -81,6 +83,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
     bool ok = false;
     for (uint32_t i = 0; i < kSpinLimit && !ok; ++i) ok = mbar_try_wait(bar, parity);
     return __all_sync(kFull, ok);
+}
+
+// As mbar_wait_bounded, for one thread.
+__device__ __forceinline__ bool mbar_wait_bounded_1(uint32_t bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kSpinLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
 }
 
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
@@ -173,7 +182,100 @@ __device__ __forceinline__ void split3(int x, int8_t &c0, int8_t &c1, int8_t &c2
     c2 = (int8_t)((x1 - b1) >> 8);
 }
 
-__global__ void __launch_bounds__(kTcWarps * 32, 2)
+// Fused merge of the G query heads of one (sequence, KV head) by the CTA that
+// finished last, from shared memory: thread 0 pulls each head's partial rows
+// (contiguous, used x 512 B) with one bulk copy while all threads stage the
+// (m, l) pairs and warp h turns them into weights 2^(m_i - M_h); then warps
+// sum the weighted rows out of shared memory, kTcWarps / G warps a head.
+// Needs G * used * (512 + 8) bytes of the ring; returns false (nothing done)
+// otherwise.  All copies of the main loop have completed, so the ring is
+// free; the copy completes on a barrier of its own.
+__device__ __forceinline__ bool merge_group_smem(const AttnParams &p, int s, int g, int used,
+                                                 uint8_t *ring, uint64_t *bars) {
+    const int G = p.G;
+    const int64_t obytes = (int64_t)G * used * kD * 4;
+    if (used <= 0 || obytes + (int64_t)G * used * 8 + kTcWarps * 32 * 16 + 2 * kTcWarps * 4 >
+                         kRingBytes)
+        return false;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t row_g = ((int64_t)s * p.Hq + (int64_t)g * G) * p.n_splits;
+    float *o_all = reinterpret_cast<float *>(ring);                     // [G][used][128]
+    float2 *ml_s = reinterpret_cast<float2 *>(ring + obytes);           // [G][used]
+    float4 *red = reinterpret_cast<float4 *>(ml_s + G * used);          // [warps][32]
+    float *L_s = reinterpret_cast<float *>(red + kTcWarps * 32);        // [warps]
+    const uint32_t bar = smem_u32(bars + kTcWarps * kTcStages);   // initialised at entry
+    if (tid == 0) {
+        // other CTAs' partials (generic writes, acquired above) are read by
+        // the async proxy
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        mbar_expect_tx(bar, (uint32_t)obytes);
+        for (int h = 0; h < G; ++h)
+            bulk_g2s(smem_u32(o_all) + (uint32_t)(h * used * kD * 4),
+                     p.part_o + (row_g + (int64_t)h * p.n_splits) * kD, (uint32_t)(used * kD * 4),
+                     bar);
+    }
+    for (int idx = tid; idx < G * used; idx += kTcWarps * 32) {
+        const int h = idx / used, i = idx - h * used;
+        ml_s[idx] = __ldcg(p.part_ml + row_g + (int64_t)h * p.n_splits + i);
+    }
+    __syncthreads();
+    if (warp < G) {
+        float2 *mh = ml_s + warp * used;
+        float M = -INFINITY;
+        for (int i = lane; i < used; i += 32) M = fmaxf(M, mh[i].x);
+        M = warp_max(M);
+        float L = 0.f;
+        for (int i = lane; i < used; i += 32) {
+            const float2 ml = mh[i];
+            const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
+            L += w * ml.y;
+            mh[i].x = w;
+        }
+        L = warp_sum(L);
+        if (lane == 0) L_s[warp] = L;
+    }
+    __syncthreads();
+    bool ok = true;
+    if (tid == 0) ok = mbar_wait_bounded_1(bar, 0);
+    ok = __syncthreads_and(ok);
+    if (!ok) {
+        if (tid == 0) record_status(7u /* TBQ4_ERR_DEVICE_TIMEOUT */);
+        return true;
+    }
+    // warp = (head h, part sub of wph); lane owns dims 4 lane .. +3
+    const int wph = kTcWarps / G;
+    const int h = warp / wph, sub = warp - h * wph;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (h < G) {
+        const float2 *mh = ml_s + h * used;
+        const float4 *oh = reinterpret_cast<const float4 *>(o_all + (int64_t)h * used * kD) + lane;
+        for (int i = sub; i < used; i += wph) {
+            const float w = mh[i].x;
+            const float4 x = oh[i * 32];
+            acc.x = fmaf(w, x.x, acc.x);
+            acc.y = fmaf(w, x.y, acc.y);
+            acc.z = fmaf(w, x.z, acc.z);
+            acc.w = fmaf(w, x.w, acc.w);
+        }
+    }
+    red[warp * 32 + lane] = acc;
+    __syncthreads();
+    if (h < G && sub == 0) {
+        float v[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int k = 0; k < wph; ++k) {
+            const float4 a = red[(warp + k) * 32 + lane];
+            v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+        }
+        const float L = L_s[h];
+        const float inv = L > 0.f ? 1.0f / L : 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) v[k] *= inv;
+        store_row(p, s, g * G + h, v, lane);
+    }
+    return true;
+}
+
+__global__ void __launch_bounds__(kTcWarps * 32, 1)
 decode_tc_kernel(const AttnParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *ring = smem;
@@ -183,25 +285,58 @@ decode_tc_kernel(const AttnParams p) {
     const int r = lane >> 2, c = lane & 3;
     const int split = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
     const int G = p.G;
+    // q first: these loads must not queue behind the bulk copies issued below
+    float qv[4] = {0.f, 0.f, 0.f, 0.f};
+    if (warp < G) {
+        const int64_t base = ((int64_t)s * p.Hq + g * G + warp) * kD + 4 * lane;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) qv[k] = load_q(p, base + k);
+    }
     const int32_t len = seq_length(p, s);
     const int32_t t0 = split * p.split_tokens;
     const int32_t t1 = min(len, t0 + p.split_tokens);
     const int n_chunks = t1 > t0 ? (t1 - t0 + kChunk - 1) / kChunk : 0;
+
+    // ---- per-warp ring: the first copies go out before the q prologue -----
+    const uint32_t ring_w = smem_u32(ring) + warp * kWarpRing;
+    uint8_t *ring_p = ring + warp * kWarpRing;
+    const uint32_t bar_w = smem_u32(bars) + warp * kTcStages * 8;
+    const uint8_t *kb = p.k + s * p.seq_stride + g * p.head_stride;
+    const uint8_t *vb = p.v + s * p.seq_stride + g * p.head_stride;
+    const int my_chunks = warp < n_chunks ? (n_chunks - warp + kTcWarps - 1) / kTcWarps : 0;
+
+    if (lane == 0) {
+        for (int st = 0; st < kTcStages; ++st) mbar_init(bar_w + 8 * st, 1);
+        if (warp == 0) mbar_init(smem_u32(bars + kTcWarps * kTcStages), 1);   // the merge's
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+
+    auto issue = [&](int k, int st) {   // lane 0: copy the warp's k-th chunk into stage st
+        const int32_t start = t0 + (warp + k * kTcWarps) * kChunk;
+        const int32_t valid = min(kChunk, t1 - start);
+        const uint32_t bytes = (uint32_t)((valid + 7) & ~7) * kBlockBytes;
+        const uint32_t bar = bar_w + 8 * st;
+        const uint32_t dst = ring_w + st * kStageBytes;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_expect_tx(bar, 2 * bytes);
+        bulk_g2s(dst, kb + (int64_t)start * kBlockBytes, bytes, bar);
+        bulk_g2s(dst + kChunkBytes, vb + (int64_t)start * kBlockBytes, bytes, bar);
+    };
+    if (lane == 0)
+        for (int k = 0; k < min(kTcStages, my_chunks); ++k) issue(k, k);
 
     // ---- q: rotate, normalise by a power of two, 18-bit integer ----------
     // q_int = rint(q_rot * 2^(18-e)) with 2^e > max|q_rot|, so |q_int| <= 2^18.
     // Per dimension pair j = (2j, 2j+1): u_j = q_int[2j+1] (weight of the raw
     // byte) and w_j = 16 q_int[2j] - q_int[2j+1] (weight of its low nibble),
     // each split into three signed bytes, pieces [3][head][pair].
-    int8_t *qu8 = reinterpret_cast<int8_t *>(ring);                     // [3][8][64]
+    int8_t *qu8 = reinterpret_cast<int8_t *>(smem + kRingBytes + kBarBytes);   // [3][8][64]
     int8_t *qw8 = qu8 + 3 * kMaxGroup * 64;                              // [3][8][64]
     float *qpar = reinterpret_cast<float *>(qw8 + 3 * kMaxGroup * 64);   // [8][2]
     if (warp < G) {
         const uint32_t sbits = lane_sign_bits(p.sign_lo, p.sign_hi, lane);
-        const int64_t base = ((int64_t)s * p.Hq + g * G + warp) * kD + 4 * lane;
-        float v[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) v[k] = load_q(p, base + k);
+        float v[4] = {qv[0], qv[1], qv[2], qv[3]};
         warp_rotate128(v, sbits, lane);
         float mx = warp_max(fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
         int e = 0;
@@ -254,35 +389,7 @@ decode_tc_kernel(const AttnParams p) {
     // per-head constants for this thread's score columns (heads 2c, 2c+1)
     const float f2a = qpar[4 * c + 0], bha = qpar[4 * c + 1];
     const float f2b = qpar[4 * c + 2], bhb = qpar[4 * c + 3];
-    __syncthreads();   // the ring is about to be overwritten by copies
 
-    // ---- per-warp ring --------------------------------------------------
-    const uint32_t ring_w = smem_u32(ring) + warp * kWarpRing;
-    uint8_t *ring_p = ring + warp * kWarpRing;
-    const uint32_t bar_w = smem_u32(bars) + warp * kTcStages * 8;
-    const uint8_t *kb = p.k + s * p.seq_stride + g * p.head_stride;
-    const uint8_t *vb = p.v + s * p.seq_stride + g * p.head_stride;
-    const int my_chunks = warp < n_chunks ? (n_chunks - warp + kTcWarps - 1) / kTcWarps : 0;
-
-    if (lane == 0) {
-        for (int st = 0; st < kTcStages; ++st) mbar_init(bar_w + 8 * st, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncwarp();
-
-    auto issue = [&](int k, int st) {   // lane 0: copy the warp's k-th chunk into stage st
-        const int32_t start = t0 + (warp + k * kTcWarps) * kChunk;
-        const int32_t valid = min(kChunk, t1 - start);
-        const uint32_t bytes = (uint32_t)((valid + 7) & ~7) * kBlockBytes;
-        const uint32_t bar = bar_w + 8 * st;
-        const uint32_t dst = ring_w + st * kStageBytes;
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_expect_tx(bar, 2 * bytes);
-        bulk_g2s(dst, kb + (int64_t)start * kBlockBytes, bytes, bar);
-        bulk_g2s(dst + kChunkBytes, vb + (int64_t)start * kBlockBytes, bytes, bar);
-    };
-    if (lane == 0)
-        for (int k = 0; k < min(kTcStages, my_chunks); ++k) issue(k, k);
 
     // Loop-invariant byte offsets inside a stage.  K: rows r (+8, +16, +24)
     // of the chunk, 16 bytes from nibble byte 16c; every such row starts at
@@ -305,9 +412,18 @@ decode_tc_kernel(const AttnParams p) {
     const uint32_t hsel = (r & 1) ? 0x7632u : 0x5410u;          // half of head n = r
     const int src0 = 4 * (2 * c) + (r >> 1), src1 = 4 * (2 * c + 1) + (r >> 1);
     bool aborted = false;
-    int st = 0;
     uint32_t phase = 0;
+    // Fused append: the warp whose chunk holds the current token (len - 1)
+    // encodes its K and V rows, exactly as quantize-append does, patches them
+    // into the staged blocks and stores them in the caches.  A length that
+    // was clamped (flagged as a capacity error) appends nothing.
+    int k_app = -1;
+    if (p.k_new != nullptr && len - 1 >= t0 && len - 1 < t1 && __ldg(p.seq_lens + s) == len) {
+        const int ci = (len - 1 - t0) / kChunk;
+        if (ci % kTcWarps == warp) k_app = ci / kTcWarps;
+    }
 
+    int st = 0;
     for (int k = 0; k < my_chunks; ++k) {
         if (!mbar_wait_bounded(bar_w + 8 * st, phase)) {
             if (lane == 0) record_status(7u /* TBQ4_ERR_DEVICE_TIMEOUT */);
@@ -318,12 +434,7 @@ decode_tc_kernel(const AttnParams p) {
         const int32_t valid = min(kChunk, t1 - cstart);
         uint8_t *kst = ring_p + st * kStageBytes;
         uint8_t *vst = kst + kChunkBytes;
-        // Fused append: if this chunk holds the current token (len - 1),
-        // encode its K and V rows here, exactly as quantize-append does,
-        // patch them into the staged blocks and store them in the caches.
-        // A length that was clamped (flagged as a capacity error) appends nothing.
-        if (p.k_new != nullptr && len - 1 >= cstart && len - 1 < cstart + valid &&
-            __ldg(p.seq_lens + s) == len) {
+        if (k == k_app) {
             const int jn = len - 1 - cstart;
             const uint32_t sbits = lane_sign_bits(p.sign_lo, p.sign_hi, lane);
             const int64_t row = ((int64_t)s * p.Hkv + g) * kD;
@@ -514,9 +625,9 @@ decode_tc_kernel(const AttnParams p) {
         l_w[warp * kMaxGroup + 2 * c + 1] = l_b;
     }
     __syncthreads();
-    // 256 threads: thread = (head half, dim); levels carry a factor 15
+    // thread = (head, dim), kTcWarps * 32 / 128 heads at a time; levels carry a factor 15
     const int d = threadIdx.x & (kD - 1);
-    for (int h = threadIdx.x >> 7; h < G; h += 2) {
+    for (int h = threadIdx.x >> 7; h < G; h += kTcWarps * 32 / kD) {
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kTcWarps; ++w) M = fmaxf(M, m_w[w * kMaxGroup + h]);
@@ -544,6 +655,8 @@ decode_tc_kernel(const AttnParams p) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();                 // every other CTA's partials, after the count
+    if (merge_group_smem(p, s, g, used_splits(p, len), ring, bars))
+        return;
     if (merge_group<kTcWarps>(p, s, g, used_splits(p, len), reinterpret_cast<float2 *>(ring),
                               kRingBytes / (int)sizeof(float2)))
         return;

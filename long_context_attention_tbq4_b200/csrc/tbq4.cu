@@ -44,7 +44,7 @@ void sign_words(uint64_t seed, uint64_t *lo, uint64_t *hi) {
 // Keys per split: one wave of the decode kernel (two CTAs per SM) over the
 // whole launch, a multiple of 32, at least 256.
 int32_t auto_split_tokens(int nseq, int Hkv, int32_t max_len) {
-    const int64_t target = (int64_t)kNumSMs * 2;
+    const int64_t target = (int64_t)kNumSMs;          // one decode CTA per SM
     int64_t per = ceil_div((int64_t)max_len * nseq * Hkv, target);
     per = ceil_div(per, 32) * 32;
     if (per < 256) per = 256;

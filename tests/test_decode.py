@@ -93,9 +93,9 @@ def test_split_counts_agree(T):
 
 
 def test_many_splits_running_merge(T):
-    # 8 heads a group and 1,875 splits of 32 keys: more (m, l) pairs than the
+    # 8 heads a group and 3,438 splits of 32 keys: more (m, l) pairs than the
     # merging CTA stages in shared memory, so it takes the running merge
-    case = W.decode_case("many_splits", 33, 1, 8, 1, [60000])
+    case = W.decode_case("many_splits", 33, 1, 8, 1, [110000])
     got, want, _ = run_case(T, case, split_tokens=32)
     check_decode(got, want)
     got2, _, _ = run_case(T, case)
