@@ -41,11 +41,6 @@ struct AttnParams {
     const float *v_new;
     uint8_t *k_wr;              // the same caches as k / v, written
     uint8_t *v_wr;
-    // Split merge inside the decode kernel: one arrival count per (sequence,
-    // KV head), zeroed on the stream before the launch; the CTA that brings
-    // it to n_splits merges the splits.  nullptr: a separate combine launch
-    // merges.
-    unsigned int *arrive;
 };
 
 __device__ __forceinline__ int32_t seq_length(const AttnParams &p, int s) {
@@ -68,8 +63,7 @@ __device__ __forceinline__ float load_q(const AttnParams &p, int64_t idx) {
 // Log-sum-exp merge of the split partials of one output row (log2 units).
 // A warp takes splits sub, sub + nsub, ... with a running max (independent
 // loads, no dependent chain over all splits); each lane owns four dimensions
-// (one float4).  Partials are read from L2 (.cg): in the fused merge they were
-// written by other CTAs of the same launch.
+// (one float4).  Partials are read from L2 (.cg).
 __device__ __forceinline__ void merge_split_run(const AttnParams &p, int64_t row0, int used,
                                                 int sub, int nsub, int lane, float4 &O,
                                                 float &M, float &L) {
@@ -146,14 +140,17 @@ __device__ __forceinline__ int used_splits(const AttnParams &p, int32_t len) {
     return p.all_splits ? p.n_splits : (len + p.split_tokens - 1) / p.split_tokens;
 }
 
-// One CTA per (sequence, query head): eight warps take interleaved splits,
+// One CTA per (sequence, query head): sixteen warps take interleaved splits,
 // warp 0 merges them and writes the output row.
-constexpr int kCombineWarps = 8;
+constexpr int kCombineWarps = 16;
 
 __global__ void __launch_bounds__(kCombineWarps * 32)
 decode_combine_kernel(const AttnParams p) {
     __shared__ float4 o_s[kCombineWarps * 32];
     __shared__ float m_s[kCombineWarps], l_s[kCombineWarps];
+    // Launched as a programmatic dependent of the split kernel: wait for all
+    // of its partials (a no-op under an ordinary launch).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int h = blockIdx.x, s = blockIdx.y;
     const int32_t len = seq_length(p, s);
@@ -165,86 +162,6 @@ decode_combine_kernel(const AttnParams p) {
     if (lane == 0) { m_s[warp] = M; l_s[warp] = L; }
     __syncthreads();
     if (warp == 0) finish_row(p, s, h, o_s, m_s, l_s, kCombineWarps, lane);
-}
-
-// Fused merge of the G query heads of one (sequence, KV head) by the CTA
-// that finished last, with every load independent of the others: (1) all
-// threads stage the splits' (m, l) in shared memory, (2) warp h turns them
-// into weights 2^(m_i - M) for head h, (3) warp h sums the weighted partial
-// rows with deeply unrolled L2 loads and stores its output row.  Needs
-// G * used float2 of shared memory; returns false (nothing done) otherwise.
-template <int kWarps>
-__device__ __forceinline__ bool merge_group(const AttnParams &p, int s, int g, int used,
-                                            float2 *ml_s, int cap_entries) {
-    const int G = p.G;
-    if (G * used > cap_entries) return false;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t row_g = ((int64_t)s * p.Hq + (int64_t)g * G) * p.n_splits;
-    for (int idx = tid; idx < G * used; idx += kWarps * 32) {
-        const int h = idx / used, i = idx - h * used;
-        ml_s[idx] = __ldcg(p.part_ml + row_g + (int64_t)h * p.n_splits + i);
-    }
-    __syncthreads();
-    if (warp < G) {
-        float2 *mh = ml_s + warp * used;
-        float M = -INFINITY;
-        for (int i = lane; i < used; i += 32) M = fmaxf(M, mh[i].x);
-        M = warp_max(M);
-        float L = 0.f;
-        for (int i = lane; i < used; i += 32) {
-            const float2 ml = mh[i];
-            const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
-            L += w * ml.y;
-            mh[i].x = w;
-        }
-        L = warp_sum(L);
-        __syncwarp();
-        const float4 *src =
-            reinterpret_cast<const float4 *>(p.part_o + (row_g + (int64_t)warp * p.n_splits) * kD) + lane;
-        float4 acc[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-        int i = 0;
-        for (; i + 16 <= used; i += 16) {
-            float4 x[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) x[u] = __ldcg(src + (int64_t)(i + u) * 32);
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const float w = mh[i + u].x;
-                float4 &a = acc[u & 3];
-                a.x = fmaf(w, x[u].x, a.x);
-                a.y = fmaf(w, x[u].y, a.y);
-                a.z = fmaf(w, x[u].z, a.z);
-                a.w = fmaf(w, x[u].w, a.w);
-            }
-        }
-        for (; i < used; ++i) {
-            const float4 x = __ldcg(src + (int64_t)i * 32);
-            const float w = mh[i].x;
-            acc[0].x = fmaf(w, x.x, acc[0].x);
-            acc[0].y = fmaf(w, x.y, acc[0].y);
-            acc[0].z = fmaf(w, x.z, acc[0].z);
-            acc[0].w = fmaf(w, x.w, acc[0].w);
-        }
-        const float inv = L > 0.f ? 1.0f / L : 0.f;
-        float v[4] = {(acc[0].x + acc[1].x) + (acc[2].x + acc[3].x),
-                      (acc[0].y + acc[1].y) + (acc[2].y + acc[3].y),
-                      (acc[0].z + acc[1].z) + (acc[2].z + acc[3].z),
-                      (acc[0].w + acc[1].w) + (acc[2].w + acc[3].w)};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) v[k] *= inv;
-        store_row(p, s, g * G + warp, v, lane);
-    }
-    return true;
-}
-
-// Called by one thread of each CTA after its partials are written and
-// fenced.  Returns true for the CTA that completes the count of its
-// (sequence, KV head).  One atomic add per CTA, no retries.
-__device__ __forceinline__ bool arrive_last(const AttnParams &p, int s, int g) {
-    const unsigned int old = atomicAdd(p.arrive + (int64_t)s * p.Hkv + g, 1u);
-    return old + 1u == (unsigned int)p.n_splits;
 }
 
 }  // namespace tbq4

@@ -42,7 +42,7 @@ constexpr int kChunkBytes = kChunk * kBlockBytes;          // 2112
 constexpr int kStageBytes = 2 * kChunkBytes + 16;          // K | V | pad
 constexpr int kWarpRing = kTcStages * kStageBytes;
 constexpr int kRingBytes = kTcWarps * kWarpRing;
-constexpr int kBarBytes = (kTcWarps * kTcStages + 1) * 8;   // + the merge barrier
+constexpr int kBarBytes = kTcWarps * kTcStages * 8;
 constexpr int kQScratchBytes = 2 * 3 * kMaxGroup * 64 + 2 * kMaxGroup * 4;   // q pieces + constants
 constexpr int kTcSmemBytes = kRingBytes + kBarBytes + kQScratchBytes + 128;
 constexpr uint32_t kSpinLimit = 1u << 22;                  // bounded mbarrier wait
@@ -83,13 +83,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
     bool ok = false;
     for (uint32_t i = 0; i < kSpinLimit && !ok; ++i) ok = mbar_try_wait(bar, parity);
     return __all_sync(kFull, ok);
-}
-
-// As mbar_wait_bounded, for one thread.
-__device__ __forceinline__ bool mbar_wait_bounded_1(uint32_t bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
 }
 
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
@@ -182,104 +175,13 @@ __device__ __forceinline__ void split3(int x, int8_t &c0, int8_t &c1, int8_t &c2
     c2 = (int8_t)((x1 - b1) >> 8);
 }
 
-// Fused merge of the G query heads of one (sequence, KV head) by the CTA that
-// finished last, from shared memory: thread 0 pulls each head's partial rows
-// (contiguous, used x 512 B) with one bulk copy while all threads stage the
-// (m, l) pairs and warp h turns them into weights 2^(m_i - M_h); then warps
-// sum the weighted rows out of shared memory, kTcWarps / G warps a head.
-// Needs G * used * (512 + 8) bytes of the ring; returns false (nothing done)
-// otherwise.  All copies of the main loop have completed, so the ring is
-// free; the copy completes on a barrier of its own.
-__device__ __forceinline__ bool merge_group_smem(const AttnParams &p, int s, int g, int used,
-                                                 uint8_t *ring, uint64_t *bars) {
-    const int G = p.G;
-    const int64_t obytes = (int64_t)G * used * kD * 4;
-    if (used <= 0 || obytes + (int64_t)G * used * 8 + kTcWarps * 32 * 16 + 2 * kTcWarps * 4 >
-                         kRingBytes)
-        return false;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t row_g = ((int64_t)s * p.Hq + (int64_t)g * G) * p.n_splits;
-    float *o_all = reinterpret_cast<float *>(ring);                     // [G][used][128]
-    float2 *ml_s = reinterpret_cast<float2 *>(ring + obytes);           // [G][used]
-    float4 *red = reinterpret_cast<float4 *>(ml_s + G * used);          // [warps][32]
-    float *L_s = reinterpret_cast<float *>(red + kTcWarps * 32);        // [warps]
-    const uint32_t bar = smem_u32(bars + kTcWarps * kTcStages);   // initialised at entry
-    if (tid == 0) {
-        // other CTAs' partials (generic writes, acquired above) are read by
-        // the async proxy
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        mbar_expect_tx(bar, (uint32_t)obytes);
-        for (int h = 0; h < G; ++h)
-            bulk_g2s(smem_u32(o_all) + (uint32_t)(h * used * kD * 4),
-                     p.part_o + (row_g + (int64_t)h * p.n_splits) * kD, (uint32_t)(used * kD * 4),
-                     bar);
-    }
-    for (int idx = tid; idx < G * used; idx += kTcWarps * 32) {
-        const int h = idx / used, i = idx - h * used;
-        ml_s[idx] = __ldcg(p.part_ml + row_g + (int64_t)h * p.n_splits + i);
-    }
-    __syncthreads();
-    if (warp < G) {
-        float2 *mh = ml_s + warp * used;
-        float M = -INFINITY;
-        for (int i = lane; i < used; i += 32) M = fmaxf(M, mh[i].x);
-        M = warp_max(M);
-        float L = 0.f;
-        for (int i = lane; i < used; i += 32) {
-            const float2 ml = mh[i];
-            const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
-            L += w * ml.y;
-            mh[i].x = w;
-        }
-        L = warp_sum(L);
-        if (lane == 0) L_s[warp] = L;
-    }
-    __syncthreads();
-    bool ok = true;
-    if (tid == 0) ok = mbar_wait_bounded_1(bar, 0);
-    ok = __syncthreads_and(ok);
-    if (!ok) {
-        if (tid == 0) record_status(7u /* TBQ4_ERR_DEVICE_TIMEOUT */);
-        return true;
-    }
-    // warp = (head h, part sub of wph); lane owns dims 4 lane .. +3
-    const int wph = kTcWarps / G;
-    const int h = warp / wph, sub = warp - h * wph;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (h < G) {
-        const float2 *mh = ml_s + h * used;
-        const float4 *oh = reinterpret_cast<const float4 *>(o_all + (int64_t)h * used * kD) + lane;
-        for (int i = sub; i < used; i += wph) {
-            const float w = mh[i].x;
-            const float4 x = oh[i * 32];
-            acc.x = fmaf(w, x.x, acc.x);
-            acc.y = fmaf(w, x.y, acc.y);
-            acc.z = fmaf(w, x.z, acc.z);
-            acc.w = fmaf(w, x.w, acc.w);
-        }
-    }
-    red[warp * 32 + lane] = acc;
-    __syncthreads();
-    if (h < G && sub == 0) {
-        float v[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int k = 0; k < wph; ++k) {
-            const float4 a = red[(warp + k) * 32 + lane];
-            v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
-        }
-        const float L = L_s[h];
-        const float inv = L > 0.f ? 1.0f / L : 0.f;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) v[k] *= inv;
-        store_row(p, s, g * G + h, v, lane);
-    }
-    return true;
-}
-
 __global__ void __launch_bounds__(kTcWarps * 32, 1)
 decode_tc_kernel(const AttnParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *ring = smem;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kRingBytes);
+    // the dependent combine kernel may be scheduled from now on
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int r = lane >> 2, c = lane & 3;
@@ -292,39 +194,54 @@ decode_tc_kernel(const AttnParams p) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) qv[k] = load_q(p, base + k);
     }
-    const int32_t len = seq_length(p, s);
+    // The first chunks are copied before the length is known, bounded by
+    // max_len (<= capacity): the split's end under the largest length.
     const int32_t t0 = split * p.split_tokens;
-    const int32_t t1 = min(len, t0 + p.split_tokens);
-    const int n_chunks = t1 > t0 ? (t1 - t0 + kChunk - 1) / kChunk : 0;
+    const int32_t t1_max = min(p.max_len, t0 + p.split_tokens);
+    const int n_chunks_max = t1_max > t0 ? (t1_max - t0 + kChunk - 1) / kChunk : 0;
 
     // ---- per-warp ring: the first copies go out before the q prologue -----
-    const uint32_t ring_w = smem_u32(ring) + warp * kWarpRing;
     uint8_t *ring_p = ring + warp * kWarpRing;
     const uint32_t bar_w = smem_u32(bars) + warp * kTcStages * 8;
     const uint8_t *kb = p.k + s * p.seq_stride + g * p.head_stride;
     const uint8_t *vb = p.v + s * p.seq_stride + g * p.head_stride;
-    const int my_chunks = warp < n_chunks ? (n_chunks - warp + kTcWarps - 1) / kTcWarps : 0;
+    // Warp w takes chunks w, w + 16, w + 32, ... of the split (fixed, so the
+    // result does not depend on timing).
 
-    if (lane == 0) {
-        for (int st = 0; st < kTcStages; ++st) mbar_init(bar_w + 8 * st, 1);
-        if (warp == 0) mbar_init(smem_u32(bars + kTcWarps * kTcStages), 1);   // the merge's
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncwarp();
-
-    auto issue = [&](int k, int st) {   // lane 0: copy the warp's k-th chunk into stage st
-        const int32_t start = t0 + (warp + k * kTcWarps) * kChunk;
-        const int32_t valid = min(kChunk, t1 - start);
+    // One thread per (warp, stage) initialises the barriers and issues the
+    // first copies: threads of the warps that do not prepare q (warps >= G)
+    // issue for all warps, so the q warps start on q at once.
+    auto issue_for = [&](int w, int ci, int st, int32_t tend) {   // chunk ci -> warp w, stage st
+        const int32_t start = t0 + ci * kChunk;
+        const int32_t valid = min(kChunk, tend - start);
         const uint32_t bytes = (uint32_t)((valid + 7) & ~7) * kBlockBytes;
-        const uint32_t bar = bar_w + 8 * st;
-        const uint32_t dst = ring_w + st * kStageBytes;
+        const uint32_t bar = smem_u32(bars) + (w * kTcStages + st) * 8;
+        const uint32_t dst = smem_u32(ring) + w * kWarpRing + st * kStageBytes;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_expect_tx(bar, 2 * bytes);
         bulk_g2s(dst, kb + (int64_t)start * kBlockBytes, bytes, bar);
         bulk_g2s(dst + kChunkBytes, vb + (int64_t)start * kBlockBytes, bytes, bar);
     };
-    if (lane == 0)
-        for (int k = 0; k < min(kTcStages, my_chunks); ++k) issue(k, k);
+    auto issue = [&](int ci, int st, int32_t tend) { issue_for(warp, ci, st, tend); };
+    {
+        const int helpers = kTcWarps - min(G, kTcWarps - 1);   // warps >= G, at least one
+        const int hw = warp - (kTcWarps - helpers);
+        for (int job = hw * 32 + lane; hw >= 0 && job < kTcWarps * kTcStages; job += helpers * 32) {
+            const int w = job / kTcStages, st = job - w * kTcStages;
+            const uint32_t bar = smem_u32(bars) + job * 8;
+            mbar_init(bar, 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+            const int ci = w + st * kTcWarps;
+            if (ci < n_chunks_max) issue_for(w, ci, st, t1_max);
+        }
+    }
+    // queue of the chunks in stages st, st+1, st+2 (mod 3); -1: none
+    int q0 = warp < n_chunks_max ? warp : -1;
+    int q1 = warp + kTcWarps < n_chunks_max ? warp + kTcWarps : -1;
+    int q2 = warp + 2 * kTcWarps < n_chunks_max ? warp + 2 * kTcWarps : -1;
+    const int32_t len = seq_length(p, s);
+    const int32_t t1 = min(len, t1_max);
+    const int n_chunks = t1 > t0 ? (t1 - t0 + kChunk - 1) / kChunk : 0;
 
     // ---- q: rotate, normalise by a power of two, 18-bit integer ----------
     // q_int = rint(q_rot * 2^(18-e)) with 2^e > max|q_rot|, so |q_int| <= 2^18.
@@ -417,24 +334,24 @@ decode_tc_kernel(const AttnParams p) {
     // encodes its K and V rows, exactly as quantize-append does, patches them
     // into the staged blocks and stores them in the caches.  A length that
     // was clamped (flagged as a capacity error) appends nothing.
-    int k_app = -1;
-    if (p.k_new != nullptr && len - 1 >= t0 && len - 1 < t1 && __ldg(p.seq_lens + s) == len) {
-        const int ci = (len - 1 - t0) / kChunk;
-        if (ci % kTcWarps == warp) k_app = ci / kTcWarps;
-    }
+    int ci_app = -1;
+    if (p.k_new != nullptr && len - 1 >= t0 && len - 1 < t1 && __ldg(p.seq_lens + s) == len)
+        ci_app = (len - 1 - t0) / kChunk;
 
+    // A warp's chunk indices grow, so the first one at or past n_chunks ends
+    // its work.
     int st = 0;
-    for (int k = 0; k < my_chunks; ++k) {
+    while (q0 >= 0 && q0 < n_chunks) {
         if (!mbar_wait_bounded(bar_w + 8 * st, phase)) {
             if (lane == 0) record_status(7u /* TBQ4_ERR_DEVICE_TIMEOUT */);
             aborted = true;
             break;
         }
-        const int32_t cstart = t0 + (warp + k * kTcWarps) * kChunk;
+        const int32_t cstart = t0 + q0 * kChunk;
         const int32_t valid = min(kChunk, t1 - cstart);
         uint8_t *kst = ring_p + st * kStageBytes;
         uint8_t *vst = kst + kChunkBytes;
-        if (k == k_app) {
+        if (q0 == ci_app) {
             const int jn = len - 1 - cstart;
             const uint32_t sbits = lane_sign_bits(p.sign_lo, p.sign_hi, lane);
             const int64_t row = ((int64_t)s * p.Hkv + g) * kD;
@@ -594,8 +511,25 @@ decode_tc_kernel(const AttnParams p) {
         }
 
         __syncwarp();
-        if (lane == 0 && k + kTcStages < my_chunks) issue(k + kTcStages, st);
+        int nxt = q2 >= 0 ? q2 + kTcWarps : -1;
+        if (nxt >= n_chunks) nxt = -1;
+        if (lane == 0 && nxt >= 0) issue(nxt, st, t1);
+        q0 = q1;
+        q1 = q2;
+        q2 = nxt;
         if (++st == kTcStages) { st = 0; phase ^= 1u; }
+    }
+
+    // Every copy still queued (issued ahead for chunks beyond the real
+    // length, or left by an aborted loop) lands before the ring is reused.
+#pragma unroll
+    for (int j = 0; j < kTcStages; ++j) {
+        const int qj = j == 0 ? q0 : (j == 1 ? q1 : q2);
+        if (qj < 0) continue;
+        int sj = st + j;
+        uint32_t par = phase;
+        if (sj >= kTcStages) { sj -= kTcStages; par ^= 1u; }
+        if (!mbar_wait_bounded(bar_w + 8 * sj, par) && lane == 0) record_status(7u);
     }
 
     // ---- warp totals, CTA merge, partial write ----------------------------
@@ -645,38 +579,6 @@ decode_tc_kernel(const AttnParams p) {
         p.part_o[row * kD + d] = O * (256.0f / 15.0f);     // 2^8 undoes the scale of P-prime
         if (d == 0) p.part_ml[row] = make_float2(M, L);
     }
-    if (p.arrive == nullptr) return;
-
-    // ---- the last CTA of this (sequence, KV head) merges its splits --------
-    __shared__ int s_last;
-    __threadfence();                 // this CTA's partials, before its arrival
-    __syncthreads();
-    if (threadIdx.x == 0) s_last = arrive_last(p, s, g);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();                 // every other CTA's partials, after the count
-    if (merge_group_smem(p, s, g, used_splits(p, len), ring, bars))
-        return;
-    if (merge_group<kTcWarps>(p, s, g, used_splits(p, len), reinterpret_cast<float2 *>(ring),
-                              kRingBytes / (int)sizeof(float2)))
-        return;
-    // more splits than shared memory holds: running merge, 8 / G warps a head
-    const int wph = kTcWarps / G;
-    const int h = warp / wph, sub = warp - h * wph;
-    float4 *o_s = reinterpret_cast<float4 *>(ring);                    // [8][32]
-    float *m_s = reinterpret_cast<float *>(o_s + kTcWarps * 32);        // [8]
-    float *l_s = m_s + kTcWarps;                                        // [8]
-    if (h < G) {
-        float4 O;
-        float M, L;
-        merge_split_run(p, ((int64_t)s * p.Hq + g * G + h) * p.n_splits, used_splits(p, len),
-                        sub, wph, lane, O, M, L);
-        o_s[32 * warp + lane] = O;
-        if (lane == 0) { m_s[warp] = M; l_s[warp] = L; }
-    }
-    __syncthreads();
-    if (h < G && sub == 0)
-        finish_row(p, s, g * G + h, o_s + 32 * warp, m_s + warp, l_s + warp, wph, lane);
 }
 
 }  // namespace tbq4

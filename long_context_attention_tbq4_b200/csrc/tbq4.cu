@@ -52,20 +52,17 @@ int32_t auto_split_tokens(int nseq, int Hkv, int32_t max_len) {
 }
 
 struct WsLayout {
-    size_t part_o, part_ml, arrive, total;
+    size_t part_o, part_ml, total;
     int n_splits;
 };
 
-// Partials, then one arrival word per (sequence, head) for the fused merge
-// (only nseq * Hkv of them are used; Hq bounds Hkv).
 WsLayout attn_ws_layout(int nseq, int Hq, int32_t max_len, int32_t split_tokens) {
     WsLayout w;
     w.n_splits = max_len > 0 ? (int)ceil_div(max_len, split_tokens) : 1;
     const size_t rows = (size_t)nseq * Hq * w.n_splits;
     w.part_o = 0;
     w.part_ml = align_up(rows * kD * sizeof(float), kWsAlign);
-    w.arrive = align_up(w.part_ml + rows * sizeof(float2), kWsAlign);
-    w.total = align_up(w.arrive + (size_t)nseq * Hq * sizeof(unsigned int), kWsAlign);
+    w.total = align_up(w.part_ml + rows * sizeof(float2), kWsAlign);
     return w;
 }
 
@@ -122,17 +119,26 @@ tbq4_status run_attention(AttnParams p, void *workspace, size_t ws_bytes,
     p.n_splits = w.n_splits;
     p.part_o = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.part_o);
     p.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) + w.part_ml);
-    // the last CTA of each (sequence, KV head) merges the splits: one launch
-    p.arrive = reinterpret_cast<unsigned int *>(static_cast<char *>(workspace) + w.arrive);
     static bool attr_set[64] = {};    // the attribute is set once per device
     if (!ensure_smem_attr((const void *)decode_tc_kernel, kTcSmemBytes, attr_set))
-        return TBQ4_ERR_LAUNCH;
-    if (cudaMemsetAsync(p.arrive, 0, (size_t)p.nseq * p.Hkv * sizeof(unsigned int), st) !=
-        cudaSuccess)
         return TBQ4_ERR_LAUNCH;
     dim3 g1(p.n_splits, p.Hkv, p.nseq);
     if (g_ev_before) cudaEventRecord(g_ev_before, st);
     decode_tc_kernel<<<g1, kTcWarps * 32, kTcSmemBytes, st>>>(p);
+    // The combine is a programmatic dependent launch: its CTAs are placed as
+    // decode CTAs retire and wait in griddepcontrol.wait for the whole decode
+    // grid, so no launch gap separates the two kernels.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.Hq, p.nseq);
+    cfg.blockDim = dim3(kCombineWarps * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, decode_combine_kernel, p) != cudaSuccess) return TBQ4_ERR_LAUNCH;
     if (g_ev_after) cudaEventRecord(g_ev_after, st);
     return launch_status();
 }

@@ -93,8 +93,8 @@ def test_split_counts_agree(T):
 
 
 def test_many_splits_running_merge(T):
-    # 8 heads a group and 3,438 splits of 32 keys: more (m, l) pairs than the
-    # merging CTA stages in shared memory, so it takes the running merge
+    # 8 heads a group and 3,438 splits of 32 keys: the combine merges
+    # thousands of partials per output row
     case = W.decode_case("many_splits", 33, 1, 8, 1, [110000])
     got, want, _ = run_case(T, case, split_tokens=32)
     check_decode(got, want)
@@ -132,10 +132,9 @@ def test_deterministic(T):
 
 
 def test_merge_with_garbage_workspace_and_graph_replay(T):
-    """The splits are merged by the last CTA of each (sequence, KV head),
-    counted in arrival words inside the workspace (zeroed on the stream by
-    each call).  A workspace holding arbitrary bytes, and replays of a
-    captured call, must give the same output as a fresh call."""
+    """The split kernel and its combine (a programmatic dependent launch)
+    share only the workspace.  A workspace holding arbitrary bytes, and
+    replays of a captured call, must give the same output as a fresh call."""
     import torch
     case = W.decode_case("merge", 91, 2, 16, 4, [5000, 12000])
     cap = 12000
