@@ -17,8 +17,9 @@ roofline of the dominant kernel, an end-to-end figure through the public
 API with host buffers, and the fp64 CPU oracle timed on the host cores.
 
 Timing: W untimed warm-up steps, then exactly K steps, each bracketed by
-CUDA events on the launching stream; the L2 cache is flushed (a 512 MiB
-memset) before every timed step, outside the events.  With N > 1 (torchrun)
+CUDA events on the launching stream; the L2 cache is flushed (512 MiB
+written, then read back, so no dirty lines are left) before every timed
+step, outside the events.  With N > 1 (torchrun)
 every rank runs an independent replica and the time is the max over ranks.
 """
 import argparse
@@ -175,6 +176,14 @@ def timing_events(torch, n):
     return ev
 
 
+def flush_l2(buf):
+    """Evict the L2: write a buffer larger than it, then read the buffer back,
+    so the write-back of the dirty lines also happens here, outside the
+    timed region, and the next step starts on a clean, cold L2."""
+    buf.zero_()
+    buf.sum()
+
+
 def bench_decode(T, torch, case, N, step_bytes, kernel_bytes, steps, warmup, flush):
     dev = torch.device("cuda")
     cap = N
@@ -210,7 +219,7 @@ def bench_decode(T, torch, case, N, step_bytes, kernel_bytes, steps, warmup, flu
     barrier()
     torch.cuda.synchronize()
     for e0, e1, k0, k1 in ev:
-        flush.zero_()
+        flush_l2(flush)
         T.tbq4_set_timing_events(k0, k1)
         e0.record()
         step()
@@ -242,7 +251,7 @@ def bench_decode(T, torch, case, N, step_bytes, kernel_bytes, steps, warmup, flu
               for _ in range(steps)]
     barrier()
     for e0, e1 in e2e_ev:
-        flush.zero_()
+        flush_l2(flush)
         e0.record()
         e2e_step()
         e1.record()
@@ -288,7 +297,7 @@ def bench_prefill(T, torch, steps, warmup, flush):
     ev = timing_events(torch, steps)
     barrier()
     for e0, e1, k0, k1 in ev:
-        flush.zero_()
+        flush_l2(flush)
         T.tbq4_set_timing_events(k0, k1)
         e0.record()
         step()
@@ -506,7 +515,8 @@ def main():
         "dtype": "f32", "data": "synthetic",
         "config": {"workload": "decode_262k", "batch": 1, "ctx": N, "Hq": case.Hq,
                    "Hkv": case.Hkv, "head_dim": D, "kv_format": "tbq4 (66 B / 128 values)",
-                   "l2": "flushed (512 MiB memset) before every timed step",
+                   "l2": "flushed before every timed step: 512 MiB written, then read back "
+                         "(no hits, no dirty lines left)",
                    "parallelism": "replicas" if world > 1 else "single"},
         "step_bytes": step_bytes,
         "pct_hbm_peak": value / world / peaks["hbm_gbs"],

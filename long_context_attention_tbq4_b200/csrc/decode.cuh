@@ -140,28 +140,88 @@ __device__ __forceinline__ int used_splits(const AttnParams &p, int32_t len) {
     return p.all_splits ? p.n_splits : (len + p.split_tokens - 1) / p.split_tokens;
 }
 
-// One CTA per (sequence, query head): sixteen warps take interleaved splits,
-// warp 0 merges them and writes the output row.
+// One CTA per (sequence, query head), sixteen warps.  Up to 64 splits: every
+// partial row (a float4 per lane, warp w takes splits w, w + 16, ...) and
+// every (m, l) is loaded at once, so the merge costs one round of L2
+// latency; the weights 2^(m_i - M) and the sum L come from block
+// reductions, the weighted rows are summed per warp and then across warps,
+// and warp 0 writes the output row.  More splits: a running merge per warp.
 constexpr int kCombineWarps = 16;
+constexpr int kCombineFast = 4;                 // splits per warp on the fast path
 
 __global__ void __launch_bounds__(kCombineWarps * 32)
 decode_combine_kernel(const AttnParams p) {
     __shared__ float4 o_s[kCombineWarps * 32];
     __shared__ float m_s[kCombineWarps], l_s[kCombineWarps];
+    __shared__ float w_s[kCombineWarps * kCombineFast];
     // Launched as a programmatic dependent of the split kernel: wait for all
     // of its partials (a no-op under an ordinary launch).
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h = blockIdx.x, s = blockIdx.y;
     const int32_t len = seq_length(p, s);
+    const int used = used_splits(p, len);
     const int64_t row0 = ((int64_t)s * p.Hq + h) * p.n_splits;
-    float4 O;
-    float M, L;
-    merge_split_run(p, row0, used_splits(p, len), warp, kCombineWarps, lane, O, M, L);
-    o_s[32 * warp + lane] = O;
-    if (lane == 0) { m_s[warp] = M; l_s[warp] = L; }
+
+    if (used > kCombineWarps * kCombineFast) {
+        float4 O;
+        float M, L;
+        merge_split_run(p, row0, used, warp, kCombineWarps, lane, O, M, L);
+        o_s[32 * warp + lane] = O;
+        if (lane == 0) { m_s[warp] = M; l_s[warp] = L; }
+        __syncthreads();
+        if (warp == 0) finish_row(p, s, h, o_s, m_s, l_s, kCombineWarps, lane);
+        return;
+    }
+    // all loads first
+    float4 x[kCombineFast];
+#pragma unroll
+    for (int k = 0; k < kCombineFast; ++k) {
+        const int i = warp + kCombineWarps * k;
+        x[k] = i < used ? __ldcg(reinterpret_cast<const float4 *>(p.part_o + (row0 + i) * kD) + lane)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float2 ml = make_float2(-INFINITY, 0.f);
+    if (tid < used) ml = __ldcg(p.part_ml + row0 + tid);
+    // M = max_i m_i
+    float mx = warp_max(ml.x);
+    if (lane == 0) m_s[warp] = mx;
     __syncthreads();
-    if (warp == 0) finish_row(p, s, h, o_s, m_s, l_s, kCombineWarps, lane);
+    float M = m_s[0];
+#pragma unroll
+    for (int w = 1; w < kCombineWarps; ++w) M = fmaxf(M, m_s[w]);
+    // weights and L = sum_i w_i l_i
+    const float wt = (ml.x == -INFINITY || M == -INFINITY) ? 0.f : exp2f(ml.x - M);
+    if (tid < used) w_s[tid] = wt;
+    const float lw = warp_sum(wt * ml.y);
+    if (lane == 0) l_s[warp] = lw;
+    __syncthreads();
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < kCombineFast; ++k) {
+        const int i = warp + kCombineWarps * k;
+        if (i < used) {
+            const float w = w_s[i];
+            acc.x = fmaf(w, x[k].x, acc.x);
+            acc.y = fmaf(w, x[k].y, acc.y);
+            acc.z = fmaf(w, x[k].z, acc.z);
+            acc.w = fmaf(w, x[k].w, acc.w);
+        }
+    }
+    o_s[32 * warp + lane] = acc;
+    __syncthreads();
+    if (warp == 0) {
+        float v[4] = {0.f, 0.f, 0.f, 0.f}, L = 0.f;
+        for (int w = 0; w < kCombineWarps; ++w) {
+            const float4 a = o_s[32 * w + lane];
+            v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+            L += l_s[w];
+        }
+        const float inv = L > 0.f ? 1.0f / L : 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) v[k] *= inv;
+        store_row(p, s, h, v, lane);
+    }
 }
 
 }  // namespace tbq4

@@ -208,9 +208,8 @@ decode_tc_kernel(const AttnParams p) {
     // Warp w takes chunks w, w + 16, w + 32, ... of the split (fixed, so the
     // result does not depend on timing).
 
-    // One thread per (warp, stage) initialises the barriers and issues the
-    // first copies: threads of the warps that do not prepare q (warps >= G)
-    // issue for all warps, so the q warps start on q at once.
+    // The last warp (never a q warp) initialises every warp's barriers and
+    // issues every warp's first chunk, so the q warps start on q at once.
     auto issue_for = [&](int w, int ci, int st, int32_t tend) {   // chunk ci -> warp w, stage st
         const int32_t start = t0 + ci * kChunk;
         const int32_t valid = min(kChunk, tend - start);
@@ -223,17 +222,12 @@ decode_tc_kernel(const AttnParams p) {
         bulk_g2s(dst + kChunkBytes, vb + (int64_t)start * kBlockBytes, bytes, bar);
     };
     auto issue = [&](int ci, int st, int32_t tend) { issue_for(warp, ci, st, tend); };
-    {
-        const int helpers = kTcWarps - min(G, kTcWarps - 1);   // warps >= G, at least one
-        const int hw = warp - (kTcWarps - helpers);
-        for (int job = hw * 32 + lane; hw >= 0 && job < kTcWarps * kTcStages; job += helpers * 32) {
-            const int w = job / kTcStages, st = job - w * kTcStages;
-            const uint32_t bar = smem_u32(bars) + job * 8;
-            mbar_init(bar, 1);
-            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-            const int ci = w + st * kTcWarps;
-            if (ci < n_chunks_max) issue_for(w, ci, st, t1_max);
-        }
+    static_assert(kTcWarps <= 32 && kMaxGroup < kTcWarps, "one issuing lane per warp");
+    if (warp == kTcWarps - 1 && lane < kTcWarps) {
+        const int w = lane;
+        for (int st = 0; st < kTcStages; ++st) mbar_init(smem_u32(bars) + (w * kTcStages + st) * 8, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (w < n_chunks_max) issue_for(w, w, 0, t1_max);   // stage 0 now, 1 and 2 after q
     }
     // queue of the chunks in stages st, st+1, st+2 (mod 3); -1: none
     int q0 = warp < n_chunks_max ? warp : -1;
@@ -306,6 +300,16 @@ decode_tc_kernel(const AttnParams p) {
     // per-head constants for this thread's score columns (heads 2c, 2c+1)
     const float f2a = qpar[4 * c + 0], bha = qpar[4 * c + 1];
     const float f2b = qpar[4 * c + 2], bhb = qpar[4 * c + 3];
+    // The rest of the first copies, after q: issued together with stage 0
+    // they would be served interleaved with it, and every warp's first chunk
+    // would land only near the end of the whole burst.
+    if (warp == kTcWarps - 1 && lane < kTcWarps) {
+        for (int st = 1; st < kTcStages; ++st) {
+            const int ci = lane + st * kTcWarps;
+            if (ci < n_chunks_max) issue_for(lane, ci, st, t1_max);
+            __syncwarp((1u << kTcWarps) - 1);
+        }
+    }
 
 
     // Loop-invariant byte offsets inside a stage.  K: rows r (+8, +16, +24)

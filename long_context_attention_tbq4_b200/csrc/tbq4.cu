@@ -41,13 +41,14 @@ void sign_words(uint64_t seed, uint64_t *lo, uint64_t *hi) {
     *hi = w[1];
 }
 
-// Keys per split: one wave of the decode kernel (two CTAs per SM) over the
-// whole launch, a multiple of 32, at least 256.
+// Keys per split: one wave of the decode kernel (one CTA per SM) over the
+// whole launch, in whole rounds of chunks for its 16 warps.
 int32_t auto_split_tokens(int nseq, int Hkv, int32_t max_len) {
     const int64_t target = (int64_t)kNumSMs;          // one decode CTA per SM
     int64_t per = ceil_div((int64_t)max_len * nseq * Hkv, target);
-    per = ceil_div(per, 32) * 32;
-    if (per < 256) per = 256;
+    // whole rounds of 32-token chunks over the 16 warps of a CTA, so every
+    // warp of a full split gets the same number of chunks
+    per = ceil_div(per, (int64_t)kChunk * kTcWarps) * ((int64_t)kChunk * kTcWarps);
     return (int32_t)per;
 }
 
