@@ -1,11 +1,12 @@
-// quantize.cuh -- TBQ4 quantise-append kernel.
+// quantize.cuh -- TBQ4 quantise-append: fp32 rows -> 66-byte blocks.
 //
-// One warp encodes one 128-value row into one 66-byte block: 512 bytes are
-// read with one 16-byte load per lane, the rotation runs in registers and
-// warp shuffles, the scale is a warp max, and each lane packs its four
-// indices into two bytes.  The op order is fixed (see warp_fwht128 and the
-// index formula below) so the bytes are identical to the codebook's
-// definition.  The kernel is HBM-bound: 512 bytes in, 66 bytes out per row.
+// Two encoders with the same op order, so the same bytes (the codebook's
+// definition, see include/tbq4.h):
+//   encode_row            one warp per row (four values per lane, the
+//                         transform over shuffles); the decode kernel uses it
+//                         to append the current token
+//   quantize_rows_kernel  one thread per row, the transform in registers;
+//                         the bulk append (HBM-bound: 512 bytes in, 66 out)
 #pragma once
 #include "common.cuh"
 
@@ -39,31 +40,138 @@ __device__ __forceinline__ uint32_t encode_row(float v[4], uint32_t sbits, int l
     return i0 | (i1 << 4) | (i2 << 8) | (i3 << 12);
 }
 
-__global__ void __launch_bounds__(256)
-quantize_append_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
-                       const int32_t *__restrict__ start_pos, int64_t capacity,
-                       uint64_t sign_lo, uint64_t sign_hi, uint8_t *__restrict__ cache) {
-    const int lane = threadIdx.x & 31;
-    const int64_t rows = (int64_t)B * n_new * Hkv;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    const uint32_t sbits = lane_sign_bits(sign_lo, sign_hi, lane);
-    for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;
-         r += nwarps) {
-        const int h = (int)(r % Hkv);
-        const int64_t t = (r / Hkv) % n_new;
-        const int b = (int)(r / ((int64_t)Hkv * n_new));
-        const float4 x4 = __ldcs(reinterpret_cast<const float4 *>(src + r * kD) + lane);
-        float v[4] = {x4.x, x4.y, x4.z, x4.w};
-        uint16_t sb;
-        const uint32_t packed = encode_row(v, sbits, lane, &sb);
-        const int64_t pos = (int64_t)__ldg(start_pos + b) + t;
-        if (pos < 0 || pos >= capacity) {
-            if (lane == 0) record_status(4u /* TBQ4_ERR_CAPACITY */);
-            continue;
+// The +-1 sign diagonal as floats, passed by value: a kernel parameter is a
+// constant-bank operand, so the signs fold into the first butterfly stage.
+struct SignTable {
+    float s[kD];
+};
+
+// One thread encodes one whole 128-value row (rows are independent, so a
+// thread per row keeps the transform in registers, with no shuffles):
+//   rotation  the same butterflies in the same order as warp_fwht128 (stride
+//             1 first; lower = a + b, upper = a - b, each rounded on its own).
+//             The sign flip is exact, so the first stage is
+//             fma(v_j, s_j, s_k v_k) and fma(v_j, s_j, -s_k v_k).
+//   scale     S = fp16(max |x_rot|), saturated at 65504.
+//   index     clamp(rne(fl32(fl32(x/S) * 7.5) + 7.5), 0, 15), 8 when S == 0.
+//             The quotient is the correctly rounded x/S by Markstein's method:
+//             r = RN(1/S) once per row, q0 = RN(x r), e = x - q0 S (exact with
+//             FMA), q = RN(q0 + e r).  The conversion to unsigned saturates
+//             negative values to 0, which with min(., 15) is the clamp.
+// Memory: a warp takes 32 rows in head-major order (row = (b Hkv + h) n_new
+// + t), so its 32 blocks are contiguous in the cache.  The rows come in with
+// one 512-byte load per row across the warp into a shared tile (16-byte
+// chunk c of row i at position c ^ (i % 8), so the per-thread reads of a
+// whole row are free of bank conflicts), and the 32 blocks go out from a
+// shared staging area as consecutive 16-bit pieces.
+constexpr int kQRows = 32;                                   // rows per warp and step
+constexpr int kQWarpBytes = kQRows * 512 + kQRows * kBlockBytes + kQRows * 8;
+constexpr int kQThreads = 128;
+constexpr int kQSmemBytes = (kQThreads / 32) * kQWarpBytes;
+
+__global__ void __launch_bounds__(kQThreads, 3)
+quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
+                     const int32_t *__restrict__ start_pos, int64_t capacity, const SignTable sg,
+                     uint8_t *__restrict__ cache) {
+    extern __shared__ __align__(16) uint8_t qsm[];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    uint8_t *wsm = qsm + wib * kQWarpBytes;
+    float4 *tile = reinterpret_cast<float4 *>(wsm);                          // [32][32]
+    uint16_t *stage = reinterpret_cast<uint16_t *>(wsm + kQRows * 512);      // [32][33]
+    int64_t *doffs = reinterpret_cast<int64_t *>(wsm + kQRows * 512 + kQRows * kBlockBytes);
+    const uint32_t rows = (uint32_t)B * (uint32_t)n_new * (uint32_t)Hkv;    // < 2^31 (host)
+    const uint32_t groups = (rows + kQRows - 1) / kQRows;
+    const uint32_t wstride = gridDim.x * (kQThreads / 32);
+    for (uint32_t gi = blockIdx.x * (kQThreads / 32) + wib; gi < groups; gi += wstride) {
+        // this lane's row and its source and destination
+        const uint32_t r = gi * kQRows + lane;
+        const bool live = r < rows;
+        const uint32_t rr = live ? r : rows - 1;
+        const uint32_t t = rr % (uint32_t)n_new, bh = rr / (uint32_t)n_new;
+        const uint32_t h = bh % (uint32_t)Hkv, b = bh / (uint32_t)Hkv;
+        const float4 *srow =
+            reinterpret_cast<const float4 *>(src + (((int64_t)b * n_new + t) * Hkv + h) * kD);
+        int64_t doff = -1;
+        if (live) {
+            const int64_t pos = (int64_t)__ldg(start_pos + b) + t;
+            if (pos < 0 || pos >= capacity) record_status(4u /* TBQ4_ERR_CAPACITY */);
+            else doff = (((int64_t)b * Hkv + h) * capacity + pos) * kBlockBytes;
         }
-        uint8_t *dst = cache + (((int64_t)b * Hkv + h) * capacity + pos) * kBlockBytes;
-        reinterpret_cast<uint16_t *>(dst + 2)[lane] = (uint16_t)packed;
-        if (lane == 0) *reinterpret_cast<uint16_t *>(dst) = sb;
+        doffs[lane] = doff;
+        // load: row i, one 16-byte chunk per lane
+#pragma unroll 8
+        for (int i = 0; i < kQRows; ++i) {
+            const float4 *pi = reinterpret_cast<const float4 *>(
+                __shfl_sync(kFull, reinterpret_cast<uintptr_t>(srow), i));
+            tile[i * 32 + (lane ^ (i & 7))] = __ldcs(pi + lane);
+        }
+        __syncwarp();
+        float v[kD];
+#pragma unroll
+        for (int c = 0; c < kD / 4; ++c) {
+            const float4 x = tile[lane * 32 + (c ^ (lane & 7))];
+            v[4 * c] = x.x;
+            v[4 * c + 1] = x.y;
+            v[4 * c + 2] = x.z;
+            v[4 * c + 3] = x.w;
+        }
+        // stage 1 with the signs folded in
+#pragma unroll
+        for (int j = 0; j < kD; j += 2) {
+            const float bb = __fmul_rn(v[j + 1], sg.s[j + 1]);
+            const float lo = __fmaf_rn(v[j], sg.s[j], bb);
+            const float hi = __fmaf_rn(v[j], sg.s[j], -bb);
+            v[j] = lo;
+            v[j + 1] = hi;
+        }
+#pragma unroll
+        for (int hs = 2; hs < kD; hs <<= 1) {
+#pragma unroll
+            for (int j = 0; j < kD; ++j) {
+                if (j & hs) continue;
+                const float a = v[j], c = v[j + hs];
+                v[j] = __fadd_rn(a, c);
+                v[j + hs] = __fsub_rn(a, c);
+            }
+        }
+        const float cr = rot_c();
+        float m = 0.f;
+#pragma unroll
+        for (int j = 0; j < kD; ++j) {
+            v[j] = __fmul_rn(v[j], cr);
+            m = fmaxf(m, fabsf(v[j]));
+        }
+        uint16_t sb = __half_as_ushort(__float2half_rn(m));
+        if ((sb & 0x7FFFu) == 0x7C00u) sb = 0x7BFFu;                 // saturate at 65504
+        const float S = half_bits_to_float(sb);
+        uint16_t *mine = stage + lane * (kBlockBytes / 2);
+        mine[0] = sb;
+        const float rs = S == 0.0f ? 0.0f : __frcp_rn(S);
+#pragma unroll
+        for (int w = 0; w < kD / 4; ++w) {                             // 4 nibbles per piece
+            uint32_t piece = 0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float x = v[4 * w + k];
+                const float q0 = __fmul_rn(x, rs);
+                const float e = __fmaf_rn(-q0, S, x);
+                const float q = __fmaf_rn(e, rs, q0);               // x / S, correctly rounded
+                const float u = __fadd_rn(__fmul_rn(q, 7.5f), 7.5f);
+                const uint32_t idx = S == 0.0f ? 8u : min(__float2uint_rn(u), 15u);
+                piece |= idx << (4 * k);
+            }
+            mine[1 + w] = (uint16_t)piece;
+        }
+        __syncwarp();
+        // store: the 32 blocks as 1,056 consecutive 16-bit pieces
+#pragma unroll
+        for (int k = 0; k < kBlockBytes / 2; ++k) {
+            const int j = lane + 32 * k;
+            const int row = j / (kBlockBytes / 2), pc = j - row * (kBlockBytes / 2);
+            const int64_t off = doffs[row];
+            if (off >= 0) *reinterpret_cast<uint16_t *>(cache + off + 2 * pc) = stage[j];
+        }
+        __syncwarp();
     }
 }
 

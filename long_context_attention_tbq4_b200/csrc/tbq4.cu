@@ -196,14 +196,19 @@ tbq4_status tbq4_quantize_append(const float *src, int B, int n_new, int Hkv,
     if (B <= 0 || n_new < 0 || Hkv <= 0) return TBQ4_ERR_SHAPE;
     if (capacity <= 0 || capacity % 8 != 0) return TBQ4_ERR_CAPACITY;
     if (n_new == 0) return TBQ4_OK;
-    uint64_t lo, hi;
-    sign_words(sign_seed, &lo, &hi);
     const int64_t rows = (int64_t)B * n_new * Hkv;
-    const int threads = 256;
-    int64_t blocks = ceil_div(rows, threads / 32);
-    if (blocks > (int64_t)kNumSMs * 16) blocks = (int64_t)kNumSMs * 16;
-    quantize_append_kernel<<<(unsigned)blocks, threads, 0, (cudaStream_t)stream>>>(
-        src, B, n_new, Hkv, start_pos, capacity, lo, hi, cache);
+    if (rows > 0x7FFFFFFFLL) return TBQ4_ERR_SHAPE;      // rows are indexed in 32 bits
+    int8_t sg8[kD];
+    tbq4_signs(sign_seed, sg8);
+    SignTable sg;
+    for (int i = 0; i < kD; ++i) sg.s[i] = (float)sg8[i];
+    static bool attr_set[64] = {};    // set once per device
+    if (!ensure_smem_attr((const void *)quantize_rows_kernel, kQSmemBytes, attr_set))
+        return TBQ4_ERR_LAUNCH;
+    int64_t blocks = ceil_div(rows, (int64_t)kQThreads);   // one row per thread
+    if (blocks > (int64_t)kNumSMs * 3) blocks = (int64_t)kNumSMs * 3;
+    quantize_rows_kernel<<<(unsigned)blocks, kQThreads, kQSmemBytes, (cudaStream_t)stream>>>(
+        src, B, n_new, Hkv, start_pos, capacity, sg, cache);
     return launch_status();
 }
 
