@@ -147,6 +147,31 @@ TBQ4_API tbq4_status tbq4_attn_decode_append(const float *q, const float *k_new,
                                              uint64_t sign_seed, void *workspace,
                                              size_t ws_bytes, uint16_t *out, void *stream);
 
+/*
+ * Multi-query decode: q_len (1-4) new query tokens per sequence, as when a
+ * model verifies speculative drafts (trefon.com, "Kontekst 262K na jednej RTX
+ * 4090", section "Konfiguracja": up to 3 drafted tokens).  Query token i of
+ * sequence b sits at position seq_lens[b] - q_len + i and attends to keys
+ * [0, seq_lens[b] - q_len + i] (bottom-right causal, as the chunked prefill),
+ * with the same arithmetic as tbq4_attn_decode.  All q_len tokens are already
+ * in the caches.
+ *   q         device, fp32 [B][q_len][Hq][128]
+ *   out       device, fp16 [B][q_len][Hq][128]
+ *   seq_lens  device, int32 [B], each >= q_len (a shorter sequence gives zero
+ *             rows for the queries that see no key)
+ * Requires (Hq / Hkv) * q_len <= 32.  The workspace size comes from
+ * tbq4_decode_mq_workspace_bytes.  q_len = 1 runs the single-query kernel.
+ * Errors as tbq4_attn_decode.
+ */
+TBQ4_API size_t tbq4_decode_mq_workspace_bytes(int B, int q_len, int Hq, int Hkv,
+                                               int32_t max_len);
+TBQ4_API tbq4_status tbq4_attn_decode_mq(const float *q, const uint8_t *k_cache,
+                                         const uint8_t *v_cache, const int32_t *seq_lens,
+                                         int32_t max_len, int B, int q_len, int Hq, int Hkv,
+                                         int64_t capacity, float softmax_scale,
+                                         uint64_t sign_seed, void *workspace, size_t ws_bytes,
+                                         uint16_t *out, void *stream);
+
 /* As tbq4_attn_decode, with the context split into pieces of
  * `split_tokens` keys (a multiple of 32; 0 = automatic).  The result does
  * not depend on the split beyond fp32 rounding.  Workspace requirement:

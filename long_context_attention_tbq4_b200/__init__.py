@@ -24,6 +24,7 @@ __all__ = [
     "D", "BLOCK_BYTES", "LIB_PATH", "Tbq4Error", "tbq4_block_bytes",
     "tbq4_cache_bytes", "tbq4_signs", "tbq4_quantize_append",
     "tbq4_decode_workspace_bytes", "tbq4_attn_decode", "tbq4_attn_decode_append",
+    "tbq4_decode_mq_workspace_bytes", "tbq4_attn_decode_mq",
     "tbq4_prefill_workspace_bytes", "tbq4_attn_prefill_chunk",
     "tbq4_set_timing_events", "tbq4_get_device_status", "empty_cache",
 ]
@@ -143,6 +144,36 @@ def tbq4_attn_decode_append(q, k_new, v_new, k_cache, v_cache, seq_lens, max_len
         int(max_len), B, Hq, Hkv, cap, float(softmax_scale), C.c_uint64(sign_seed),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out),
         _stream(stream)), "tbq4_attn_decode_append")
+    return out
+
+
+def tbq4_decode_mq_workspace_bytes(B, q_len, Hq, Hkv, max_len) -> int:
+    return int(lib.tbq4_decode_mq_workspace_bytes(B, q_len, Hq, Hkv, max_len))
+
+
+def tbq4_attn_decode_mq(q, k_cache, v_cache, seq_lens, max_len, softmax_scale, sign_seed=0,
+                        workspace=None, out=None, stream=None):
+    """q fp32 [B][q_len][Hq][128]: the last q_len tokens of each sequence
+    (already in the caches); returns fp16 [B][q_len][Hq][128]."""
+    _need(q, torch.float32, "q", 4)
+    _need(k_cache, torch.uint8, "k_cache", 4)
+    _need(v_cache, torch.uint8, "v_cache", 4)
+    _need(seq_lens, torch.int32, "seq_lens", 1)
+    B, q_len, Hq, d = q.shape
+    _, Hkv, cap, nb = k_cache.shape
+    if d != D or nb != BLOCK_BYTES or v_cache.shape != k_cache.shape or k_cache.shape[0] != B:
+        raise ValueError("shape mismatch between q and caches")
+    need = tbq4_decode_mq_workspace_bytes(B, q_len, Hq, Hkv, max_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((B, q_len, Hq, D), dtype=torch.float16, device=q.device)
+    _need(out, torch.float16, "out", 4)
+    check(lib.tbq4_attn_decode_mq(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), int(max_len), B, q_len, Hq, Hkv,
+        cap, float(softmax_scale), C.c_uint64(sign_seed), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)),
+        "tbq4_attn_decode_mq")
     return out
 
 

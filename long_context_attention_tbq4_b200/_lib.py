@@ -24,6 +24,9 @@ SIGNATURES = {
     "tbq4_attn_decode_append": (_i, [_p, _p, _p, _p, _p, _p, _i32, _i, _i, _i, _i64, _f,
                                      _u64, _p, _sz, _p, _p]),
     "tbq4_decode_workspace_bytes_split": (_sz, [_i, _i, _i, _i32, _i32]),
+    "tbq4_decode_mq_workspace_bytes": (_sz, [_i, _i, _i, _i, _i32]),
+    "tbq4_attn_decode_mq": (_i, [_p, _p, _p, _p, _i32, _i, _i, _i, _i, _i64, _f, _u64, _p, _sz,
+                                 _p, _p]),
     "tbq4_attn_decode_split": (_i, [_p, _p, _p, _p, _i32, _i, _i, _i, _i64, _f,
                                     _u64, _i32, _p, _sz, _p, _p]),
     "tbq4_attn_decode_noalloc": (_i, [_p, _p, _p, _p, _i32, _i, _i, _i, _i64, _f, _u64,

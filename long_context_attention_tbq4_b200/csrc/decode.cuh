@@ -34,6 +34,9 @@ struct AttnParams {
     void *out;                  // [nseq][Hq][128], fp16 or bf16
     int out_bf16;
     int all_splits;             // combine every split (prefill) instead of ceil(len/split)
+    // Multi-query decode: query tokens per sequence (0 or 1: one).  The
+    // combine's rows are then (sequence, query token) pairs, b * q_len + i.
+    int q_len;
     // Fused append (decode step): the current token's K and V rows, fp32
     // [nseq][Hkv][128], encoded into the caches at position len - 1 by the
     // CTA that streams that position.  nullptr: no append.
@@ -159,7 +162,7 @@ decode_combine_kernel(const AttnParams p) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h = blockIdx.x, s = blockIdx.y;
-    const int32_t len = seq_length(p, s);
+    const int32_t len = seq_length(p, p.q_len > 1 ? s / p.q_len : s);
     const int used = used_splits(p, len);
     const int64_t row0 = ((int64_t)s * p.Hq + h) * p.n_splits;
 

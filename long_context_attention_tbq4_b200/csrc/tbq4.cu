@@ -9,6 +9,7 @@
 #include "quantize.cuh"
 #include "decode.cuh"
 #include "decode_tc.cuh"
+#include "decode_mq.cuh"
 #include "prefill_tc.cuh"
 
 #include <algorithm>
@@ -49,6 +50,7 @@ int32_t auto_split_tokens(int nseq, int Hkv, int32_t max_len) {
     // whole rounds of 32-token chunks over the 16 warps of a CTA, so every
     // warp of a full split gets the same number of chunks
     per = ceil_div(per, (int64_t)kChunk * kTcWarps) * ((int64_t)kChunk * kTcWarps);
+    if (per < (int64_t)kChunk * kTcWarps) per = (int64_t)kChunk * kTcWarps;
     return (int32_t)per;
 }
 
@@ -114,23 +116,29 @@ tbq4_status launch_status() {
 tbq4_status run_attention(AttnParams p, void *workspace, size_t ws_bytes,
                           cudaStream_t st) {
     if (p.split_tokens <= 0 || p.split_tokens % 32 != 0) return TBQ4_ERR_SHAPE;
-    const WsLayout w = attn_ws_layout(p.nseq, p.Hq, p.max_len, p.split_tokens);
+    const int qrows = p.nseq * (p.q_len > 1 ? p.q_len : 1);    // combine rows per head
+    const WsLayout w = attn_ws_layout(qrows, p.Hq, p.max_len, p.split_tokens);
     if (ws_bytes < w.total) return TBQ4_ERR_WORKSPACE;
     if (w.n_splits > 65535 * 16) return TBQ4_ERR_SHAPE;
     p.n_splits = w.n_splits;
     p.part_o = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.part_o);
     p.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) + w.part_ml);
-    static bool attr_set[64] = {};    // the attribute is set once per device
-    if (!ensure_smem_attr((const void *)decode_tc_kernel, kTcSmemBytes, attr_set))
+    static bool attr_set[64] = {}, attr_mq[64] = {};    // set once per device
+    const bool mq = p.q_len > 1;
+    if (mq ? !ensure_smem_attr((const void *)dmq::decode_mq_kernel, dmq::kSmemBytes, attr_mq)
+           : !ensure_smem_attr((const void *)decode_tc_kernel, kTcSmemBytes, attr_set))
         return TBQ4_ERR_LAUNCH;
     dim3 g1(p.n_splits, p.Hkv, p.nseq);
     if (g_ev_before) cudaEventRecord(g_ev_before, st);
-    decode_tc_kernel<<<g1, kTcWarps * 32, kTcSmemBytes, st>>>(p);
+    if (mq)
+        dmq::decode_mq_kernel<<<g1, dmq::kThreads, dmq::kSmemBytes, st>>>(p);
+    else
+        decode_tc_kernel<<<g1, kTcWarps * 32, kTcSmemBytes, st>>>(p);
     // The combine is a programmatic dependent launch: its CTAs are placed as
     // decode CTAs retire and wait in griddepcontrol.wait for the whole decode
     // grid, so no launch gap separates the two kernels.
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.Hq, p.nseq);
+    cfg.gridDim = dim3(p.Hq, qrows);
     cfg.blockDim = dim3(kCombineWarps * 32);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
@@ -286,6 +294,53 @@ tbq4_status tbq4_attn_decode_split(const float *q, const uint8_t *k_cache,
     return decode_impl(q, k_cache, v_cache, seq_lens, max_len, B, Hq, Hkv, capacity,
                        softmax_scale, sign_seed, split_tokens, workspace, ws_bytes, out, stream,
                        nullptr, nullptr);
+}
+
+size_t tbq4_decode_mq_workspace_bytes(int B, int q_len, int Hq, int Hkv, int32_t max_len) {
+    if (B <= 0 || q_len <= 0 || Hq <= 0 || Hkv <= 0 || max_len < 0) return 0;
+    const int32_t split = auto_split_tokens(B, Hkv, max_len);
+    return attn_ws_layout(B * q_len, Hq, max_len, split).total;
+}
+
+tbq4_status tbq4_attn_decode_mq(const float *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                                const int32_t *seq_lens, int32_t max_len, int B, int q_len,
+                                int Hq, int Hkv, int64_t capacity, float softmax_scale,
+                                uint64_t sign_seed, void *workspace, size_t ws_bytes,
+                                uint16_t *out, void *stream) {
+    if (!q || !k_cache || !v_cache || !seq_lens || !workspace || !out) return TBQ4_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(workspace, kWsAlign) || !aligned(out, 2) || !aligned(seq_lens, 4))
+        return TBQ4_ERR_ALIGN;
+    if (B <= 0 || B > 65535 || Hkv <= 0 || Hkv > 65535 || Hq <= 0 || Hq % Hkv != 0 ||
+        Hq / Hkv > kMaxGroup || max_len < 0 || q_len < 1 || q_len > dmq::kMaxQLen ||
+        (Hq / Hkv) * q_len > dmq::kCols || (int64_t)B * q_len > 65535)
+        return TBQ4_ERR_SHAPE;
+    if (capacity <= 0 || capacity % 8 != 0 || (int64_t)max_len > capacity)
+        return TBQ4_ERR_CAPACITY;
+    if (!std::isfinite(softmax_scale)) return TBQ4_ERR_SHAPE;
+    if (q_len == 1)       // one query token: the single-query kernel, same result
+        return decode_impl(q, k_cache, v_cache, seq_lens, max_len, B, Hq, Hkv, capacity,
+                           softmax_scale, sign_seed, 0, workspace, ws_bytes, out, stream,
+                           nullptr, nullptr);
+    AttnParams p = {};
+    p.q = q;
+    p.k = k_cache;
+    p.v = v_cache;
+    p.head_stride = capacity * kBlockBytes;
+    p.seq_stride = (int64_t)Hkv * p.head_stride;
+    p.seq_lens = seq_lens;
+    p.max_len = max_len;
+    p.capacity = capacity;
+    p.nseq = B;
+    p.q_len = q_len;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = Hq / Hkv;
+    p.split_tokens = auto_split_tokens(B, Hkv, max_len);
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    sign_words(sign_seed, &p.sign_lo, &p.sign_hi);
+    p.out = out;
+    return run_attention(p, workspace, ws_bytes, (cudaStream_t)stream);
 }
 
 tbq4_status tbq4_attn_decode_append(const float *q, const float *k_new, const float *v_new,

@@ -130,6 +130,31 @@ def ragged_decode():
     return DecodeCase("ragged_decode_8", q, k, v, lens, Hq, Hkv)
 
 
+def mq_case(name, seed, B, q_len, Hq, Hkv, lens, dist="normal"):
+    """Multi-query decode inputs (q_len new tokens per sequence, already in
+    the caches).  Draw order: q N(0,1) fp32 [B][q_len][Hq][128], then K for
+    every sequence, then V for every sequence ([L_b][Hkv][128], N(0,1) or
+    Student-t nu=4)."""
+    rng = np.random.default_rng(seed)
+    lens = np.asarray(lens, np.int32)
+    q = normal(rng, (B, q_len, Hq, D))
+
+    def draw(L):
+        if dist == "normal":
+            return normal(rng, (int(L), Hkv, D))
+        return rng.standard_t(4, (int(L), Hkv, D)).astype(np.float32)
+
+    k = [draw(L) for L in lens]
+    v = [draw(L) for L in lens]
+    return DecodeCase(name, q, k, v, lens, Hq, Hkv)
+
+
+def mq_262k():
+    """4 new tokens over a 262,144-token context (the last 4 included), 24/4
+    heads, N(0,1), seed 5: the speculative verification step of the decode."""
+    return mq_case("mq4_262k", 5, 1, 4, 24, 4, [262144])
+
+
 def prefill_case(name, seed, n_cached, n_new, Hq=24, Hkv=4):
     """Chunked prefill inputs.  Draw order: q fp32 N(0,1) [n_new][Hq][128]
     rounded to bf16; K [n_cached + n_new][Hkv][128]; V likewise (all N(0,1)

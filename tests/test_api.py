@@ -157,3 +157,27 @@ def test_decode_append_rejects_bad_arguments(T):
     assert d(Hq=7) == 3
     assert d(cap=60) == 4
     assert d(ws_bytes=16) == 5
+
+
+def test_decode_mq_rejects_bad_arguments(T):
+    from long_context_attention_tbq4_b200._lib import lib as L
+
+    def d(**kw):
+        a = dict(q=A, k=A, v=A, lens=A, max_len=64, B=1, ql=2, Hq=8, Hkv=2, cap=64, scale=0.1,
+                 seed=0, ws=A2, ws_bytes=1 << 30, out=A, stream=None)
+        a.update(kw)
+        return L.tbq4_attn_decode_mq(a["q"], a["k"], a["v"], a["lens"], a["max_len"], a["B"],
+                                     a["ql"], a["Hq"], a["Hkv"], a["cap"], a["scale"], a["seed"],
+                                     a["ws"], a["ws_bytes"], a["out"], a["stream"])
+    assert d(q=None) == 1
+    assert d(q=MIS) == 2
+    assert d(ql=0) == 3                               # q_len in [1, 4]
+    assert d(ql=5) == 3
+    assert d(cap=60) == 4
+    assert d(ws_bytes=16) == 5
+
+
+def test_decode_mq_workspace_query(T):
+    assert T.tbq4_decode_mq_workspace_bytes(1, 4, 24, 4, 262144) > \
+        T.tbq4_decode_workspace_bytes(1, 24, 4, 262144)
+    assert T.tbq4_decode_mq_workspace_bytes(0, 4, 24, 4, 100) == 0
