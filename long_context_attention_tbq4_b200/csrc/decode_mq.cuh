@@ -71,7 +71,8 @@ constexpr int kOffFlags = kOffQPar + kCols * 2 * 4;               // [2][16] int
 constexpr int kOffXch = kOffFlags + 2 * kSoftWarps * 4;           // [4][32] floats
 constexpr int kOffXfin = kOffXch + 4 * kCols * 4;                 // [4][64] floats
 constexpr int kOffBar = kOffXfin + 4 * 2 * kCols * 4;
-constexpr int kNumBars = 2 * kRawStages + 5 * 2 + 4;    // + 2 vote, max, final
+constexpr int kSoftGroups = kSoftWarps / 4;            // warpgroups, 8 query rows each
+constexpr int kNumBars = 2 * kRawStages + 5 * 2 + 3 * kSoftGroups + 1;   // + vote, max per group, final
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffTmemPtr + 16 + 1024;     // + alignment slack
 static_assert(kOffBuf % 1024 == 0 && kOffRaw % 16 == 0 && kOffBar % 8 == 0, "align");
@@ -181,10 +182,12 @@ decode_mq_kernel(const AttnParams p) {
     auto p_full = [&](int b) { return bx + 8 * (6 + b); };     // P' written -> MMA
     auto tile_free = [&](int b) { return bx + 8 * (8 + b); };  // PV done -> buffer free
     // Exchanges between warps of one role use mbarriers with bounded waits
-    // (a warp that gives up on a wait must not leave the others blocked).
-    auto vote = [&](int b) { return bx + 8 * (10 + b); };      // softmax: grow flags
-    const uint32_t mx_bar = bx + 8 * 12;                        // softmax: tile maxima
-    const uint32_t fin_bar = bx + 8 * 13;                       // softmax: final sums
+    // (a warp that gives up on a wait must not leave the others blocked).  A
+    // softmax warpgroup owns its query rows, so its running maxima are agreed
+    // among its own four warps.
+    auto vote = [&](int b, int wgi) { return bx + 8 * (10 + 2 * wgi + b); };   // grow flags
+    auto mx_bar = [&](int wgi) { return bx + 8 * (10 + 2 * kSoftGroups + wgi); }; // tile maxima
+    const uint32_t fin_bar = bx + 8 * (10 + 3 * kSoftGroups);                 // final sums
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + kOffTmemPtr);
     float *qpar = reinterpret_cast<float *>(smem + kOffQPar);
 
@@ -199,9 +202,9 @@ decode_mq_kernel(const AttnParams p) {
             tc::bar_init(s_empty(b), kSoftWarps);
             tc::bar_init(p_full(b), kSoftWarps);
             tc::bar_init(tile_free(b), 1);
-            tc::bar_init(vote(b), kSoftWarps);
+            for (int w = 0; w < kSoftGroups; ++w) tc::bar_init(vote(b, w), 4);
         }
-        tc::bar_init(mx_bar, kSoftWarps);
+        for (int w = 0; w < kSoftGroups; ++w) tc::bar_init(mx_bar(w), 4);
         tc::bar_init(fin_bar, kSoftWarps);
         tc::fence_barrier_init();
     }
@@ -468,6 +471,11 @@ decode_mq_kernel(const AttnParams p) {
             __syncwarp();
             if (lane == 0) tc::bar_arrive(s_empty(b));
 
+            if (8 * wg >= NQ) {                 // no query row of this warpgroup is in use
+                __syncwarp();
+                if (lane == 0) tc::bar_arrive(p_full(b));
+                continue;
+            }
             const float *sig = reinterpret_cast<const float *>(smem + kOffBuf + b * kBufBytes + kSig);
             const int32_t ta = t0 + j * kTile + t;            // absolute token
             const float sk = sig[t], sv = ta < t1 ? sig[kTile + t] : 0.f;
@@ -486,11 +494,11 @@ decode_mq_kernel(const AttnParams p) {
             const bool wgrow = __any_sync(kFull, grow);
             if (lane == 0) flags[kSoftWarps * b + ws] = wgrow ? 1 : 0;
             __syncwarp();
-            if (lane == 0) tc::bar_arrive(vote(b));
-            if (!tc::bar_wait_warp(vote(b), par, kSpin)) { record_status(7u); ok = false; break; }
+            if (lane == 0) tc::bar_arrive(vote(b, wg));
+            if (!tc::bar_wait_warp(vote(b, wg), par, kSpin)) { record_status(7u); ok = false; break; }
             int any = 0;
 #pragma unroll
-            for (int w = 0; w < kSoftWarps; ++w) any |= flags[kSoftWarps * b + w];
+            for (int w = 0; w < 4; ++w) any |= flags[kSoftWarps * b + 4 * wg + w];
             if (any) {
                 // move the maxima to the tile's (where larger) and rescale
                 float lg[8];
@@ -501,8 +509,8 @@ decode_mq_kernel(const AttnParams p) {
                     if (lane == 0) xch[kCols * q4 + 8 * wg + k] = wm;
                 }
                 __syncwarp();
-                if (lane == 0) tc::bar_arrive(mx_bar);
-                if (!tc::bar_wait_warp(mx_bar, mx_phase, kSpin)) { record_status(7u); ok = false; break; }
+                if (lane == 0) tc::bar_arrive(mx_bar(wg));
+                if (!tc::bar_wait_warp(mx_bar(wg), mx_phase, kSpin)) { record_status(7u); ok = false; break; }
                 mx_phase ^= 1u;
                 uint32_t cs[8];
 #pragma unroll
