@@ -50,7 +50,8 @@ constexpr int kQBits = 18;                                 // |q_int| <= 2^18
 
 static_assert(kStageBytes % 16 == 0, "stage must keep 16-byte alignment");
 constexpr float kLazyRescale = 8.0f;                       // log2 units
-static_assert(kRingBytes >= kTcWarps * kMaxGroup * kD * 4 + 2 * kTcWarps * kMaxGroup * 4,
+static_assert(kRingBytes >= kTcWarps * kMaxGroup * kD * 4 + 3 * kTcWarps * kMaxGroup * 4 +
+                                kMaxGroup * 8,
               "merge buffers reuse the ring");
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -563,25 +564,36 @@ decode_tc_kernel(const AttnParams p) {
         l_w[warp * kMaxGroup + 2 * c + 1] = l_b;
     }
     __syncthreads();
-    // thread = (head, dim), kTcWarps * 32 / 128 heads at a time; levels carry a factor 15
-    const int d = threadIdx.x & (kD - 1);
-    for (int h = threadIdx.x >> 7; h < G; h += kTcWarps * 32 / kD) {
+    // per-(warp, head) weights 2^(m_w - M_h) and each head's (M, L), once:
+    // lane h of warp 0
+    float *wt = l_w + kTcWarps * kMaxGroup;                              // [W][8]
+    float2 *ml_h = reinterpret_cast<float2 *>(wt + kTcWarps * kMaxGroup);  // [8]
+    if (warp == 0 && lane < G) {
+        const int h = lane;
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kTcWarps; ++w) M = fmaxf(M, m_w[w * kMaxGroup + h]);
-        float O = 0.f, L = 0.f;
-        if (M != -INFINITY) {
+        float L = 0.f;
 #pragma unroll
-            for (int w = 0; w < kTcWarps; ++w) {
-                const float mw = m_w[w * kMaxGroup + h];
-                const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
-                O += f * o_w[(w * kMaxGroup + h) * kD + d];
-                L += f * l_w[w * kMaxGroup + h];
-            }
+        for (int w = 0; w < kTcWarps; ++w) {
+            const float mw = m_w[w * kMaxGroup + h];
+            const float f = (mw == -INFINITY || M == -INFINITY) ? 0.f : exp2f(mw - M);
+            wt[w * kMaxGroup + h] = f;
+            L = fmaf(f, l_w[w * kMaxGroup + h], L);
         }
+        ml_h[h] = make_float2(M, L);
+    }
+    __syncthreads();
+    // thread = (head, dim), kTcWarps * 32 / 128 heads at a time; levels carry a factor 15
+    const int d = threadIdx.x & (kD - 1);
+    for (int h = threadIdx.x >> 7; h < G; h += kTcWarps * 32 / kD) {
+        float O = 0.f;
+#pragma unroll
+        for (int w = 0; w < kTcWarps; ++w)
+            O = fmaf(wt[w * kMaxGroup + h], o_w[(w * kMaxGroup + h) * kD + d], O);
         const int64_t row = ((int64_t)s * p.Hq + g * G + h) * p.n_splits + split;
         p.part_o[row * kD + d] = O * (256.0f / 15.0f);     // 2^8 undoes the scale of P-prime
-        if (d == 0) p.part_ml[row] = make_float2(M, L);
+        if (d == 0) p.part_ml[row] = ml_h[h];
     }
 }
 
