@@ -157,14 +157,16 @@ decode_combine_kernel(const AttnParams p) {
     __shared__ float4 o_s[kCombineWarps * 32];
     __shared__ float m_s[kCombineWarps], l_s[kCombineWarps];
     __shared__ float w_s[kCombineWarps * kCombineFast];
-    // Launched as a programmatic dependent of the split kernel: wait for all
-    // of its partials (a no-op under an ordinary launch).
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int h = blockIdx.x, s = blockIdx.y;
+    // The lengths are an input of the split kernel, not one of its results,
+    // so they are read before the wait and only the partials' loads follow it.
     const int32_t len = seq_length(p, p.q_len > 1 ? s / p.q_len : s);
     const int used = used_splits(p, len);
     const int64_t row0 = ((int64_t)s * p.Hq + h) * p.n_splits;
+    // Launched as a programmatic dependent of the split kernel: wait for all
+    // of its partials (a no-op under an ordinary launch).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (used > kCombineWarps * kCombineFast) {
         float4 O;

@@ -50,7 +50,7 @@ constexpr int kQBits = 18;                                 // |q_int| <= 2^18
 
 static_assert(kStageBytes % 16 == 0, "stage must keep 16-byte alignment");
 constexpr float kLazyRescale = 8.0f;                       // log2 units
-static_assert(kRingBytes >= kTcWarps * kMaxGroup * kD * 4 + 3 * kTcWarps * kMaxGroup * 4 +
+static_assert(kRingBytes >= kTcWarps * 32 * 36 * 4 + 3 * kTcWarps * kMaxGroup * 4 +
                                 kMaxGroup * 8,
               "merge buffers reuse the ring");
 
@@ -228,7 +228,7 @@ decode_tc_kernel(const AttnParams p) {
         const int w = lane;
         for (int st = 0; st < kTcStages; ++st) mbar_init(smem_u32(bars) + (w * kTcStages + st) * 8, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        if (w < n_chunks_max) issue_for(w, w, 0, t1_max);   // stage 0 now, 1 and 2 after q
+        if (w < n_chunks_max) issue_for(w, w, 0, t1_max);   // stage 0 now, the others later
     }
     // queue of the chunks in stages st, st+1, st+2 (mod 3); -1: none
     int q0 = warp < n_chunks_max ? warp : -1;
@@ -301,16 +301,14 @@ decode_tc_kernel(const AttnParams p) {
     // per-head constants for this thread's score columns (heads 2c, 2c+1)
     const float f2a = qpar[4 * c + 0], bha = qpar[4 * c + 1];
     const float f2b = qpar[4 * c + 2], bhb = qpar[4 * c + 3];
-    // The rest of the first copies, after q: issued together with stage 0
-    // they would be served interleaved with it, and every warp's first chunk
-    // would land only near the end of the whole burst.
-    if (warp == kTcWarps - 1 && lane < kTcWarps) {
-        for (int st = 1; st < kTcStages; ++st) {
-            const int ci = lane + st * kTcWarps;
-            if (ci < n_chunks_max) issue_for(lane, ci, st, t1_max);
-            __syncwarp((1u << kTcWarps) - 1);
-        }
-    }
+    // The rest of the first copies go out later: issued together with stage
+    // 0 they would be served interleaved with it, so every warp's first chunk
+    // would land only near the end of the whole burst; and cp.async.bulk
+    // stalls the issuing thread while the copies before it are queued.  So
+    // each warp issues its own stage 1 now and its stage 2 once its first
+    // chunk has been consumed.
+    bool stage2_pending = true;
+    if (lane == 0 && warp + kTcWarps < n_chunks_max) issue_for(warp, warp + kTcWarps, 1, t1_max);
 
 
     // Loop-invariant byte offsets inside a stage.  K: rows r (+8, +16, +24)
@@ -516,6 +514,10 @@ decode_tc_kernel(const AttnParams p) {
         }
 
         __syncwarp();
+        if (stage2_pending) {                 // first chunk: the deferred stage 2
+            stage2_pending = false;
+            if (lane == 0 && q2 >= 0) issue(q2, 2, t1_max);
+        }
         int nxt = q2 >= 0 ? q2 + kTcWarps : -1;
         if (nxt >= n_chunks) nxt = -1;
         if (lane == 0 && nxt >= 0) issue(nxt, st, t1);
@@ -526,11 +528,12 @@ decode_tc_kernel(const AttnParams p) {
     }
 
     // Every copy still queued (issued ahead for chunks beyond the real
-    // length, or left by an aborted loop) lands before the ring is reused.
+    // length, or left by an aborted loop) lands before the ring is reused;
+    // with no chunk consumed, the deferred stage 2 was never issued.
 #pragma unroll
     for (int j = 0; j < kTcStages; ++j) {
         const int qj = j == 0 ? q0 : (j == 1 ? q1 : q2);
-        if (qj < 0) continue;
+        if (qj < 0 || (j == 2 && stage2_pending)) continue;
         int sj = st + j;
         uint32_t par = phase;
         if (sj >= kTcStages) { sj -= kTcStages; par ^= 1u; }
@@ -545,17 +548,24 @@ decode_tc_kernel(const AttnParams p) {
     }
     if (aborted) { m_a = m_b = -INFINITY; }
     __syncthreads();     // every warp is done with its ring
-    float *o_w = reinterpret_cast<float *>(ring);                       // [W][8][128]
-    float *m_w = o_w + kTcWarps * kMaxGroup * kD;                        // [W][8]
+    // Each lane's 32 accumulators go out as eight 16-byte stores to its own
+    // row of 36 floats (eight lanes per wavefront, no bank conflicts): (head
+    // h, dim d) is element 2 (d % 16) + h % 2 of fragment lane 4 (d / 16) + h / 2.
+    constexpr int kLaneStride = 36;
+    float *o_w = reinterpret_cast<float *>(ring);                       // [W][32][36]
+    float *m_w = o_w + kTcWarps * 32 * kLaneStride;                      // [W][8]
     float *l_w = m_w + kTcWarps * kMaxGroup;                             // [W][8]
-    // sum_t P'_t (2n - 15) = 2^11 sum_t P'_t (n - 8) 2^-10 + sum_t P'_t
+    float *wt = l_w + kTcWarps * kMaxGroup;                              // [W][8]
+    float2 *ml_h = reinterpret_cast<float2 *>(wt + kTcWarps * kMaxGroup);  // [8]
+    {
+        // sum_t P'_t (2n - 15) = 2^11 sum_t P'_t (n - 8) 2^-10 + sum_t P'_t
+        float4 *mine = reinterpret_cast<float4 *>(o_w + (warp * 32 + lane) * kLaneStride);
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-        const int d0 = 16 * r + 2 * mt;
-        o_w[(warp * kMaxGroup + 2 * c) * kD + d0] = fmaf(kVLevelScale, o[mt][0], rr[0]);
-        o_w[(warp * kMaxGroup + 2 * c + 1) * kD + d0] = fmaf(kVLevelScale, o[mt][1], rr[1]);
-        o_w[(warp * kMaxGroup + 2 * c) * kD + d0 + 1] = fmaf(kVLevelScale, o[mt][2], rr[2]);
-        o_w[(warp * kMaxGroup + 2 * c + 1) * kD + d0 + 1] = fmaf(kVLevelScale, o[mt][3], rr[3]);
+        for (int mt = 0; mt < 8; ++mt)
+            mine[mt] = make_float4(fmaf(kVLevelScale, o[mt][0], rr[0]),
+                                   fmaf(kVLevelScale, o[mt][1], rr[1]),
+                                   fmaf(kVLevelScale, o[mt][2], rr[2]),
+                                   fmaf(kVLevelScale, o[mt][3], rr[3]));
     }
     if (r == 0) {
         m_w[warp * kMaxGroup + 2 * c] = m_a;
@@ -564,36 +574,47 @@ decode_tc_kernel(const AttnParams p) {
         l_w[warp * kMaxGroup + 2 * c + 1] = l_b;
     }
     __syncthreads();
-    // per-(warp, head) weights 2^(m_w - M_h) and each head's (M, L), once:
-    // lane h of warp 0
-    float *wt = l_w + kTcWarps * kMaxGroup;                              // [W][8]
-    float2 *ml_h = reinterpret_cast<float2 *>(wt + kTcWarps * kMaxGroup);  // [8]
-    if (warp == 0 && lane < G) {
-        const int h = lane;
+    // per-(warp, head) weights 2^(m_w - M_h) and each head's (M, L), in warp
+    // 0: lane = (quarter wq of the warps, head h)
+    if (warp == 0) {
+        const int h = lane & 7, wq = lane >> 3;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kTcWarps; ++w) M = fmaxf(M, m_w[w * kMaxGroup + h]);
+        for (int k = 0; k < kTcWarps / 4; ++k)
+            M = fmaxf(M, m_w[(wq * (kTcWarps / 4) + k) * kMaxGroup + h]);
+        M = fmaxf(M, __shfl_xor_sync(kFull, M, 8));
+        M = fmaxf(M, __shfl_xor_sync(kFull, M, 16));
         float L = 0.f;
 #pragma unroll
-        for (int w = 0; w < kTcWarps; ++w) {
-            const float mw = m_w[w * kMaxGroup + h];
+        for (int k = 0; k < kTcWarps / 4; ++k) {
+            const int i = (wq * (kTcWarps / 4) + k) * kMaxGroup + h;
+            const float mw = m_w[i];
             const float f = (mw == -INFINITY || M == -INFINITY) ? 0.f : exp2f(mw - M);
-            wt[w * kMaxGroup + h] = f;
-            L = fmaf(f, l_w[w * kMaxGroup + h], L);
+            wt[i] = f;
+            L = fmaf(f, l_w[i], L);
         }
-        ml_h[h] = make_float2(M, L);
+        L += __shfl_xor_sync(kFull, L, 8);
+        L += __shfl_xor_sync(kFull, L, 16);
+        if (wq == 0) ml_h[h] = make_float2(M, L);
     }
     __syncthreads();
-    // thread = (head, dim), kTcWarps * 32 / 128 heads at a time; levels carry a factor 15
-    const int d = threadIdx.x & (kD - 1);
-    for (int h = threadIdx.x >> 7; h < G; h += kTcWarps * 32 / kD) {
-        float O = 0.f;
+    // One warp per (16-dim block rb, head pair cb): lane 2 j + k holds head
+    // 2 cb + k, dim 16 rb + j, which is element `lane` of fragment lane
+    // 4 rb + cb, so the 32 loads of a warp hit 32 different banks.  The
+    // levels carry a factor 15.
+    for (int it = warp; it < 8 * ((G + 1) >> 1); it += kTcWarps) {
+        const int rb = it & 7, cb = it >> 3;
+        const int h = 2 * cb + (lane & 1), d = 16 * rb + (lane >> 1);
+        if (h < G) {
+            const float *src = o_w + (4 * rb + cb) * kLaneStride + lane;
+            float O = 0.f;
 #pragma unroll
-        for (int w = 0; w < kTcWarps; ++w)
-            O = fmaf(wt[w * kMaxGroup + h], o_w[(w * kMaxGroup + h) * kD + d], O);
-        const int64_t row = ((int64_t)s * p.Hq + g * G + h) * p.n_splits + split;
-        p.part_o[row * kD + d] = O * (256.0f / 15.0f);     // 2^8 undoes the scale of P-prime
-        if (d == 0) p.part_ml[row] = ml_h[h];
+            for (int w = 0; w < kTcWarps; ++w)
+                O = fmaf(wt[w * kMaxGroup + h], src[w * 32 * kLaneStride], O);
+            const int64_t row = ((int64_t)s * p.Hq + g * G + h) * p.n_splits + split;
+            p.part_o[row * kD + d] = O * (256.0f / 15.0f);     // 2^8 undoes the scale of P-prime
+            if (d == 0) p.part_ml[row] = ml_h[h];
+        }
     }
 }
 
