@@ -148,6 +148,54 @@ TBQ4_API tbq4_status tbq4_attn_decode_append(const float *q, const float *k_new,
                                              size_t ws_bytes, uint16_t *out, void *stream);
 
 /*
+ * Paged caches (block table).  Instead of one [B][Hkv][capacity][66] cache, K
+ * and V each live in a pool of pages shared by all sequences:
+ *   pool         device, uint8 [n_pages][Hkv][page_size][66], 16-byte aligned
+ *   block_table  device, int32 [B][max_pages]: token t of sequence b is row
+ *                t % page_size of page block_table[b][t / page_size]
+ *   page_size    tokens per page, a multiple of 32 (>= 32)
+ * A sequence can hold max_pages * page_size tokens.  The layout inside a
+ * page is the contiguous layout (tokens of one KV head back to back), so
+ * every 32-token chunk of a stream is one contiguous copy.  This is the
+ * paged variant of the page's fixed per-sequence KV cache for ragged batches
+ * (trefon.com, "Kontekst 262K na jednej RTX 4090", sections "Konfiguracja"
+ * and "Od czego zaczalem": the quantised K/V blocks read by the attention
+ * kernel).  The caller owns the pools and the table; pages need no
+ * initialisation before they are written.
+ *
+ * tbq4_quantize_append_paged: as tbq4_quantize_append, with positions
+ * mapped through the table.  A position at or past max_pages * page_size,
+ * or a page id outside [0, n_pages), skips that row and flags
+ * TBQ4_ERR_CAPACITY in the device status.
+ *
+ * tbq4_attn_decode_paged: as tbq4_attn_decode (k_new = v_new = NULL) or
+ * tbq4_attn_decode_append (both non-NULL, fp32 [B][Hkv][128], 16-byte
+ * aligned; the new rows are written into the pools at seq_lens[b] - 1),
+ * same arithmetic and the same result bit for bit.  Requires max_len <=
+ * max_pages * page_size; the table entries of pages holding real tokens
+ * (t < seq_lens[b]) must be in [0, n_pages).  Entries past a sequence's
+ * length are read only as hints and may hold anything; a bad entry within
+ * the length makes that chunk read page 0 and flags TBQ4_ERR_CAPACITY.
+ * The workspace size comes from tbq4_decode_workspace_bytes.
+ * Errors: TBQ4_ERR_NULL (a NULL pointer, or only one of k_new / v_new),
+ * TBQ4_ERR_ALIGN, TBQ4_ERR_SHAPE (page_size, max_pages, n_pages or the
+ * head counts), TBQ4_ERR_CAPACITY (max_len above the table's reach).
+ */
+TBQ4_API tbq4_status tbq4_quantize_append_paged(const float *src, int B, int n_new, int Hkv,
+                                                const int32_t *start_pos,
+                                                const int32_t *block_table, int max_pages,
+                                                int page_size, int64_t n_pages,
+                                                uint64_t sign_seed, uint8_t *pool, void *stream);
+TBQ4_API tbq4_status tbq4_attn_decode_paged(const float *q, const float *k_new,
+                                            const float *v_new, uint8_t *k_pool,
+                                            uint8_t *v_pool, const int32_t *block_table,
+                                            int max_pages, int page_size, int64_t n_pages,
+                                            const int32_t *seq_lens, int32_t max_len, int B,
+                                            int Hq, int Hkv, float softmax_scale,
+                                            uint64_t sign_seed, void *workspace,
+                                            size_t ws_bytes, uint16_t *out, void *stream);
+
+/*
  * Multi-query decode: q_len (1-4) new query tokens per sequence, as when a
  * model verifies speculative drafts (trefon.com, "Kontekst 262K na jednej RTX
  * 4090", section "Konfiguracja": up to 3 drafted tokens).  Query token i of

@@ -27,6 +27,7 @@ __all__ = [
     "tbq4_decode_mq_workspace_bytes", "tbq4_attn_decode_mq",
     "tbq4_prefill_workspace_bytes", "tbq4_attn_prefill_chunk",
     "tbq4_set_timing_events", "tbq4_get_device_status", "empty_cache",
+    "empty_pool", "tbq4_quantize_append_paged", "tbq4_attn_decode_paged",
 ]
 
 
@@ -144,6 +145,78 @@ def tbq4_attn_decode_append(q, k_new, v_new, k_cache, v_cache, seq_lens, max_len
         int(max_len), B, Hq, Hkv, cap, float(softmax_scale), C.c_uint64(sign_seed),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out),
         _stream(stream)), "tbq4_attn_decode_append")
+    return out
+
+
+def empty_pool(n_pages, n_kv_heads, page_size, device="cuda"):
+    """An uninitialised page pool [n_pages][Hkv][page_size][66] uint8
+    (page_size a multiple of 32)."""
+    return torch.empty((n_pages, n_kv_heads, page_size, BLOCK_BYTES), dtype=torch.uint8,
+                       device=device)
+
+
+def _pool_shape(pool, name):
+    _need(pool, torch.uint8, name, 4)
+    n_pages, Hkv, page_size, nb = pool.shape
+    if nb != BLOCK_BYTES:
+        raise ValueError(f"{name}: last dimension must be {BLOCK_BYTES}")
+    return n_pages, Hkv, page_size
+
+
+def tbq4_quantize_append_paged(src, start_pos, block_table, pool, sign_seed=0, stream=None):
+    """src fp32 [B][n_new][Hkv][128]; start_pos int32 [B]; block_table int32
+    [B][max_pages]; pool uint8 [n_pages][Hkv][page_size][66] (written)."""
+    _need(src, torch.float32, "src", 4)
+    _need(start_pos, torch.int32, "start_pos", 1)
+    _need(block_table, torch.int32, "block_table", 2)
+    n_pages, Hkv, page_size = _pool_shape(pool, "pool")
+    B, n_new, h, d = src.shape
+    if d != D or h != Hkv or block_table.shape[0] != B:
+        raise ValueError("shape mismatch between src, block_table and pool")
+    check(lib.tbq4_quantize_append_paged(
+        _ptr(src), B, n_new, Hkv, _ptr(start_pos), _ptr(block_table), block_table.shape[1],
+        page_size, n_pages, C.c_uint64(sign_seed), _ptr(pool), _stream(stream)),
+        "tbq4_quantize_append_paged")
+    return pool
+
+
+def tbq4_attn_decode_paged(q, k_pool, v_pool, block_table, seq_lens, max_len, softmax_scale,
+                           sign_seed=0, k_new=None, v_new=None, workspace=None, out=None,
+                           stream=None):
+    """Decode attention over paged caches: q fp32 [B][Hq][128]; pools uint8
+    [n_pages][Hkv][page_size][66]; block_table int32 [B][max_pages]; with
+    k_new / v_new (fp32 [B][Hkv][128]) the step's rows are written at
+    seq_lens[b]-1 first.  Returns fp16 [B][Hq][128]."""
+    _need(q, torch.float32, "q", 3)
+    _need(block_table, torch.int32, "block_table", 2)
+    _need(seq_lens, torch.int32, "seq_lens", 1)
+    n_pages, Hkv, page_size = _pool_shape(k_pool, "k_pool")
+    if v_pool.shape != k_pool.shape:
+        raise ValueError("k_pool and v_pool differ in shape")
+    _pool_shape(v_pool, "v_pool")
+    B, Hq, d = q.shape
+    if d != D or block_table.shape[0] != B:
+        raise ValueError("shape mismatch between q, block_table and pools")
+    if (k_new is None) != (v_new is None):
+        raise ValueError("give both k_new and v_new, or neither")
+    if k_new is not None:
+        _need(k_new, torch.float32, "k_new", 3)
+        _need(v_new, torch.float32, "v_new", 3)
+        if tuple(k_new.shape) != (B, Hkv, D) or tuple(v_new.shape) != (B, Hkv, D):
+            raise ValueError("k_new / v_new must be [B][Hkv][128]")
+    need = tbq4_decode_workspace_bytes(B, Hq, Hkv, max_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float16, device=q.device)
+    _need(out, torch.float16, "out", 3)
+    check(lib.tbq4_attn_decode_paged(
+        _ptr(q), _ptr(k_new) if k_new is not None else None,
+        _ptr(v_new) if v_new is not None else None, _ptr(k_pool), _ptr(v_pool),
+        _ptr(block_table), block_table.shape[1], page_size, n_pages, _ptr(seq_lens),
+        int(max_len), B, Hq, Hkv, float(softmax_scale), C.c_uint64(sign_seed), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)),
+        "tbq4_attn_decode_paged")
     return out
 
 

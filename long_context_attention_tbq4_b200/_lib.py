@@ -23,6 +23,9 @@ SIGNATURES = {
                               _p, _sz, _p, _p]),
     "tbq4_attn_decode_append": (_i, [_p, _p, _p, _p, _p, _p, _i32, _i, _i, _i, _i64, _f,
                                      _u64, _p, _sz, _p, _p]),
+    "tbq4_quantize_append_paged": (_i, [_p, _i, _i, _i, _p, _p, _i, _i, _i64, _u64, _p, _p]),
+    "tbq4_attn_decode_paged": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i64, _p, _i32, _i, _i, _i,
+                                    _f, _u64, _p, _sz, _p, _p]),
     "tbq4_decode_workspace_bytes_split": (_sz, [_i, _i, _i, _i32, _i32]),
     "tbq4_decode_mq_workspace_bytes": (_sz, [_i, _i, _i, _i, _i32]),
     "tbq4_attn_decode_mq": (_i, [_p, _p, _p, _p, _i32, _i, _i, _i, _i, _i64, _f, _u64, _p, _sz,

@@ -44,7 +44,28 @@ struct AttnParams {
     const float *v_new;
     uint8_t *k_wr;              // the same caches as k / v, written
     uint8_t *v_wr;
+    // Paged caches: k and v are pools [n_pages][Hkv][page_size][66] and
+    // token t of sequence s lives in page block_table[s][t / page_size], row
+    // t % page_size.  nullptr: contiguous caches (seq_stride, head_stride).
+    const int32_t *block_table;
+    int max_pages;              // row length of block_table
+    int page_size;              // tokens per page, a multiple of 32
+    int64_t n_pages;
 };
+
+// Byte offset of token t of (sequence s, KV head g) in a paged pool.  An
+// out-of-range page id reads page 0 instead (so no access leaves the pool);
+// *bad reports it, for the caller to flag when the token is a real one.
+__device__ __forceinline__ int64_t paged_offset(const AttnParams &p, int32_t pid, int g, int32_t t,
+                                                bool *bad) {
+    *bad = pid < 0 || (int64_t)pid >= p.n_pages;
+    if (*bad) pid = 0;
+    return (((int64_t)pid * p.Hkv + g) * p.page_size + t % p.page_size) * kBlockBytes;
+}
+
+__device__ __forceinline__ int32_t page_id(const AttnParams &p, int s, int32_t t) {
+    return __ldg(p.block_table + (int64_t)s * p.max_pages + t / p.page_size);
+}
 
 __device__ __forceinline__ int32_t seq_length(const AttnParams &p, int s) {
     int32_t len = p.seq_lens ? __ldg(p.seq_lens + s) : p.len_base + s;

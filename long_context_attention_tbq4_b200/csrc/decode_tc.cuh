@@ -176,6 +176,8 @@ __device__ __forceinline__ void split3(int x, int8_t &c0, int8_t &c1, int8_t &c2
     c2 = (int8_t)((x1 - b1) >> 8);
 }
 
+// kPaged: the caches are page pools addressed through p.block_table.
+template <bool kPaged>
 __global__ void __launch_bounds__(kTcWarps * 32, 1)
 decode_tc_kernel(const AttnParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -204,14 +206,28 @@ decode_tc_kernel(const AttnParams p) {
     // ---- per-warp ring: the first copies go out before the q prologue -----
     uint8_t *ring_p = ring + warp * kWarpRing;
     const uint32_t bar_w = smem_u32(bars) + warp * kTcStages * 8;
-    const uint8_t *kb = p.k + s * p.seq_stride + g * p.head_stride;
-    const uint8_t *vb = p.v + s * p.seq_stride + g * p.head_stride;
+    const uint8_t *kb = kPaged ? p.k : p.k + s * p.seq_stride + g * p.head_stride;
+    const uint8_t *vb = kPaged ? p.v : p.v + s * p.seq_stride + g * p.head_stride;
     // Warp w takes chunks w, w + 16, w + 32, ... of the split (fixed, so the
-    // result does not depend on timing).
+    // result does not depend on timing).  A chunk never crosses a page (the
+    // page size is a multiple of 32 tokens and so is t0).
 
-    // The last warp (never a q warp) initialises every warp's barriers and
-    // issues every warp's first chunk, so the q warps start on q at once.
-    auto issue_for = [&](int w, int ci, int st, int32_t tend) {   // chunk ci -> warp w, stage st
+    // page id of chunk ci (paged), and the chunk's byte offset from kb / vb
+    auto pid_of = [&](int ci) -> int32_t {
+        if constexpr (kPaged) return page_id(p, s, t0 + ci * kChunk);
+        else return 0;
+    };
+    auto chunk_ofs = [&](int ci, int32_t pid, bool *bad) -> int64_t {
+        const int32_t start = t0 + ci * kChunk;
+        if constexpr (kPaged) {
+            return paged_offset(p, pid, g, start, bad);
+        } else {
+            *bad = false;
+            return (int64_t)start * kBlockBytes;
+        }
+    };
+    // chunk ci -> warp w, stage st; ofs from chunk_ofs
+    auto issue_for = [&](int w, int ci, int st, int32_t tend, int64_t ofs) {
         const int32_t start = t0 + ci * kChunk;
         const int32_t valid = min(kChunk, tend - start);
         const uint32_t bytes = (uint32_t)((valid + 7) & ~7) * kBlockBytes;
@@ -219,24 +235,37 @@ decode_tc_kernel(const AttnParams p) {
         const uint32_t dst = smem_u32(ring) + w * kWarpRing + st * kStageBytes;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_expect_tx(bar, 2 * bytes);
-        bulk_g2s(dst, kb + (int64_t)start * kBlockBytes, bytes, bar);
-        bulk_g2s(dst + kChunkBytes, vb + (int64_t)start * kBlockBytes, bytes, bar);
+        bulk_g2s(dst, kb + ofs, bytes, bar);
+        bulk_g2s(dst + kChunkBytes, vb + ofs, bytes, bar);
     };
-    auto issue = [&](int ci, int st, int32_t tend) { issue_for(warp, ci, st, tend); };
+    auto issue = [&](int ci, int st, int32_t tend, int64_t ofs) { issue_for(warp, ci, st, tend, ofs); };
+    // The last warp (never a q warp) initialises every warp's barriers and
+    // issues every warp's first chunk, so the q warps start on q at once.
     static_assert(kTcWarps <= 32 && kMaxGroup < kTcWarps, "one issuing lane per warp");
+    bool bad0 = false;      // paged: lane w of the last warp, chunk w's page id
     if (warp == kTcWarps - 1 && lane < kTcWarps) {
         const int w = lane;
         for (int st = 0; st < kTcStages; ++st) mbar_init(smem_u32(bars) + (w * kTcStages + st) * 8, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        if (w < n_chunks_max) issue_for(w, w, 0, t1_max);   // stage 0 now, the others later
+        if (w < n_chunks_max)                               // stage 0 now, the others later
+            issue_for(w, w, 0, t1_max, chunk_ofs(w, pid_of(w), &bad0));
     }
     // queue of the chunks in stages st, st+1, st+2 (mod 3); -1: none
     int q0 = warp < n_chunks_max ? warp : -1;
     int q1 = warp + kTcWarps < n_chunks_max ? warp + kTcWarps : -1;
     int q2 = warp + 2 * kTcWarps < n_chunks_max ? warp + 2 * kTcWarps : -1;
+    // paged: the page ids of the next copies, loaded well before their use
+    int32_t pid1 = 0, pid2 = 0, pid_n = 0;
+    if (kPaged && lane == 0) {
+        if (q1 >= 0) pid1 = pid_of(q1);
+        if (q2 >= 0) pid2 = pid_of(q2);
+        if (q2 >= 0 && q2 + kTcWarps < n_chunks_max) pid_n = pid_of(q2 + kTcWarps);
+    }
     const int32_t len = seq_length(p, s);
     const int32_t t1 = min(len, t1_max);
     const int n_chunks = t1 > t0 ? (t1 - t0 + kChunk - 1) / kChunk : 0;
+    // a bad page id is an error only where the chunk holds real tokens
+    if (kPaged && bad0 && lane < n_chunks) record_status(4u /* TBQ4_ERR_CAPACITY */);
 
     // ---- q: rotate, normalise by a power of two, 18-bit integer ----------
     // q_int = rint(q_rot * 2^(18-e)) with 2^e > max|q_rot|, so |q_int| <= 2^18.
@@ -308,7 +337,12 @@ decode_tc_kernel(const AttnParams p) {
     // each warp issues its own stage 1 now and its stage 2 once its first
     // chunk has been consumed.
     bool stage2_pending = true;
-    if (lane == 0 && warp + kTcWarps < n_chunks_max) issue_for(warp, warp + kTcWarps, 1, t1_max);
+    if (lane == 0 && q1 >= 0) {
+        bool bad;
+        const int64_t o = chunk_ofs(q1, pid1, &bad);
+        if (bad && q1 < n_chunks) record_status(4u);
+        issue(q1, 1, t1_max, o);
+    }
 
 
     // Loop-invariant byte offsets inside a stage.  K: rows r (+8, +16, +24)
@@ -358,7 +392,13 @@ decode_tc_kernel(const AttnParams p) {
             const int jn = len - 1 - cstart;
             const uint32_t sbits = lane_sign_bits(p.sign_lo, p.sign_hi, lane);
             const int64_t row = ((int64_t)s * p.Hkv + g) * kD;
-            const int64_t gofs = s * p.seq_stride + g * p.head_stride + (int64_t)(len - 1) * kBlockBytes;
+            bool gbad = false;
+            int64_t gofs;
+            if constexpr (kPaged)
+                gofs = paged_offset(p, page_id(p, s, len - 1), g, len - 1, &gbad);
+            else
+                gofs = s * p.seq_stride + g * p.head_stride + (int64_t)(len - 1) * kBlockBytes;
+            if (gbad && lane == 0) record_status(4u);
 #pragma unroll
             for (int kv = 0; kv < 2; ++kv) {
                 const float4 x4 = reinterpret_cast<const float4 *>((kv ? p.v_new : p.k_new) + row)[lane];
@@ -368,10 +408,10 @@ decode_tc_kernel(const AttnParams p) {
                 uint8_t *sa = (kv ? vst : kst) + jn * kBlockBytes;
                 uint8_t *ga = (kv ? p.v_wr : p.k_wr) + gofs;
                 reinterpret_cast<uint16_t *>(sa + 2)[lane] = (uint16_t)packed;
-                reinterpret_cast<uint16_t *>(ga + 2)[lane] = (uint16_t)packed;
+                if (!gbad) reinterpret_cast<uint16_t *>(ga + 2)[lane] = (uint16_t)packed;
                 if (lane == 0) {
                     *reinterpret_cast<uint16_t *>(sa) = sb;
-                    *reinterpret_cast<uint16_t *>(ga) = sb;
+                    if (!gbad) *reinterpret_cast<uint16_t *>(ga) = sb;
                 }
             }
             __syncwarp();
@@ -516,11 +556,22 @@ decode_tc_kernel(const AttnParams p) {
         __syncwarp();
         if (stage2_pending) {                 // first chunk: the deferred stage 2
             stage2_pending = false;
-            if (lane == 0 && q2 >= 0) issue(q2, 2, t1_max);
+            if (lane == 0 && q2 >= 0) {
+                bool bad;
+                const int64_t o = chunk_ofs(q2, pid2, &bad);
+                if (bad && q2 < n_chunks) record_status(4u);
+                issue(q2, 2, t1_max, o);
+            }
         }
         int nxt = q2 >= 0 ? q2 + kTcWarps : -1;
         if (nxt >= n_chunks) nxt = -1;
-        if (lane == 0 && nxt >= 0) issue(nxt, st, t1);
+        if (lane == 0 && nxt >= 0) {          // nxt < n_chunks: real tokens
+            bool bad;
+            const int64_t o = chunk_ofs(nxt, pid_n, &bad);
+            if (bad) record_status(4u);
+            issue(nxt, st, t1, o);
+            if (kPaged && nxt + kTcWarps < n_chunks) pid_n = pid_of(nxt + kTcWarps);
+        }
         q0 = q1;
         q1 = q2;
         q2 = nxt;

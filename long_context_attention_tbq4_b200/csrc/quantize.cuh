@@ -64,6 +64,15 @@ struct SignTable {
 // chunk c of row i at position c ^ (i % 8), so the per-thread reads of a
 // whole row are free of bank conflicts), and the 32 blocks go out from a
 // shared staging area as consecutive 16-bit pieces.
+// Paged destination: row (b, pos) goes to page table[b][pos / page_size],
+// row pos % page_size, of a pool [n_pages][Hkv][page_size][66].  A null
+// table means the contiguous cache [B][Hkv][capacity][66].
+struct PageMap {
+    const int32_t *table;
+    int max_pages, page_size;
+    int64_t n_pages;
+};
+
 constexpr int kQRows = 32;                                   // rows per warp and step
 constexpr int kQWarpBytes = kQRows * 512 + kQRows * kBlockBytes + kQRows * 8;
 constexpr int kQThreads = 128;
@@ -72,7 +81,7 @@ constexpr int kQSmemBytes = (kQThreads / 32) * kQWarpBytes;
 __global__ void __launch_bounds__(kQThreads, 3)
 quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
                      const int32_t *__restrict__ start_pos, int64_t capacity, const SignTable sg,
-                     uint8_t *__restrict__ cache) {
+                     const PageMap pm, uint8_t *__restrict__ cache) {
     extern __shared__ __align__(16) uint8_t qsm[];
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     uint8_t *wsm = qsm + wib * kQWarpBytes;
@@ -91,13 +100,19 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
         const uint32_t h = bh % (uint32_t)Hkv, b = bh / (uint32_t)Hkv;
         const float4 *srow =
             reinterpret_cast<const float4 *>(src + (((int64_t)b * n_new + t) * Hkv + h) * kD);
-        int64_t doff = -1;
+        int64_t doff = -1;          // -1: nothing stored (tail lane or bad position)
         if (live) {
             const int64_t pos = (int64_t)__ldg(start_pos + b) + t;
-            if (pos < 0 || pos >= capacity) record_status(4u /* TBQ4_ERR_CAPACITY */);
-            else doff = (((int64_t)b * Hkv + h) * capacity + pos) * kBlockBytes;
+            if (pos < 0 || pos >= capacity) {
+                record_status(4u /* TBQ4_ERR_CAPACITY */);
+            } else if (pm.table) {
+                const int32_t pid = __ldg(pm.table + (int64_t)b * pm.max_pages + pos / pm.page_size);
+                if (pid < 0 || (int64_t)pid >= pm.n_pages) record_status(4u);
+                else doff = (((int64_t)pid * Hkv + h) * pm.page_size + pos % pm.page_size) * kBlockBytes;
+            } else {
+                doff = (((int64_t)b * Hkv + h) * capacity + pos) * kBlockBytes;
+            }
         }
-        doffs[lane] = doff;
         // load: row i, one 16-byte chunk per lane
 #pragma unroll 8
         for (int i = 0; i < kQRows; ++i) {
@@ -162,6 +177,7 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
             }
             mine[1 + w] = (uint16_t)piece;
         }
+        doffs[lane] = doff;
         __syncwarp();
         // store: the 32 blocks as 1,056 consecutive 16-bit pieces
 #pragma unroll

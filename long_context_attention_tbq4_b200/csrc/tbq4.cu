@@ -123,17 +123,21 @@ tbq4_status run_attention(AttnParams p, void *workspace, size_t ws_bytes,
     p.n_splits = w.n_splits;
     p.part_o = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.part_o);
     p.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) + w.part_ml);
-    static bool attr_set[64] = {}, attr_mq[64] = {};    // set once per device
-    const bool mq = p.q_len > 1;
+    static bool attr_set[64] = {}, attr_paged[64] = {}, attr_mq[64] = {};  // once per device
+    const bool mq = p.q_len > 1, paged = p.block_table != nullptr;
+    if (mq && paged) return TBQ4_ERR_SHAPE;
     if (mq ? !ensure_smem_attr((const void *)dmq::decode_mq_kernel, dmq::kSmemBytes, attr_mq)
-           : !ensure_smem_attr((const void *)decode_tc_kernel, kTcSmemBytes, attr_set))
+           : paged ? !ensure_smem_attr((const void *)decode_tc_kernel<true>, kTcSmemBytes, attr_paged)
+                   : !ensure_smem_attr((const void *)decode_tc_kernel<false>, kTcSmemBytes, attr_set))
         return TBQ4_ERR_LAUNCH;
     dim3 g1(p.n_splits, p.Hkv, p.nseq);
     if (g_ev_before) cudaEventRecord(g_ev_before, st);
     if (mq)
         dmq::decode_mq_kernel<<<g1, dmq::kThreads, dmq::kSmemBytes, st>>>(p);
+    else if (paged)
+        decode_tc_kernel<true><<<g1, kTcWarps * 32, kTcSmemBytes, st>>>(p);
     else
-        decode_tc_kernel<<<g1, kTcWarps * 32, kTcSmemBytes, st>>>(p);
+        decode_tc_kernel<false><<<g1, kTcWarps * 32, kTcSmemBytes, st>>>(p);
     // The combine is a programmatic dependent launch: its CTAs are placed as
     // decode CTAs retire and wait in griddepcontrol.wait for the whole decode
     // grid, so no launch gap separates the two kernels.
@@ -195,9 +199,13 @@ void tbq4_signs(uint64_t seed, int8_t out[128]) {
     }
 }
 
-tbq4_status tbq4_quantize_append(const float *src, int B, int n_new, int Hkv,
-                                 const int32_t *start_pos, int64_t capacity,
-                                 uint64_t sign_seed, uint8_t *cache, void *stream) {
+}  // extern "C"
+
+namespace {
+
+tbq4_status quantize_impl(const float *src, int B, int n_new, int Hkv, const int32_t *start_pos,
+                          int64_t capacity, uint64_t sign_seed, const PageMap &pm,
+                          uint8_t *cache, void *stream) {
     if (!src || !start_pos || !cache) return TBQ4_ERR_NULL;
     if (!aligned(src, 16) || !aligned(cache, 16) || !aligned(start_pos, 4))
         return TBQ4_ERR_ALIGN;
@@ -216,8 +224,34 @@ tbq4_status tbq4_quantize_append(const float *src, int B, int n_new, int Hkv,
     int64_t blocks = ceil_div(rows, (int64_t)kQThreads);   // one row per thread
     if (blocks > (int64_t)kNumSMs * 3) blocks = (int64_t)kNumSMs * 3;
     quantize_rows_kernel<<<(unsigned)blocks, kQThreads, kQSmemBytes, (cudaStream_t)stream>>>(
-        src, B, n_new, Hkv, start_pos, capacity, sg, cache);
+        src, B, n_new, Hkv, start_pos, capacity, sg, pm, cache);
     return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+tbq4_status tbq4_quantize_append(const float *src, int B, int n_new, int Hkv,
+                                 const int32_t *start_pos, int64_t capacity,
+                                 uint64_t sign_seed, uint8_t *cache, void *stream) {
+    const PageMap contiguous = {nullptr, 0, 0, 0};
+    return quantize_impl(src, B, n_new, Hkv, start_pos, capacity, sign_seed, contiguous, cache,
+                         stream);
+}
+
+tbq4_status tbq4_quantize_append_paged(const float *src, int B, int n_new, int Hkv,
+                                       const int32_t *start_pos, const int32_t *block_table,
+                                       int max_pages, int page_size, int64_t n_pages,
+                                       uint64_t sign_seed, uint8_t *pool, void *stream) {
+    if (!block_table) return TBQ4_ERR_NULL;
+    if (!aligned(block_table, 4)) return TBQ4_ERR_ALIGN;
+    if (page_size < 32 || page_size % 32 != 0 || max_pages <= 0 || n_pages <= 0 ||
+        n_pages > 0x7FFFFFFFLL)
+        return TBQ4_ERR_SHAPE;
+    const PageMap pm = {block_table, max_pages, page_size, n_pages};
+    return quantize_impl(src, B, n_new, Hkv, start_pos, (int64_t)max_pages * page_size,
+                         sign_seed, pm, pool, stream);
 }
 
 size_t tbq4_decode_workspace_bytes_split(int B, int Hq, int Hkv, int32_t max_len,
@@ -236,13 +270,36 @@ size_t tbq4_decode_workspace_bytes(int B, int Hq, int Hkv, int32_t max_len) {
 
 namespace {
 
+// A block table and its pools (nullptr table: contiguous caches).
+struct PagedArgs {
+    const int32_t *block_table;
+    int max_pages, page_size;
+    int64_t n_pages;
+};
+
+// Checks a paged layout; sets *capacity to the tokens a table row can map.
+tbq4_status check_paged(const PagedArgs &pg, int64_t *capacity) {
+    if (!pg.block_table) return TBQ4_ERR_NULL;
+    if (!aligned(pg.block_table, 4)) return TBQ4_ERR_ALIGN;
+    if (pg.page_size < 32 || pg.page_size % 32 != 0 || pg.max_pages <= 0 || pg.n_pages <= 0 ||
+        pg.n_pages > 0x7FFFFFFFLL)
+        return TBQ4_ERR_SHAPE;
+    *capacity = (int64_t)pg.max_pages * pg.page_size;
+    return TBQ4_OK;
+}
+
 tbq4_status decode_impl(const float *q, const uint8_t *k_cache, const uint8_t *v_cache,
                         const int32_t *seq_lens, int32_t max_len, int B, int Hq, int Hkv,
                         int64_t capacity, float softmax_scale, uint64_t sign_seed,
                         int32_t split_tokens, void *workspace, size_t ws_bytes, uint16_t *out,
-                        void *stream, const float *k_new, const float *v_new) {
+                        void *stream, const float *k_new, const float *v_new,
+                        const PagedArgs *pg = nullptr) {
     if (!q || !k_cache || !v_cache || !seq_lens || !workspace || !out)
         return TBQ4_ERR_NULL;
+    if (pg) {
+        const tbq4_status e = check_paged(*pg, &capacity);
+        if (e != TBQ4_OK) return e;
+    }
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
         !aligned(workspace, kWsAlign) || !aligned(out, 2) || !aligned(seq_lens, 4))
         return TBQ4_ERR_ALIGN;
@@ -276,6 +333,14 @@ tbq4_status decode_impl(const float *q, const uint8_t *k_cache, const uint8_t *v
         p.v_new = v_new;
         p.k_wr = const_cast<uint8_t *>(k_cache);
         p.v_wr = const_cast<uint8_t *>(v_cache);
+    }
+    if (pg) {
+        p.head_stride = 0;
+        p.seq_stride = 0;
+        p.block_table = pg->block_table;
+        p.max_pages = pg->max_pages;
+        p.page_size = pg->page_size;
+        p.n_pages = pg->n_pages;
     }
     return run_attention(p, workspace, ws_bytes, (cudaStream_t)stream);
 }
@@ -353,6 +418,20 @@ tbq4_status tbq4_attn_decode_append(const float *q, const float *k_new, const fl
     return decode_impl(q, k_cache, v_cache, seq_lens, max_len, B, Hq, Hkv, capacity,
                        softmax_scale, sign_seed, 0, workspace, ws_bytes, out, stream, k_new,
                        v_new);
+}
+
+tbq4_status tbq4_attn_decode_paged(const float *q, const float *k_new, const float *v_new,
+                                   uint8_t *k_pool, uint8_t *v_pool, const int32_t *block_table,
+                                   int max_pages, int page_size, int64_t n_pages,
+                                   const int32_t *seq_lens, int32_t max_len, int B, int Hq,
+                                   int Hkv, float softmax_scale, uint64_t sign_seed,
+                                   void *workspace, size_t ws_bytes, uint16_t *out,
+                                   void *stream) {
+    if ((k_new == nullptr) != (v_new == nullptr)) return TBQ4_ERR_NULL;
+    if (k_new && (!aligned(k_new, 16) || !aligned(v_new, 16))) return TBQ4_ERR_ALIGN;
+    const PagedArgs pg = {block_table, max_pages, page_size, n_pages};
+    return decode_impl(q, k_pool, v_pool, seq_lens, max_len, B, Hq, Hkv, 0, softmax_scale,
+                       sign_seed, 0, workspace, ws_bytes, out, stream, k_new, v_new, &pg);
 }
 
 tbq4_status tbq4_attn_decode(const float *q, const uint8_t *k_cache,

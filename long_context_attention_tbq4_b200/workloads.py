@@ -178,3 +178,20 @@ def round_capacity(n, multiple=4096):
     minimum the page uses for fewer CUDA-graph recaptures: trefon.com,
     "Kontekst 262K na jednej RTX 4090", section 2)."""
     return ((int(n) + multiple - 1) // multiple) * multiple
+
+
+def page_table(seed, lens, page_size, spare=3, max_pages=None):
+    """A block table for paged caches: every sequence gets the pages its
+    length needs, drawn without replacement from a shuffled pool that has
+    `spare` unused pages; a row's unused tail is filled with -1.  Returns
+    (table int32 [B][max_pages], n_pages)."""
+    need = [(int(n) + page_size - 1) // page_size for n in lens]
+    width = max(max(need, default=0), 1) if max_pages is None else int(max_pages)
+    n_pages = sum(need) + spare
+    perm = np.random.default_rng(seed).permutation(n_pages).astype(np.int32)
+    table = np.full((len(lens), width), -1, np.int32)
+    at = 0
+    for b, k in enumerate(need):
+        table[b, :k] = perm[at:at + k]
+        at += k
+    return table, n_pages

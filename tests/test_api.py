@@ -181,3 +181,61 @@ def test_decode_mq_workspace_query(T):
     assert T.tbq4_decode_mq_workspace_bytes(1, 4, 24, 4, 262144) > \
         T.tbq4_decode_workspace_bytes(1, 24, 4, 262144)
     assert T.tbq4_decode_mq_workspace_bytes(0, 4, 24, 4, 100) == 0
+
+
+def test_paged_rejects_bad_arguments(T):
+    from long_context_attention_tbq4_b200._lib import lib as L
+
+    def d(**kw):
+        a = dict(q=A, kn=None, vn=None, k=A, v=A, table=A, max_pages=4, page=32, n_pages=8,
+                 lens=A, max_len=64, B=1, Hq=8, Hkv=2, scale=0.1, seed=0, ws=A2,
+                 ws_bytes=1 << 30, out=A, stream=None)
+        a.update(kw)
+        return L.tbq4_attn_decode_paged(a["q"], a["kn"], a["vn"], a["k"], a["v"], a["table"],
+                                        a["max_pages"], a["page"], a["n_pages"], a["lens"],
+                                        a["max_len"], a["B"], a["Hq"], a["Hkv"], a["scale"],
+                                        a["seed"], a["ws"], a["ws_bytes"], a["out"],
+                                        a["stream"])
+    assert d(table=None) == 1                         # TBQ4_ERR_NULL
+    assert d(kn=A) == 1                               # one new row without the other
+    assert d(k=None) == 1
+    assert d(table=C.c_void_p(0x10002)) == 2          # TBQ4_ERR_ALIGN
+    assert d(kn=C.c_void_p(0x10008), vn=A) == 2
+    assert d(page=48) == 3                            # TBQ4_ERR_SHAPE: not a multiple of 32
+    assert d(page=16) == 3
+    assert d(max_pages=0) == 3
+    assert d(n_pages=0) == 3
+    assert d(Hq=7) == 3
+    assert d(max_len=129) == 4                        # 4 pages of 32 reach 128 tokens
+    assert d(ws_bytes=16) == 5                        # TBQ4_ERR_WORKSPACE
+
+    def q(**kw):
+        a = dict(src=A, B=1, n=4, Hkv=2, pos=A, table=A, max_pages=4, page=32, n_pages=8,
+                 seed=0, pool=A, stream=None)
+        a.update(kw)
+        return L.tbq4_quantize_append_paged(a["src"], a["B"], a["n"], a["Hkv"], a["pos"],
+                                            a["table"], a["max_pages"], a["page"],
+                                            a["n_pages"], a["seed"], a["pool"], a["stream"])
+    assert q(table=None) == 1
+    assert q(pool=None) == 1
+    assert q(table=C.c_void_p(0x10001)) == 2
+    assert q(page=40) == 3
+    assert q(n_pages=0) == 3
+    assert q(n=0) == 0                                # nothing to do, nothing launched
+
+
+
+def test_page_table_generator():
+    """The seeded block tables the paged tests use: every page id at most
+    once, rows as long as their sequence needs, -1 past that."""
+    from long_context_attention_tbq4_b200 import workloads as W
+    lens = [0, 1, 32, 33, 1000]
+    table, n_pages = W.page_table(3, lens, 32, spare=2)
+    assert table.shape == (5, 32) and n_pages == 0 + 1 + 1 + 2 + 32 + 2
+    used = table[table >= 0]
+    assert len(used) == len(set(used.tolist())) == n_pages - 2
+    assert used.min() >= 0 and used.max() < n_pages
+    for b, n in enumerate(lens):
+        k = (n + 31) // 32
+        assert (table[b, :k] >= 0).all() and (table[b, k:] == -1).all()
+    assert np.array_equal(W.page_table(3, lens, 32, spare=2)[0], table)   # seeded
