@@ -45,6 +45,12 @@ constexpr int kRingBytes = kTcWarps * kWarpRing;
 constexpr int kBarBytes = kTcWarps * kTcStages * 8;
 constexpr int kQScratchBytes = 2 * 3 * kMaxGroup * 64 + 2 * kMaxGroup * 4;   // q pieces + constants
 constexpr int kTcSmemBytes = kRingBytes + kBarBytes + kQScratchBytes + 128;
+// Paged caches: the page id of every chunk of the split, copied into shared
+// memory during the q prologue (so no table load sits on the copy path).
+// Paged launches keep splits at or below kPidCap chunks.
+constexpr int kPidCap = 4096;
+constexpr int kTcSmemBytesPaged = kTcSmemBytes + kPidCap * 4;
+static_assert(kTcSmemBytesPaged <= 227 * 1024, "shared memory per CTA");
 constexpr uint32_t kSpinLimit = 1u << 22;                  // bounded mbarrier wait
 constexpr int kQBits = 18;                                 // |q_int| <= 2^18
 
@@ -212,18 +218,28 @@ decode_tc_kernel(const AttnParams p) {
     // result does not depend on timing).  A chunk never crosses a page (the
     // page size is a multiple of 32 tokens and so is t0).
 
-    // page id of chunk ci (paged), and the chunk's byte offset from kb / vb
-    auto pid_of = [&](int ci) -> int32_t {
-        if constexpr (kPaged) return page_id(p, s, t0 + ci * kChunk);
-        else return 0;
+    // Paged: every chunk's byte offset in the pools, in 64-byte units (a
+    // chunk starts on a multiple of 32 tokens, 2,112 bytes, inside a page of
+    // a multiple of 32 tokens, so offsets are multiples of 64 and 32 bits
+    // reach 256 GB); kBadChunk marks an out-of-range page id.  Filled below,
+    // read after the q barrier.
+    constexpr uint32_t kBadChunk = 0xFFFFFFFFu;
+    uint32_t *cofs_s = reinterpret_cast<uint32_t *>(smem + kTcSmemBytes);
+    auto chunk_cofs = [&](int ci) -> uint32_t {
+        bool bad;
+        const int32_t t = t0 + ci * kChunk;
+        const int64_t o = paged_offset(p, page_id(p, s, t), g, t, &bad);
+        return bad ? kBadChunk : (uint32_t)(o >> 6);
     };
-    auto chunk_ofs = [&](int ci, int32_t pid, bool *bad) -> int64_t {
-        const int32_t start = t0 + ci * kChunk;
+    // byte offset of chunk ci from kb / vb; *bad: an out-of-range page id
+    auto chunk_ofs = [&](int ci, bool *bad) -> int64_t {
         if constexpr (kPaged) {
-            return paged_offset(p, pid, g, start, bad);
+            const uint32_t v = cofs_s[ci];
+            *bad = v == kBadChunk;
+            return *bad ? 0 : (int64_t)v << 6;
         } else {
             *bad = false;
-            return (int64_t)start * kBlockBytes;
+            return (int64_t)(t0 + ci * kChunk) * kBlockBytes;
         }
     };
     // chunk ci -> warp w, stage st; ofs from chunk_ofs
@@ -239,33 +255,49 @@ decode_tc_kernel(const AttnParams p) {
         bulk_g2s(dst + kChunkBytes, vb + ofs, bytes, bar);
     };
     auto issue = [&](int ci, int st, int32_t tend, int64_t ofs) { issue_for(warp, ci, st, tend, ofs); };
-    // The last warp (never a q warp) initialises every warp's barriers and
-    // issues every warp's first chunk, so the q warps start on q at once.
+    // Contiguous caches: the last warp (never a q warp) initialises every
+    // warp's barriers and issues every warp's first chunk, so the q warps
+    // start on q at once.  Paged: each warp does its own once its first page
+    // id is in.
     static_assert(kTcWarps <= 32 && kMaxGroup < kTcWarps, "one issuing lane per warp");
-    bool bad0 = false;      // paged: lane w of the last warp, chunk w's page id
-    if (warp == kTcWarps - 1 && lane < kTcWarps) {
+    bool bad0 = false;      // paged: the first chunk's page id (lane 0 of each warp)
+    if (!kPaged && warp == kTcWarps - 1 && lane < kTcWarps) {
         const int w = lane;
         for (int st = 0; st < kTcStages; ++st) mbar_init(smem_u32(bars) + (w * kTcStages + st) * 8, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        if (w < n_chunks_max)                               // stage 0 now, the others later
-            issue_for(w, w, 0, t1_max, chunk_ofs(w, pid_of(w), &bad0));
+        if (w < n_chunks_max) {                             // stage 0 now, the others later
+            bool bad;
+            issue_for(w, w, 0, t1_max, chunk_ofs(w, &bad));
+        }
+    }
+    if (kPaged) {
+        // every warp sets up its own ring and issues its first chunk (the
+        // page id load overlaps the q loads); the warps past the q warps copy
+        // the remaining page ids
+        uint32_t c0 = 0;
+        if (lane == 0 && warp < n_chunks_max) c0 = chunk_cofs(warp);
+        if (warp >= kMaxGroup)
+            for (int i = kTcWarps + threadIdx.x - kMaxGroup * 32; i < n_chunks_max;
+                 i += (kTcWarps - kMaxGroup) * 32)
+                cofs_s[i] = chunk_cofs(i);
+        if (lane == 0) {
+            for (int st = 0; st < kTcStages; ++st) mbar_init(smem_u32(bars) + (warp * kTcStages + st) * 8, 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+            if (warp < n_chunks_max) {
+                cofs_s[warp] = c0;
+                issue_for(warp, warp, 0, t1_max, chunk_ofs(warp, &bad0));
+            }
+        }
     }
     // queue of the chunks in stages st, st+1, st+2 (mod 3); -1: none
     int q0 = warp < n_chunks_max ? warp : -1;
     int q1 = warp + kTcWarps < n_chunks_max ? warp + kTcWarps : -1;
     int q2 = warp + 2 * kTcWarps < n_chunks_max ? warp + 2 * kTcWarps : -1;
-    // paged: the page ids of the next copies, loaded well before their use
-    int32_t pid1 = 0, pid2 = 0, pid_n = 0;
-    if (kPaged && lane == 0) {
-        if (q1 >= 0) pid1 = pid_of(q1);
-        if (q2 >= 0) pid2 = pid_of(q2);
-        if (q2 >= 0 && q2 + kTcWarps < n_chunks_max) pid_n = pid_of(q2 + kTcWarps);
-    }
     const int32_t len = seq_length(p, s);
     const int32_t t1 = min(len, t1_max);
     const int n_chunks = t1 > t0 ? (t1 - t0 + kChunk - 1) / kChunk : 0;
     // a bad page id is an error only where the chunk holds real tokens
-    if (kPaged && bad0 && lane < n_chunks) record_status(4u /* TBQ4_ERR_CAPACITY */);
+    if (kPaged && bad0 && warp < n_chunks) record_status(4u);
 
     // ---- q: rotate, normalise by a power of two, 18-bit integer ----------
     // q_int = rint(q_rot * 2^(18-e)) with 2^e > max|q_rot|, so |q_int| <= 2^18.
@@ -339,8 +371,8 @@ decode_tc_kernel(const AttnParams p) {
     bool stage2_pending = true;
     if (lane == 0 && q1 >= 0) {
         bool bad;
-        const int64_t o = chunk_ofs(q1, pid1, &bad);
-        if (bad && q1 < n_chunks) record_status(4u);
+        const int64_t o = chunk_ofs(q1, &bad);
+        if (bad && q1 < n_chunks) record_status(4u /* TBQ4_ERR_CAPACITY */);
         issue(q1, 1, t1_max, o);
     }
 
@@ -558,7 +590,7 @@ decode_tc_kernel(const AttnParams p) {
             stage2_pending = false;
             if (lane == 0 && q2 >= 0) {
                 bool bad;
-                const int64_t o = chunk_ofs(q2, pid2, &bad);
+                const int64_t o = chunk_ofs(q2, &bad);
                 if (bad && q2 < n_chunks) record_status(4u);
                 issue(q2, 2, t1_max, o);
             }
@@ -567,10 +599,9 @@ decode_tc_kernel(const AttnParams p) {
         if (nxt >= n_chunks) nxt = -1;
         if (lane == 0 && nxt >= 0) {          // nxt < n_chunks: real tokens
             bool bad;
-            const int64_t o = chunk_ofs(nxt, pid_n, &bad);
+            const int64_t o = chunk_ofs(nxt, &bad);
             if (bad) record_status(4u);
             issue(nxt, st, t1, o);
-            if (kPaged && nxt + kTcWarps < n_chunks) pid_n = pid_of(nxt + kTcWarps);
         }
         q0 = q1;
         q1 = q2;

@@ -51,6 +51,8 @@ int32_t auto_split_tokens(int nseq, int Hkv, int32_t max_len) {
     // warp of a full split gets the same number of chunks
     per = ceil_div(per, (int64_t)kChunk * kTcWarps) * ((int64_t)kChunk * kTcWarps);
     if (per < (int64_t)kChunk * kTcWarps) per = (int64_t)kChunk * kTcWarps;
+    // at most kPidCap chunks, the page ids a paged CTA keeps in shared memory
+    if (per > (int64_t)kPidCap * kChunk) per = (int64_t)kPidCap * kChunk;
     return (int32_t)per;
 }
 
@@ -126,8 +128,10 @@ tbq4_status run_attention(AttnParams p, void *workspace, size_t ws_bytes,
     static bool attr_set[64] = {}, attr_paged[64] = {}, attr_mq[64] = {};  // once per device
     const bool mq = p.q_len > 1, paged = p.block_table != nullptr;
     if (mq && paged) return TBQ4_ERR_SHAPE;
+    if (paged && p.split_tokens > kPidCap * kChunk) return TBQ4_ERR_SHAPE;
     if (mq ? !ensure_smem_attr((const void *)dmq::decode_mq_kernel, dmq::kSmemBytes, attr_mq)
-           : paged ? !ensure_smem_attr((const void *)decode_tc_kernel<true>, kTcSmemBytes, attr_paged)
+           : paged ? !ensure_smem_attr((const void *)decode_tc_kernel<true>, kTcSmemBytesPaged,
+                                       attr_paged)
                    : !ensure_smem_attr((const void *)decode_tc_kernel<false>, kTcSmemBytes, attr_set))
         return TBQ4_ERR_LAUNCH;
     dim3 g1(p.n_splits, p.Hkv, p.nseq);
@@ -135,7 +139,7 @@ tbq4_status run_attention(AttnParams p, void *workspace, size_t ws_bytes,
     if (mq)
         dmq::decode_mq_kernel<<<g1, dmq::kThreads, dmq::kSmemBytes, st>>>(p);
     else if (paged)
-        decode_tc_kernel<true><<<g1, kTcWarps * 32, kTcSmemBytes, st>>>(p);
+        decode_tc_kernel<true><<<g1, kTcWarps * 32, kTcSmemBytesPaged, st>>>(p);
     else
         decode_tc_kernel<false><<<g1, kTcWarps * 32, kTcSmemBytes, st>>>(p);
     // The combine is a programmatic dependent launch: its CTAs are placed as
