@@ -13,10 +13,10 @@
 //               8,448 bytes each) into a 2-stage raw ring
 //   warp 1      tensor-memory allocation; lane 0 issues every tcgen05.mma
 //   warps 4-7   dequantisation: raw nibbles -> bf16 operand tiles in a
-//               3-slot ring of 32 KB (K tile: keys x dims, exact levels
-//               2n-15; V^T tile: dims x keys, (2n-15) S_v/15 rounded once;
-//               both K-major with the 128-byte swizzle), plus the per-token
-//               factor S_k * scale * log2(e) / 15 for the softmax
+//               3-slot ring of 32 KB (K tile: keys x dims, (2n-15) S_k *
+//               scale * log2(e) / 15 rounded once, so S comes out of the
+//               MMA in log2 units; V^T tile: dims x keys, (2n-15) S_v/15
+//               rounded once; both K-major with the 128-byte swizzle)
 //   warps 8-11  softmax of M-tile 0 (thread = query row = TMEM lane)
 //   warps 12-15 softmax of M-tile 1
 // Tensor memory (512 columns): M-tile a has S at [256a, 256a+128) (P, bf16,
@@ -41,16 +41,19 @@ constexpr int kRawStages = 2;
 constexpr int kRawStageBytes = 2 * kRawBytes + 16;      // K | V | pad
 constexpr int kSlots = 3;
 constexpr int kOpBytes = kTile * kD * 2;                // 32 KB bf16 operand tile
-constexpr int kSigRing = 4;
 constexpr float kRescaleThreshold = 8.0f;               // log2 units
 constexpr float kFastSumLimit = 256.0f;                 // 2^kRescaleThreshold
 constexpr uint32_t kSpin = 1u << 22;
+// The producer and the dequantisation warps run ahead of the tensor core;
+// their waits sleep this long between polls, leaving issue slots to the
+// softmax warps on the same schedulers.
+constexpr uint32_t kLazyNs = 128;
 // Registers per thread after the prologue, per warpgroup: producer/MMA,
 // dequantisation, and each softmax warpgroup (which holds a full S row of 128
 // floats).  Their sum x 128 threads must fit in what the CTA was launched
 // with, 512 threads x the compiled count; the host refuses to launch if the
 // compiled count is below kMinLaunchRegs.
-constexpr uint32_t kRegsCtl = 40, kRegsDeq = 88, kRegsSoft = 192;
+constexpr uint32_t kRegsCtl = 56, kRegsDeq = 88, kRegsSoft = 184;
 constexpr int kMinLaunchRegs = 128;
 static_assert((kRegsCtl + kRegsDeq + 2 * kRegsSoft) * 128 <= kMinLaunchRegs * kThreads,
               "register split exceeds the launch budget");
@@ -59,9 +62,8 @@ static_assert((kRegsCtl + kRegsDeq + 2 * kRegsSoft) * 128 <= kMinLaunchRegs * kT
 constexpr int kOffQ = 0;                                        // 2 x 32 KB
 constexpr int kOffSlot = kOffQ + 2 * kOpBytes;                  // 3 x 32 KB
 constexpr int kOffRaw = kOffSlot + kSlots * kOpBytes;           // 2 x 16,912
-constexpr int kOffSig = kOffRaw + kRawStages * kRawStageBytes;  // 4 x (128 + 128) floats
-constexpr int kOffBar = kOffSig + kSigRing * 2 * kTile * 4;
-constexpr int kNumBars = 2 * kRawStages + 2 * kSlots + 2 * kSigRing + 6;
+constexpr int kOffBar = kOffRaw + kRawStages * kRawStageBytes;
+constexpr int kNumBars = 2 * kRawStages + 2 * kSlots + 6;
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffTmemPtr + 16 + 1024;              // + alignment slack
 
@@ -70,11 +72,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 constexpr uint32_t kIdesc = tc::idesc_bf16(128, 128);
 
-// bf16x2 constants: {2, 2}, {-143, -143}; 64 + n -> 2n - 15.
-constexpr uint32_t kB2Two = 0x40004000u;
-constexpr uint32_t kB2Neg143 = 0xC30FC30Fu;
-constexpr uint32_t kB2Magic64 = 0x42804280u;
-// {128 + n} from a nibble in mantissa bits 0-3, and {-136}: 128 + n - 136 = n - 8.
+// bf16x2 constants: {128 + n} from a nibble in mantissa bits 0-3, and {-136}: 128 + n - 136 = n - 8.
 constexpr uint32_t kB2Magic128 = 0x43004300u;
 constexpr uint32_t kB2Neg136 = 0xC308C308u;
 
@@ -91,16 +89,12 @@ __device__ __forceinline__ uint32_t badd2(uint32_t x, uint32_t a) {
     return *reinterpret_cast<uint32_t *>(&r);
 }
 
-// V level times the token's factor S_v/15, in one rounding: with n - 8
-// exact, (n - 8) * 2 s + s = (2n - 15) s.  v holds nibbles in bits 0-3 and
-// 16-19; s2 = {2 s_a, 2 s_b}, s1 = {s_a, s_b}.
+// A level times its token's factor s, in one rounding: with n - 8 exact,
+// (n - 8) * 2 s + s = (2n - 15) s.  v holds nibbles in bits 0-3 and 16-19;
+// s2 = {2 s_a, 2 s_b}, s1 = {s_a, s_b}.  V: s = S_v / 15; K: s = S_k *
+// softmax_scale * log2(e) / 15.
 __device__ __forceinline__ uint32_t v_scaled(uint32_t v, uint32_t s2, uint32_t s1) {
     return bfma2(badd2((v & 0x000F000Fu) | kB2Magic128, kB2Neg136), s2, s1);
-}
-
-// Nibbles at bit offset `sh` of both 16-bit halves of v -> bf16 64+n.
-__device__ __forceinline__ uint32_t nib_pair(uint32_t v, int sh) {
-    return ((sh >= 0 ? (v >> sh) : (v << -sh)) & 0x001E001Eu) | kB2Magic64;
 }
 
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
@@ -188,19 +182,15 @@ prefill_tc_kernel(const PrefillParams p) {
     auto raw_empty = [&](int s) { return bar0 + 8 * (kRawStages + s); };
     auto slot_full = [&](int s) { return bar0 + 8 * (2 * kRawStages + s); };
     auto slot_empty = [&](int s) { return bar0 + 8 * (2 * kRawStages + kSlots + s); };
-    auto sig_full = [&](int s) { return bar0 + 8 * (2 * kRawStages + 2 * kSlots + s); };
-    auto sig_empty = [&](int s) { return bar0 + 8 * (2 * kRawStages + 2 * kSlots + kSigRing + s); };
-    const uint32_t barx = bar0 + 8 * (2 * kRawStages + 2 * kSlots + 2 * kSigRing);
+    const uint32_t barx = bar0 + 8 * (2 * kRawStages + 2 * kSlots);
     auto s_full = [&](int a) { return barx + 8 * a; };
     auto p_full = [&](int a) { return barx + 8 * (2 + a); };
     auto o_done = [&](int a) { return barx + 8 * (4 + a); };
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + kOffTmemPtr);
-    float *sig = reinterpret_cast<float *>(smem + kOffSig);          // [ring][2][128]
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kRawStages; ++s) { tc::bar_init(raw_full(s), 1); tc::bar_init(raw_empty(s), 4); }
         for (int s = 0; s < kSlots; ++s) { tc::bar_init(slot_full(s), 4); tc::bar_init(slot_empty(s), 1); }
-        for (int s = 0; s < kSigRing; ++s) { tc::bar_init(sig_full(s), 4); tc::bar_init(sig_empty(s), 8); }
         for (int a = 0; a < 2; ++a) {
             tc::bar_init(s_full(a), 1);
             tc::bar_init(p_full(a), 4);
@@ -249,7 +239,7 @@ prefill_tc_kernel(const PrefillParams p) {
             for (int j = 0; j < n_tiles; ++j) {
                 const int st = j % kRawStages;
                 if (j >= kRawStages &&
-                    !tc::bar_wait(raw_empty(st), ((j / kRawStages) - 1) & 1, kSpin)) {
+                    !tc::bar_wait_lazy(raw_empty(st), ((j / kRawStages) - 1) & 1, kSpin, kLazyNs)) {
                     record_status(7u);
                     break;
                 }
@@ -329,35 +319,32 @@ prefill_tc_kernel(const PrefillParams p) {
             const int st = j % kRawStages;
             const uint32_t raw = sbase + kOffRaw + st * kRawStageBytes;
             const int64_t t0 = (int64_t)(tile_begin + j) * kTile;
-            if (!tc::bar_wait_warp(raw_full(st), (j / kRawStages) & 1, kSpin)) { record_status(7u); break; }
-            // per-token factors for the softmax
-            const int sr = j % kSigRing;
-            if (j >= kSigRing &&
-                !tc::bar_wait_warp(sig_empty(sr), ((j / kSigRing) - 1) & 1, kSpin)) { record_status(7u); break; }
-            {
-                const bool in = t0 + t < keys_total;
-                const float sk = __half2float(__ushort_as_half(lds16(raw + t * kBlockBytes)));
-                sig[(sr * 2 + 0) * kTile + t] = in ? sk * p.scale_log2_15 : 0.f;
-            }
-            __syncwarp();
-            if (lane == 0) tc::bar_arrive(sig_full(sr));
-
-            // K tile: token t -> row t, dims contiguous
+            if (!tc::bar_wait_lazy_warp(raw_full(st), (j / kRawStages) & 1, kSpin, kLazyNs)) { record_status(7u); break; }
+            // K tile: token t -> row t, dims contiguous, each level times the
+            // token's factor S_k * scale * log2(e) / 15 rounded once (so S
+            // leaves the MMA in log2 units); 0 past the cache end, where the
+            // raw bytes are stale
             {
                 const int u = 2 * j, slot = u % kSlots;
-                if (u >= kSlots && !tc::bar_wait_warp(slot_empty(slot), ((u / kSlots) - 1) & 1, kSpin)) {
+                if (u >= kSlots && !tc::bar_wait_lazy_warp(slot_empty(slot), ((u / kSlots) - 1) & 1, kSpin, kLazyNs)) {
                     record_status(7u);
                     break;
                 }
                 const uint32_t dst = sbase + kOffSlot + slot * kOpBytes;
                 const uint32_t src = raw + t * kBlockBytes + 2;
+                const float fk = t0 + t < keys_total
+                    ? __half2float(__ushort_as_half(lds16(src - 2))) * p.scale_log2_15 : 0.f;
+                const __nv_bfloat162 f1b = __floats2bfloat162_rn(fk, fk);
+                const __nv_bfloat162 f2b = __hmul2(f1b, __floats2bfloat162_rn(2.f, 2.f));
+                const uint32_t f1 = *reinterpret_cast<const uint32_t *>(&f1b);
+                const uint32_t f2 = *reinterpret_cast<const uint32_t *>(&f2b);
 #pragma unroll 4
                 for (int w = 0; w < 16; ++w) {
                     const uint32_t x = funnel_word(src + 4 * w);
-                    const uint32_t l0 = bfma2(nib_pair(x, -1), kB2Two, kB2Neg143);   // b0.lo, b2.lo
-                    const uint32_t h0 = bfma2(nib_pair(x, 3), kB2Two, kB2Neg143);    // b0.hi, b2.hi
-                    const uint32_t l1 = bfma2(nib_pair(x, 7), kB2Two, kB2Neg143);    // b1.lo, b3.lo
-                    const uint32_t h1 = bfma2(nib_pair(x, 11), kB2Two, kB2Neg143);   // b1.hi, b3.hi
+                    const uint32_t l0 = v_scaled(x, f2, f1);          // b0.lo, b2.lo
+                    const uint32_t h0 = v_scaled(x >> 4, f2, f1);     // b0.hi, b2.hi
+                    const uint32_t l1 = v_scaled(x >> 8, f2, f1);     // b1.lo, b3.lo
+                    const uint32_t h1 = v_scaled(x >> 12, f2, f1);    // b1.hi, b3.hi
                     sts128(dst + sw128_off(t, 8 * w), __byte_perm(l0, h0, 0x5410),
                            __byte_perm(l1, h1, 0x5410), __byte_perm(l0, h0, 0x7632),
                            __byte_perm(l1, h1, 0x7632));
@@ -370,7 +357,7 @@ prefill_tc_kernel(const PrefillParams p) {
             // (2pp, 2pp+1) x dims [64 hf, 64 hf + 64)
             {
                 const int u = 2 * j + 1, slot = u % kSlots;
-                if (u >= kSlots && !tc::bar_wait_warp(slot_empty(slot), ((u / kSlots) - 1) & 1, kSpin)) {
+                if (u >= kSlots && !tc::bar_wait_lazy_warp(slot_empty(slot), ((u / kSlots) - 1) & 1, kSpin, kLazyNs)) {
                     record_status(7u);
                     break;
                 }
@@ -423,73 +410,76 @@ prefill_tc_kernel(const PrefillParams p) {
         float m = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < n_tiles && active; ++j) {
-            const int sr = j % kSigRing;
-            if (!tc::bar_wait_warp(s_full(a), j & 1, kSpin) ||
-                !tc::bar_wait_warp(sig_full(sr), (j / kSigRing) & 1, kSpin)) {
+            if (!tc::bar_wait_warp(s_full(a), j & 1, kSpin)) {
                 record_status(7u);
                 ok = false;
                 break;
             }
             tc::fence_after_sync();
-            const float *sk = sig + (sr * 2 + 0) * kTile;
             const int64_t kt = (int64_t)(tile_begin + j) * kTile;
             const bool diag = kt + kTile - 1 > p.n_cached + i0;
             // Causal mask only on tiles that reach past the block's first row:
             // column col is masked when kt + col > lim, i.e. col > rel.
             const int rel = diag ? (int)(lim - kt) : kTile;
-            // The whole S row of this thread goes to registers with one wait;
-            // from then on P may overwrite S in tensor memory.
+            // The whole S row of this thread goes to registers with one wait.
             float sr_[kTile];
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch)
                 tc::tmem_ld32(t_s + 32 * ch, *reinterpret_cast<float(*)[32]>(sr_ + 32 * ch));
             tc::tmem_wait_ld();
             // Fast path (every row of the warp has a finite running max): P =
-            // exp2(S*sk - m) with the stale m, kept if each row's sum of P over
-            // the tile stays <= 2^8 (which bounds every P by 2^8).
+            // exp2(S - m) with the stale m, kept if each row's sum of P over
+            // the tile stays <= 2^8 (which bounds every P by 2^8).  P is packed
+            // in registers and written over S only once it is kept, so S stays
+            // in tensor memory for the slow path and the S registers die as P
+            // is formed.
             bool done = false;
             if (!__any_sync(kFull, m == -INFINITY)) {
                 const float2 negm = make_float2(-m, -m);
                 float2 lf[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                uint32_t pk[kTile / 2];
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const int col = 32 * ch + e;
-                        const float2 skv = *reinterpret_cast<const float2 *>(sk + col);
-                        float2 d = __ffma2_rn(make_float2(sr_[col], sr_[col + 1]), skv, negm);
-                        if (diag) {
-                            if (col > rel) d.x = -INFINITY;
-                            if (col + 1 > rel) d.y = -INFINITY;
-                        }
-                        const float2 pr = make_float2(tc::ex2(d.x), tc::ex2(d.y));
-                        lf[(e >> 1) & 1] = __fadd2_rn(lf[(e >> 1) & 1], pr);
-                        __nv_bfloat162 bb = __floats2bfloat162_rn(pr.x, pr.y);
-                        pk[e >> 1] = *reinterpret_cast<uint32_t *>(&bb);
+                for (int e = 0; e < kTile; e += 2) {
+                    float2 d = __fadd2_rn(make_float2(sr_[e], sr_[e + 1]), negm);
+                    if (diag) {
+                        if (e > rel) d.x = -INFINITY;
+                        if (e + 1 > rel) d.y = -INFINITY;
                     }
-                    tc::tmem_st16(t_s + 16 * ch, pk);
+                    const float2 pr = make_float2(tc::ex2(d.x), tc::ex2(d.y));
+                    lf[(e >> 1) & 1] = __fadd2_rn(lf[(e >> 1) & 1], pr);
+                    __nv_bfloat162 bb = __floats2bfloat162_rn(pr.x, pr.y);
+                    pk[e >> 1] = *reinterpret_cast<uint32_t *>(&bb);
                 }
                 const float lt = (lf[0].x + lf[0].y) + (lf[1].x + lf[1].y);
                 if (!__any_sync(kFull, !(lt <= kFastSumLimit))) {
                     l += lt;
                     done = true;
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch)
+                        tc::tmem_st16(t_s + 16 * ch, *reinterpret_cast<uint32_t(*)[16]>(pk + 16 * ch));
                 }
             }
             if (!done) {
-                // exact row max, O rescale when it grows past the threshold,
-                // then P again from the registers (over whatever the fast path
-                // wrote)
+                // exact row max from S reloaded 32 columns at a time, O rescale
+                // when it grows past the threshold, then P (column block c of P
+                // lands on S columns already read: P's 64 columns cover S
+                // columns 0-63, read in the first two blocks)
                 float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+                for (int ch = 0; ch < 4; ++ch) {
+                    float sc[32];
+                    tc::tmem_ld32(t_s + 32 * ch, sc);
+                    tc::tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < kTile; e += 2) {
-                    const float2 skv = *reinterpret_cast<const float2 *>(sk + e);
-                    float2 z = __fmul2_rn(make_float2(sr_[e], sr_[e + 1]), skv);
-                    if (diag) {
-                        if (e > rel) z.x = -INFINITY;
-                        if (e + 1 > rel) z.y = -INFINITY;
+                    for (int e = 0; e < 32; e += 2) {
+                        const int col = 32 * ch + e;
+                        float2 z = make_float2(sc[e], sc[e + 1]);
+                        if (diag) {
+                            if (col > rel) z.x = -INFINITY;
+                            if (col + 1 > rel) z.y = -INFINITY;
+                        }
+                        mx4[(e >> 1) & 3] = fmaxf(mx4[(e >> 1) & 3], fmaxf(z.x, z.y));
                     }
-                    mx4[(e >> 1) & 3] = fmaxf(mx4[(e >> 1) & 3], fmaxf(z.x, z.y));
                 }
                 const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
                 const float m_new = fmaxf(m, mx);
@@ -520,14 +510,16 @@ prefill_tc_kernel(const PrefillParams p) {
                 const float m_use = (m == -INFINITY) ? 0.f : m;
                 const float2 negm = make_float2(-m_use, -m_use);
                 float2 lacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
+#pragma unroll 1
                 for (int ch = 0; ch < 4; ++ch) {
+                    float sc[32];
+                    tc::tmem_ld32(t_s + 32 * ch, sc);
+                    tc::tmem_wait_ld();
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
                         const int col = 32 * ch + e;
-                        const float2 skv = *reinterpret_cast<const float2 *>(sk + col);
-                        float2 z = __ffma2_rn(make_float2(sr_[col], sr_[col + 1]), skv, negm);
+                        float2 z = __fadd2_rn(make_float2(sc[e], sc[e + 1]), negm);
                         if (diag) {
                             if (col > rel) z.x = -INFINITY;
                             if (col + 1 > rel) z.y = -INFINITY;
@@ -544,19 +536,7 @@ prefill_tc_kernel(const PrefillParams p) {
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) {
-                tc::bar_arrive(p_full(a));
-                tc::bar_arrive(sig_empty(sr));
-            }
-        }
-        if (!active) {
-            // the unused M-tile of an odd group still releases the sig ring
-            for (int j = 0; j < n_tiles; ++j) {
-                const int sr = j % kSigRing;
-                if (!tc::bar_wait_warp(sig_full(sr), (j / kSigRing) & 1, kSpin)) { record_status(7u); break; }
-                __syncwarp();
-                if (lane == 0) tc::bar_arrive(sig_empty(sr));
-            }
+            if (lane == 0) tc::bar_arrive(p_full(a));
         }
         // ---- partial (O unnormalised, m, l) for this split -----------------
         const int h = 2 * pair + a;

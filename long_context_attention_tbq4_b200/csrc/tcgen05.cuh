@@ -60,6 +60,23 @@ __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, uint32_t
     return false;
 }
 
+// Bounded wait that sleeps `ns` nanoseconds between polls, for a thread
+// that runs ahead of its consumers: a polling warp takes issue slots from
+// the warps it shares a scheduler with.  False after `limit` polls.
+__device__ __forceinline__ bool bar_wait_lazy(uint32_t bar, uint32_t parity, uint32_t limit,
+                                              uint32_t ns) {
+    for (uint32_t i = 0; i < limit; ++i) {
+        if (bar_try_wait(bar, parity)) return true;
+        __nanosleep(ns);
+    }
+    return false;
+}
+__device__ __forceinline__ bool bar_wait_lazy_warp(uint32_t bar, uint32_t parity, uint32_t limit,
+                                                   uint32_t ns) {
+    const bool ok = bar_wait_lazy(bar, parity, limit, ns);
+    return __all_sync(0xffffffffu, ok);
+}
+
 // Bounded wait by a whole warp: every lane polls, and the result is the
 // same in every lane (a warp never splits on a timeout).
 __device__ __forceinline__ bool bar_wait_warp(uint32_t bar, uint32_t parity, uint32_t limit) {
