@@ -53,7 +53,7 @@ constexpr uint32_t kLazyNs = 128;
 // floats).  Their sum x 128 threads must fit in what the CTA was launched
 // with, 512 threads x the compiled count; the host refuses to launch if the
 // compiled count is below kMinLaunchRegs.
-constexpr uint32_t kRegsCtl = 56, kRegsDeq = 88, kRegsSoft = 184;
+constexpr uint32_t kRegsCtl = 64, kRegsDeq = 80, kRegsSoft = 184;
 constexpr int kMinLaunchRegs = 128;
 static_assert((kRegsCtl + kRegsDeq + 2 * kRegsSoft) * 128 <= kMinLaunchRegs * kThreads,
               "register split exceeds the launch budget");
@@ -258,8 +258,16 @@ prefill_tc_kernel(const PrefillParams p) {
         // ======================= MMA issuer ==================================
         if (lane == 0 && n_tiles > 0) {
             bool ok = true;
+            // polled with test_wait and a short sleep: a thread suspended in
+            // try_wait resumed here about half a microsecond after its phase
+            // completed
             auto wait = [&](uint32_t bar, uint32_t par) {
-                if (ok && !tc::bar_wait(bar, par, kSpin)) { ok = false; record_status(7u); }
+                bool got = false;
+                for (uint32_t i = 0; ok && i < kSpin && !got; ++i) {
+                    got = tc::bar_test(bar, par);
+                    if (!got) __nanosleep(20);
+                }
+                if (ok && !got) { ok = false; record_status(7u); }
                 return ok;
             };
             const uint32_t qa = sbase + kOffQ;
