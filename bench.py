@@ -539,6 +539,7 @@ def main():
         pre["roofline"] = {"bound": "tensor", "achieved": pre["attn_kernel_tflops"],
                            "peak": pk, "unit": "TFLOP/s",
                            "frac": pre["attn_kernel_tflops"] / pk,
+                           "traffic": recorded_traffic("prefill_tc_kernel"),
                            "peak_source": peaks["source"] + " (bf16 burst)"}
         line["prefill"] = pre
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
