@@ -22,6 +22,7 @@ import numpy as np
 from . import build as _build
 
 BLOCK_BYTES = 66
+BLOCK_BYTES3 = 50       # the 3-bit variant (TBQ3)
 D = 128
 
 _lib = None
@@ -62,6 +63,17 @@ def lib():
         L.oracle_attn_prefill.argtypes = [p, C.c_int, C.c_int64, p, p, C.c_int,
                                           C.c_int, C.c_int64, C.c_double,
                                           C.c_uint64, p, C.c_int, p]
+        L.oracle_block_bytes3.restype = C.c_int
+        L.oracle_level_index3.argtypes = [C.c_float, C.c_float]
+        L.oracle_level_index3.restype = C.c_int
+        L.oracle_quantize_block3.argtypes = [p, p, p]
+        L.oracle_dequant_block3.argtypes = [p, p]
+        L.oracle_quantize_append3.argtypes = [p, C.c_int, C.c_int, C.c_int, p,
+                                              C.c_int64, C.c_uint64, p]
+        L.oracle_quantize_append3.restype = C.c_int64
+        L.oracle_attn_decode3.argtypes = [p, p, p, p, C.c_int, C.c_int, C.c_int,
+                                          C.c_int64, C.c_double, C.c_uint64, p,
+                                          C.c_int, p]
         _lib = L
     return _lib
 
@@ -209,3 +221,67 @@ def attn_prefill(q, n_cached, k_cache, v_cache, softmax_scale, seed,
                               _ptr(v_cache), Hq, Hkv, cap, float(softmax_scale),
                               C.c_uint64(seed), rp, nr, _ptr(out))
     return out
+
+
+# ---------------------------------------------------------------- TBQ3
+# The 3-bit variant: 128 values in 50 bytes (fp16 scale, then 16 groups of 8
+# indices as 24-bit little-endian words), levels S*(2i-7)/7.  See
+# tbq4_oracle.c for the layout this library fixes.
+def block_bytes3() -> int:
+    return int(lib().oracle_block_bytes3())
+
+
+def level_index3(x_rot: float, S: float) -> int:
+    return int(lib().oracle_level_index3(C.c_float(x_rot), C.c_float(S)))
+
+
+def quantize_block3(x: np.ndarray, s: np.ndarray) -> np.ndarray:
+    x = _c(x, np.float32)
+    s = _c(s, np.int8)
+    out = np.zeros(BLOCK_BYTES3, np.uint8)
+    lib().oracle_quantize_block3(_ptr(x), _ptr(s), _ptr(out))
+    return out
+
+
+def dequant_block3(blk: np.ndarray) -> np.ndarray:
+    blk = _c(blk, np.uint8)
+    out = np.zeros(D, np.float64)
+    lib().oracle_dequant_block3(_ptr(blk), _ptr(out))
+    return out
+
+
+def quantize_append3(src: np.ndarray, start_pos, capacity: int, seed: int,
+                     cache: np.ndarray) -> int:
+    """src [B][n_new][Hkv][128] fp32; cache [B][Hkv][capacity][50] uint8
+    (updated in place).  Returns the number of rows skipped as out of range."""
+    src = _c(src, np.float32)
+    B, n_new, Hkv, d = src.shape
+    assert d == D and cache.dtype == np.uint8 and cache.flags.c_contiguous
+    assert cache.shape == (B, Hkv, capacity, BLOCK_BYTES3)
+    sp = _c(start_pos, np.int32)
+    return int(lib().oracle_quantize_append3(_ptr(src), B, n_new, Hkv, _ptr(sp),
+                                             capacity, C.c_uint64(seed), _ptr(cache)))
+
+
+def attn_decode3(q, k_cache, v_cache, seq_lens, softmax_scale, seed,
+                 rows=None) -> np.ndarray:
+    """q [B][Hq][128] fp32; 3-bit caches [B][Hkv][capacity][50]; returns
+    [B][Hq][128] float64 (rows not listed in ``rows`` are NaN)."""
+    q = _c(q, np.float32)
+    B, Hq, d = q.shape
+    _, Hkv, cap, nb = k_cache.shape
+    assert d == D and nb == BLOCK_BYTES3 and v_cache.shape == k_cache.shape
+    k_cache = _c(k_cache, np.uint8)
+    v_cache = _c(v_cache, np.uint8)
+    sl = _c(seq_lens, np.int32)
+    out = np.full((B, Hq, D), np.nan, np.float64)
+    if rows is None:
+        rp, nr = None, 0
+    else:
+        rows = _c(rows, np.int32)
+        rp, nr = _ptr(rows), len(rows)
+    lib().oracle_attn_decode3(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(sl),
+                              B, Hq, Hkv, cap, float(softmax_scale),
+                              C.c_uint64(seed), rp, nr, _ptr(out))
+    return out
+

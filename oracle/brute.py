@@ -7,6 +7,8 @@ Written straight from the definitions, with no numpy and no shared code with
   rational arithmetic (ties to the even index);
 * dequant: unpack a 66-byte block (scale bytes first, even element in the
   low nibble) into S*(2i-15)/15;
+* nearest_level_index3, unpack3, dequant3: the same for the 3-bit variant
+  (8 levels S*(2i-7)/7; a 50-byte block read as a little-endian bit stream);
 * attention: softmax(scale * q_rot . k) v with math.fsum, in the rotated
   domain, then rotated back with the explicit Hadamard entries.
 """
@@ -26,6 +28,21 @@ def nearest_level_index(x_rot: float, S: float) -> int:
     best, best_d = None, None
     for i in range(16):
         d = abs(x - s * (2 * i - 15) / 15)
+        if best_d is None or d < best_d or (d == best_d and i % 2 == 0):
+            best, best_d = i, d
+    return best
+
+
+def nearest_level_index3(x_rot: float, S: float) -> int:
+    """The 3-bit codebook: argmin over the 8 levels S*(2i-7)/7, ties to the
+    even index; index 4 when S == 0."""
+    if S == 0:
+        return 4
+    x = Fraction(x_rot)
+    s = Fraction(S)
+    best, best_d = None, None
+    for i in range(8):
+        d = abs(x - s * (2 * i - 7) / 7)
         if best_d is None or d < best_d or (d == best_d and i % 2 == 0):
             best, best_d = i, d
     return best
@@ -53,6 +70,22 @@ def dequant(block) -> list:
     return out
 
 
+def unpack3(block) -> list:
+    """The 128 indices of a 50-byte 3-bit block, read one bit at a time from
+    the byte string (bit 3i+b of the little-endian stream after the scale is
+    bit b of index i)."""
+    block = [int(b) for b in block]
+    bits = []
+    for byte in block[2:]:
+        bits.extend((byte >> k) & 1 for k in range(8))
+    return [bits[3 * i] | (bits[3 * i + 1] << 1) | (bits[3 * i + 2] << 2) for i in range(128)]
+
+
+def dequant3(block) -> list:
+    S = f16_bits_to_float(int(block[0]) | (int(block[1]) << 8))
+    return [S * (2 * i - 7) / 7 for i in unpack3(block)]
+
+
 def rotate(x, s) -> list:
     """R x with R[i][j] = H[i][j] s_j / sqrt(128)."""
     n = len(x)
@@ -69,11 +102,12 @@ def unrotate(y, s) -> list:
             for j in range(n)]
 
 
-def attend(q, k_blocks, v_blocks, scale, s) -> list:
-    """One query row over a handful of keys (blocks given as byte lists)."""
+def attend(q, k_blocks, v_blocks, scale, s, deq=dequant) -> list:
+    """One query row over a handful of keys (blocks given as byte lists;
+    deq = dequant3 for 3-bit blocks)."""
     q_rot = rotate([float(v) for v in q], s)
-    ks = [dequant(b) for b in k_blocks]
-    vs = [dequant(b) for b in v_blocks]
+    ks = [deq(b) for b in k_blocks]
+    vs = [deq(b) for b in v_blocks]
     logits = [scale * math.fsum(a * b for a, b in zip(q_rot, k)) for k in ks]
     m = max(logits)
     p = [math.exp(z - m) for z in logits]

@@ -264,13 +264,16 @@ int64_t oracle_quantize_append(const float *src, int B, int n_new, int Hkv,
 }
 
 /* -------------------------------------------------------------- attention */
+typedef void (*dequant_fn)(const uint8_t *blk, double *out);
+
 /* One attention row in the rotated domain, all in double:
  *   q_rot = R q;  logit_t = scale * q_rot . Khat_t  (t < n_keys);
  *   p = softmax(logit);  o_rot = sum_t p_t Vhat_t;  o = R^T o_rot.
- * k_rows / v_rows point at the first block of the (b, kv head) stream. */
-static void attend_row(const double *R, const double *q, const uint8_t *k_rows,
-                       const uint8_t *v_rows, int64_t n_keys, double scale,
-                       double *o) {
+ * k_rows / v_rows point at the first block of the (b, kv head) stream;
+ * blocks are nbytes apart and dequantised by dq. */
+static void attend_row_fmt(const double *R, const double *q, const uint8_t *k_rows,
+                           const uint8_t *v_rows, int64_t n_keys, double scale,
+                           int nbytes, dequant_fn dq, double *o) {
     double q_rot[OD], o_rot[OD], kd[OD], vd[OD];
     for (int i = 0; i < OD; ++i) {
         double acc = 0.0;
@@ -284,7 +287,7 @@ static void attend_row(const double *R, const double *q, const uint8_t *k_rows,
     double *logit = (double *)malloc((size_t)n_keys * sizeof(double));
     double m = -INFINITY;
     for (int64_t t = 0; t < n_keys; ++t) {
-        oracle_dequant_block(k_rows + t * OBLOCK, kd);
+        dq(k_rows + t * nbytes, kd);
         double dot = 0.0;
         for (int i = 0; i < OD; ++i) dot += q_rot[i] * kd[i];
         logit[t] = scale * dot;
@@ -295,7 +298,7 @@ static void attend_row(const double *R, const double *q, const uint8_t *k_rows,
     for (int64_t t = 0; t < n_keys; ++t) {
         double p = exp(logit[t] - m);
         l += p;
-        oracle_dequant_block(v_rows + t * OBLOCK, vd);
+        dq(v_rows + t * nbytes, vd);
         for (int i = 0; i < OD; ++i) o_rot[i] += p * vd[i];
     }
     free(logit);
@@ -305,6 +308,12 @@ static void attend_row(const double *R, const double *q, const uint8_t *k_rows,
         for (int i = 0; i < OD; ++i) acc += R[i * OD + j] * o_rot[i];
         o[j] = acc;
     }
+}
+
+static void attend_row(const double *R, const double *q, const uint8_t *k_rows,
+                       const uint8_t *v_rows, int64_t n_keys, double scale,
+                       double *o) {
+    attend_row_fmt(R, q, k_rows, v_rows, n_keys, scale, OBLOCK, oracle_dequant_block, o);
 }
 
 /* Decode attention.  q [B][Hq][128] fp32 (unrotated); caches
@@ -362,6 +371,115 @@ void oracle_attn_prefill(const float *q, int n_new, int64_t n_cached,
         int64_t base = (int64_t)g * capacity * OBLOCK;
         attend_row(R, qd, k_cache + base, v_cache + base, n_cached + i + 1,
                    softmax_scale, out + (int64_t)row * OD);
+    }
+    free(R);
+}
+
+/* ==================================================================== TBQ3 */
+/* A 3-bit variant with the same rotation and the same scale.  The page
+ * names TBQ3 next to TBQ4 and mentions a fix to its 3-bit packing
+ * (trefon.com, "Kontekst 262K na jednej RTX 4090: co dodalem do
+ * llama.cpp-turboq", section "6. Ten sam cache na Apple silicon") but gives
+ * no layout, so this library fixes one:
+ *   - 128 values in 50 bytes: the fp16 scale (little endian), then 48 bytes;
+ *   - 8 symmetric levels (i - 3.5)/3.5 * S = S * (2i - 7)/7;
+ *   - index = clamp(rne(fl32(fl32(x/S)*3.5)+3.5), 0, 7), index 4 when S == 0;
+ *   - indices 8g .. 8g+7 form one 24-bit little-endian word, index 8g+k at
+ *     bits 3k .. 3k+2, stored as bytes 2+3g, 3+3g, 4+3g.
+ * Cache layout [B][Hkv][capacity][50]. */
+#define OBLOCK3 50
+
+int oracle_block_bytes3(void) { return OBLOCK3; }
+
+/* Index of one rotated value against the block scale, 3-bit codebook. */
+int oracle_level_index3(float x_rot, float S) {
+    if (S == 0.0f) return 4;
+    float t = x_rot / S;
+    float u = t * 3.5f;
+    float v = u + 3.5f;
+    float r = rne_f32(v);
+    if (r < 0.0f) r = 0.0f;
+    if (r > 7.0f) r = 7.0f;
+    return (int)r;
+}
+
+/* One 128-value block -> 50 bytes. */
+void oracle_quantize_block3(const float *x, const int8_t *s, uint8_t *out) {
+    float xr[OD];
+    oracle_rotate_f32(x, s, xr);
+    uint16_t sb = oracle_block_scale_bits(xr);
+    float S = (float)oracle_f16_bits_to_f64(sb);
+    int idx[OD];
+    for (int i = 0; i < OD; ++i) idx[i] = oracle_level_index3(xr[i], S);
+    out[0] = (uint8_t)(sb & 0xFFu);
+    out[1] = (uint8_t)(sb >> 8);
+    for (int g = 0; g < OD / 8; ++g) {
+        uint32_t w = 0;
+        for (int k = 0; k < 8; ++k) w |= (uint32_t)idx[8 * g + k] << (3 * k);
+        out[2 + 3 * g] = (uint8_t)(w & 0xFFu);
+        out[3 + 3 * g] = (uint8_t)((w >> 8) & 0xFFu);
+        out[4 + 3 * g] = (uint8_t)((w >> 16) & 0xFFu);
+    }
+}
+
+/* Dequantise one 3-bit block into the rotated domain: S * (2*idx - 7) / 7. */
+void oracle_dequant_block3(const uint8_t *blk, double *out) {
+    uint16_t sb = (uint16_t)(blk[0] | (blk[1] << 8));
+    double S = oracle_f16_bits_to_f64(sb);
+    for (int g = 0; g < OD / 8; ++g) {
+        uint32_t w = (uint32_t)blk[2 + 3 * g] | ((uint32_t)blk[3 + 3 * g] << 8) |
+                     ((uint32_t)blk[4 + 3 * g] << 16);
+        for (int k = 0; k < 8; ++k) {
+            int i = (int)((w >> (3 * k)) & 7u);
+            out[8 * g + k] = S * (double)(2 * i - 7) / 7.0;
+        }
+    }
+}
+
+/* Quantise-append into a [B][Hkv][capacity][50] cache; as
+ * oracle_quantize_append otherwise. */
+int64_t oracle_quantize_append3(const float *src, int B, int n_new, int Hkv,
+                                const int32_t *start_pos, int64_t capacity,
+                                uint64_t seed, uint8_t *cache) {
+    int8_t s[OD];
+    oracle_signs(seed, s);
+    int64_t rows = (int64_t)B * n_new * Hkv;
+    int64_t skipped = 0;
+#pragma omp parallel for schedule(static) reduction(+ : skipped)
+    for (int64_t r = 0; r < rows; ++r) {
+        int h = (int)(r % Hkv);
+        int64_t t = (r / Hkv) % n_new;
+        int b = (int)(r / ((int64_t)Hkv * n_new));
+        int64_t pos = (int64_t)start_pos[b] + t;
+        if (pos < 0 || pos >= capacity) { skipped += 1; continue; }
+        uint8_t *dst = cache + (((int64_t)b * Hkv + h) * capacity + pos) * OBLOCK3;
+        oracle_quantize_block3(src + r * OD, s, dst);
+    }
+    return skipped;
+}
+
+/* Decode attention over 3-bit caches [B][Hkv][capacity][50]; as
+ * oracle_attn_decode otherwise. */
+void oracle_attn_decode3(const float *q, const uint8_t *k_cache,
+                         const uint8_t *v_cache, const int32_t *seq_lens, int B,
+                         int Hq, int Hkv, int64_t capacity, double softmax_scale,
+                         uint64_t seed, const int32_t *rows, int n_rows,
+                         double *out) {
+    int8_t s[OD];
+    oracle_signs(seed, s);
+    double *R = (double *)malloc(OD * OD * sizeof(double));
+    oracle_rotation_matrix(s, R);
+    int G = Hq / Hkv;
+    int total = rows ? n_rows : B * Hq;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int k = 0; k < total; ++k) {
+        int row = rows ? rows[k] : k;
+        int b = row / Hq, h = row % Hq, g = h / G;
+        double qd[OD];
+        for (int i = 0; i < OD; ++i) qd[i] = (double)q[(int64_t)row * OD + i];
+        int64_t base = ((int64_t)b * Hkv + g) * capacity * OBLOCK3;
+        attend_row_fmt(R, qd, k_cache + base, v_cache + base, seq_lens[b], softmax_scale,
+                       OBLOCK3, oracle_dequant_block3, out + (int64_t)row * OD);
     }
     free(R);
 }
