@@ -196,6 +196,35 @@ TBQ4_API tbq4_status tbq4_attn_decode_paged(const float *q, const float *k_new,
                                             size_t ws_bytes, uint16_t *out, void *stream);
 
 /*
+ * TBQ3: the 3-bit variant.  The page names a 3-bit KV cache type next to
+ * TBQ4 and a fix to its 3-bit packing (trefon.com, "Kontekst 262K na jednej
+ * RTX 4090: co dodalem do llama.cpp-turboq", section "6. Ten sam cache na
+ * Apple silicon") without its layout; this library fixes it:
+ *   block  128 values in 50 bytes (3.125 bits per value): the fp16 scale
+ *          S = fp16(max |x_rot|) (little endian, saturating), then 16 groups
+ *          of three bytes, each a little-endian 24-bit word holding indices
+ *          8g .. 8g+7 (index 8g+k at bits 3k .. 3k+2)
+ *   levels (i - 3.5)/3.5 * S = S (2i - 7)/7, i = 0..7;
+ *          i = clamp(rne(fl32(fl32(x_rot/S) * 3.5) + 3.5), 0, 7), 4 if S == 0
+ *   rotation, sign seed and cache layout as TBQ4, with 50-byte blocks:
+ *          [B][Hkv][capacity][50], capacity % 8 == 0.
+ * tbq3_quantize_append and tbq3_attn_decode take the arguments of
+ * tbq4_quantize_append and tbq4_attn_decode, with the same errors; the decode
+ * workspace is tbq4_decode_workspace_bytes(B, Hq, Hkv, max_len).
+ */
+TBQ4_API size_t tbq3_block_bytes(void);   /* 50 */
+TBQ4_API size_t tbq3_cache_bytes(int batch, int n_kv_heads, int64_t capacity);
+TBQ4_API tbq4_status tbq3_quantize_append(const float *src, int B, int n_new, int Hkv,
+                                          const int32_t *start_pos, int64_t capacity,
+                                          uint64_t sign_seed, uint8_t *cache, void *stream);
+TBQ4_API tbq4_status tbq3_attn_decode(const float *q, const uint8_t *k_cache,
+                                      const uint8_t *v_cache, const int32_t *seq_lens,
+                                      int32_t max_len, int B, int Hq, int Hkv,
+                                      int64_t capacity, float softmax_scale,
+                                      uint64_t sign_seed, void *workspace, size_t ws_bytes,
+                                      uint16_t *out, void *stream);
+
+/*
  * Multi-query decode: q_len (1-4) new query tokens per sequence, as when a
  * model verifies speculative drafts (trefon.com, "Kontekst 262K na jednej RTX
  * 4090", section "Konfiguracja": up to 3 drafted tokens).  Query token i of

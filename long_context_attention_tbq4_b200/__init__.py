@@ -28,6 +28,7 @@ __all__ = [
     "tbq4_prefill_workspace_bytes", "tbq4_attn_prefill_chunk",
     "tbq4_set_timing_events", "tbq4_get_device_status", "empty_cache",
     "empty_pool", "tbq4_quantize_append_paged", "tbq4_attn_decode_paged",
+    "BLOCK_BYTES3", "empty_cache3", "tbq3_quantize_append", "tbq3_attn_decode",
 ]
 
 
@@ -217,6 +218,54 @@ def tbq4_attn_decode_paged(q, k_pool, v_pool, block_table, seq_lens, max_len, so
         int(max_len), B, Hq, Hkv, float(softmax_scale), C.c_uint64(sign_seed), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)),
         "tbq4_attn_decode_paged")
+    return out
+
+
+BLOCK_BYTES3 = 50      # TBQ3: the 3-bit variant (see include/tbq4.h)
+
+
+def empty_cache3(batch, n_kv_heads, capacity, device="cuda"):
+    """An uninitialised 3-bit cache [B][Hkv][capacity][50] (capacity % 8 == 0)."""
+    return torch.empty((batch, n_kv_heads, capacity, BLOCK_BYTES3), dtype=torch.uint8,
+                       device=device)
+
+
+def tbq3_quantize_append(src, start_pos, cache, sign_seed=0, stream=None):
+    """As tbq4_quantize_append, into a 3-bit cache [B][Hkv][capacity][50]."""
+    _need(src, torch.float32, "src", 4)
+    _need(start_pos, torch.int32, "start_pos", 1)
+    _need(cache, torch.uint8, "cache", 4)
+    B, n_new, Hkv, d = src.shape
+    if d != D or tuple(cache.shape[:2]) != (B, Hkv) or cache.shape[3] != BLOCK_BYTES3:
+        raise ValueError("shape mismatch between src and cache")
+    check(lib.tbq3_quantize_append(_ptr(src), B, n_new, Hkv, _ptr(start_pos),
+                                   cache.shape[2], C.c_uint64(sign_seed), _ptr(cache),
+                                   _stream(stream)), "tbq3_quantize_append")
+    return cache
+
+
+def tbq3_attn_decode(q, k_cache, v_cache, seq_lens, max_len, softmax_scale, sign_seed=0,
+                     workspace=None, out=None, stream=None):
+    """As tbq4_attn_decode, over 3-bit caches [B][Hkv][capacity][50]."""
+    _need(q, torch.float32, "q", 3)
+    _need(k_cache, torch.uint8, "k_cache", 4)
+    _need(v_cache, torch.uint8, "v_cache", 4)
+    _need(seq_lens, torch.int32, "seq_lens", 1)
+    B, Hq, d = q.shape
+    _, Hkv, cap, nb = k_cache.shape
+    if d != D or nb != BLOCK_BYTES3 or v_cache.shape != k_cache.shape or k_cache.shape[0] != B:
+        raise ValueError("shape mismatch between q and caches")
+    need = tbq4_decode_workspace_bytes(B, Hq, Hkv, max_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float16, device=q.device)
+    _need(out, torch.float16, "out", 3)
+    check(lib.tbq3_attn_decode(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), int(max_len), B, Hq, Hkv, cap,
+        float(softmax_scale), C.c_uint64(sign_seed), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)),
+        "tbq3_attn_decode")
     return out
 
 

@@ -24,6 +24,10 @@ SIGNATURES = {
     "tbq4_attn_decode_append": (_i, [_p, _p, _p, _p, _p, _p, _i32, _i, _i, _i, _i64, _f,
                                      _u64, _p, _sz, _p, _p]),
     "tbq4_quantize_append_paged": (_i, [_p, _i, _i, _i, _p, _p, _i, _i, _i64, _u64, _p, _p]),
+    "tbq3_block_bytes": (_sz, []),
+    "tbq3_cache_bytes": (_sz, [_i, _i, _i64]),
+    "tbq3_quantize_append": (_i, [_p, _i, _i, _i, _p, _i64, _u64, _p, _p]),
+    "tbq3_attn_decode": (_i, [_p, _p, _p, _p, _i32, _i, _i, _i, _i64, _f, _u64, _p, _sz, _p, _p]),
     "tbq4_attn_decode_paged": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i64, _p, _i32, _i, _i, _i,
                                     _f, _u64, _p, _sz, _p, _p]),
     "tbq4_decode_workspace_bytes_split": (_sz, [_i, _i, _i, _i32, _i32]),

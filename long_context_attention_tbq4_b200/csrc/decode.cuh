@@ -51,6 +51,7 @@ struct AttnParams {
     int max_pages;              // row length of block_table
     int page_size;              // tokens per page, a multiple of 32
     int64_t n_pages;
+    int tbq3;                   // 1: 3-bit caches [..][50] (decode only)
 };
 
 // Byte offset of token t of (sequence s, KV head g) in a paged pool.  An

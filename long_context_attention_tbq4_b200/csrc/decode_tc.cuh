@@ -182,10 +182,26 @@ __device__ __forceinline__ void split3(int x, int8_t &c0, int8_t &c1, int8_t &c2
     c2 = (int8_t)((x1 - b1) >> 8);
 }
 
+// TBQ3 (3-bit) blocks hold index i where TBQ4 holds nibble n: with n = i + 4
+// the level 2n - 15 equals the 3-bit level 2i - 7, and only the block
+// factor changes (S/7 instead of S/15).  So the 3-bit kernel expands each
+// group of eight 3-bit indices (a 24-bit word) into eight nibbles n = i + 4
+// in a register and runs the 4-bit arithmetic unchanged.
+__device__ __forceinline__ uint32_t tbq3_nibbles(uint32_t g) {
+    uint32_t t = (g & 0x00000FFFu) | ((g & 0x00FFF000u) << 4);    // 4 fields per half
+    t = (t & 0x003F003Fu) | ((t & 0x0FC00FC0u) << 2);             // 2 fields per byte
+    t = (t & 0x07070707u) | ((t & 0x38383838u) << 1);             // one per nibble
+    return t + 0x44444444u;                                       // i + 4, no carries
+}
+
 // kPaged: the caches are page pools addressed through p.block_table.
-template <bool kPaged>
+// kBits: 4 (TBQ4, 66-byte blocks) or 3 (TBQ3, 50-byte blocks; the stage
+// layout is the same, a 3-bit chunk fills 1,600 of its 2,112 bytes).
+template <bool kPaged, int kBits = 4>
 __global__ void __launch_bounds__(kTcWarps * 32, 1)
 decode_tc_kernel(const AttnParams p) {
+    static_assert(kBits == 4 || !kPaged, "paged caches hold 4-bit blocks");
+    constexpr int kBlk = kBits == 4 ? kBlockBytes : kBlockBytes3;
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *ring = smem;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kRingBytes);
@@ -239,14 +255,14 @@ decode_tc_kernel(const AttnParams p) {
             return *bad ? 0 : (int64_t)v << 6;
         } else {
             *bad = false;
-            return (int64_t)(t0 + ci * kChunk) * kBlockBytes;
+            return (int64_t)(t0 + ci * kChunk) * kBlk;
         }
     };
     // chunk ci -> warp w, stage st; ofs from chunk_ofs
     auto issue_for = [&](int w, int ci, int st, int32_t tend, int64_t ofs) {
         const int32_t start = t0 + ci * kChunk;
         const int32_t valid = min(kChunk, tend - start);
-        const uint32_t bytes = (uint32_t)((valid + 7) & ~7) * kBlockBytes;
+        const uint32_t bytes = (uint32_t)((valid + 7) & ~7) * kBlk;
         const uint32_t bar = smem_u32(bars) + (w * kTcStages + st) * 8;
         const uint32_t dst = smem_u32(ring) + w * kWarpRing + st * kStageBytes;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -333,7 +349,8 @@ decode_tc_kernel(const AttnParams p) {
         if (lane == 0) {
             // log2 logit = (2 S - 15 sum q) * S_k * scale * log2(e) / 15 * 2^(e-18),
             // and the integer MMAs return 16 S
-            const float fh = p.scale_log2 * (1.0f / 15.0f) * ldexpf(1.0f, e - kQBits);
+            const float fh = p.scale_log2 * (kBits == 4 ? 1.0f / 15.0f : 1.0f / 7.0f) *
+                             ldexpf(1.0f, e - kQBits);
             qpar[2 * warp + 0] = 0.125f * fh;
             qpar[2 * warp + 1] = -15.0f * (float)qsum * fh;
         }
@@ -381,12 +398,14 @@ decode_tc_kernel(const AttnParams p) {
     // of the chunk, 16 bytes from nibble byte 16c; every such row starts at
     // the same offset mod 4 (16-row and 8-row steps are multiples of 4 bytes),
     // so one aligned base and one funnel shift serve all four rows.
-    const int koff = r * kBlockBytes + 2 + 16 * c;
+    // (3-bit: 12 bytes from byte 12c, the same 32 dimensions)
+    const int koff = r * kBlk + 2 + (kBits == 4 ? 16 : 12) * c;
     const int kbase = koff & ~3;
     const uint32_t ksh = (uint32_t)(koff & 3) * 8u;
     // V: tokens 2c + {0, 1, 8, 9} (+16 for the second k-step), nibble
     // bytes 8r .. 8r+7; even tokens sit 2 bytes past a 4-byte boundary.
-    const int voff = 2 * c * kBlockBytes + 2 + 8 * r;
+    // (3-bit: 6 bytes from byte 6r)
+    const int voff = 2 * c * kBlk + 2 + (kBits == 4 ? 8 : 6) * r;
 
     float o[8][4];
 #pragma unroll
@@ -420,7 +439,7 @@ decode_tc_kernel(const AttnParams p) {
         const int32_t valid = min(kChunk, t1 - cstart);
         uint8_t *kst = ring_p + st * kStageBytes;
         uint8_t *vst = kst + kChunkBytes;
-        if (q0 == ci_app) {
+        if (kBits == 4 && q0 == ci_app) {
             const int jn = len - 1 - cstart;
             const uint32_t sbits = lane_sign_bits(p.sign_lo, p.sign_hi, lane);
             const int64_t row = ((int64_t)s * p.Hkv + g) * kD;
@@ -454,15 +473,38 @@ decode_tc_kernel(const AttnParams p) {
 #pragma unroll
         for (int tile = 0; tile < 2; ++tile) {
             int acc[3][4];
-            const uint8_t *k0 = kst + kbase + tile * 16 * kBlockBytes;   // row r
-            const uint8_t *k1 = k0 + 8 * kBlockBytes;                     // row r + 8
-            uint32_t w0[5], w1[5];
+            const uint8_t *k0 = kst + kbase + tile * 16 * kBlk;           // row r
+            const uint8_t *k1 = k0 + 8 * kBlk;                            // row r + 8
+            uint32_t xk0[4], xk1[4];     // nibble bytes 16c + 4i .. +3 of the two rows
+            if constexpr (kBits == 4) {
+                uint32_t w0[5], w1[5];
 #pragma unroll
-            for (int i = 0; i < 5; ++i) { w0[i] = ld_u32(k0 + 4 * i); w1[i] = ld_u32(k1 + 4 * i); }
+                for (int i = 0; i < 5; ++i) { w0[i] = ld_u32(k0 + 4 * i); w1[i] = ld_u32(k1 + 4 * i); }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    xk0[i] = __funnelshift_r(w0[i], w0[i + 1], ksh);
+                    xk1[i] = __funnelshift_r(w1[i], w1[i + 1], ksh);
+                }
+            } else {
+                uint32_t w0[4], w1[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) { w0[i] = ld_u32(k0 + 4 * i); w1[i] = ld_u32(k1 + 4 * i); }
+                const uint32_t *wr[2] = {w0, w1};
+                uint32_t *xr[2] = {xk0, xk1};
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t W0 = __funnelshift_r(wr[h][0], wr[h][1], ksh);
+                    const uint32_t W1 = __funnelshift_r(wr[h][1], wr[h][2], ksh);
+                    const uint32_t W2 = __funnelshift_r(wr[h][2], wr[h][3], ksh);
+                    xr[h][0] = tbq3_nibbles(W0 & 0x00FFFFFFu);
+                    xr[h][1] = tbq3_nibbles(__funnelshift_r(W0, W1, 24) & 0x00FFFFFFu);
+                    xr[h][2] = tbq3_nibbles(__funnelshift_r(W1, W2, 16) & 0x00FFFFFFu);
+                    xr[h][3] = tbq3_nibbles(W2 >> 8);
+                }
+            }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const uint32_t x0 = __funnelshift_r(w0[i], w0[i + 1], ksh);   // raw bytes
-                const uint32_t x1 = __funnelshift_r(w1[i], w1[i + 1], ksh);
+                const uint32_t x0 = xk0[i], x1 = xk1[i];                       // raw bytes
                 const uint32_t lo0 = x0 & 0x0F0F0F0Fu, lo1 = x1 & 0x0F0F0F0Fu;
 #pragma unroll
                 for (int pc = 0; pc < 3; ++pc) {
@@ -484,8 +526,8 @@ decode_tc_kernel(const AttnParams p) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int j = 8 * u + r;
-            sk[u] = ld_half(kst + j * kBlockBytes);
-            sv[u] = ld_half(vst + j * kBlockBytes);
+            sk[u] = ld_half(kst + j * kBlk);
+            sv[u] = ld_half(vst + j * kBlk);
             ta[u] = fmaf(sc[u >> 1][2 * (u & 1) + 0], f2a, bha);   // logit / S_k
             tb[u] = fmaf(sc[u >> 1][2 * (u & 1) + 1], f2b, bhb);
             xa[u] = fmaf(ta[u], sk[u], -m_a);                       // logit - m
@@ -559,8 +601,18 @@ decode_tc_kernel(const AttnParams p) {
             uint32_t xw[4][2];   // [token 2c, 2c+1, 2c+8, 2c+9][word]
 #pragma unroll
             for (int tt = 0; tt < 4; ++tt) {
-                const uint8_t *a = vst + voff + (16 * ks + (tt & 1) + 8 * (tt >> 1)) * kBlockBytes;
-                if (tt & 1) {            // odd token: its nibbles are 4-byte aligned
+                const int tok = 16 * ks + (tt & 1) + 8 * (tt >> 1);
+                const uint8_t *a = vst + voff + tok * kBlk;
+                if constexpr (kBits == 3) {
+                    // 6 bytes (two 24-bit groups) from an even offset: two
+                    // aligned words always cover them
+                    const int off = voff + tok * kBlk;
+                    const uint32_t lo = ld_u32(vst + (off & ~3)), hi = ld_u32(vst + (off & ~3) + 4);
+                    const uint32_t sh = (uint32_t)(off & 3) * 8u;
+                    const uint32_t d0 = __funnelshift_r(lo, hi, sh), d1 = hi >> sh;
+                    xw[tt][0] = tbq3_nibbles(d0 & 0x00FFFFFFu);
+                    xw[tt][1] = tbq3_nibbles(__funnelshift_r(d0, d1, 24) & 0x00FFFFFFu);
+                } else if (tt & 1) {     // odd token: its nibbles are 4-byte aligned
                     xw[tt][0] = ld_u32(a);
                     xw[tt][1] = ld_u32(a + 4);
                 } else {                 // even token: 2 bytes past a 4-byte boundary
@@ -694,7 +746,8 @@ decode_tc_kernel(const AttnParams p) {
             for (int w = 0; w < kTcWarps; ++w)
                 O = fmaf(wt[w * kMaxGroup + h], src[w * 32 * kLaneStride], O);
             const int64_t row = ((int64_t)s * p.Hq + g * G + h) * p.n_splits + split;
-            p.part_o[row * kD + d] = O * (256.0f / 15.0f);     // 2^8 undoes the scale of P-prime
+            // 2^8 undoes the scale of P-prime; the block factor is S/15 (S/7 for 3 bits)
+            p.part_o[row * kD + d] = O * (kBits == 4 ? 256.0f / 15.0f : 256.0f / 7.0f);
             if (d == 0) p.part_ml[row] = ml_h[h];
         }
     }

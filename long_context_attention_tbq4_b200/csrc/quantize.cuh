@@ -75,14 +75,22 @@ struct PageMap {
 
 constexpr int kQRows = 32;                                   // rows per warp and step
 constexpr int kQWarpBytes = kQRows * 512 + kQRows * kBlockBytes + kQRows * 8;
+// The 3-bit variant (TBQ3): the same rotation and scale, 8 levels
+// (i - 3.5)/3.5 * S, index clamp(rne(fl32(fl32(x/S)*3.5)+3.5), 0, 7) (4 when
+// S == 0), indices 8g .. 8g+7 as one little-endian 24-bit word (index 8g+k
+// at bits 3k .. 3k+2): 2 + 48 = 50 bytes per block.
+constexpr int kBlockBytes3 = 50;
 constexpr int kQThreads = 128;
 constexpr int kQSmemBytes = (kQThreads / 32) * kQWarpBytes;
 
+// kBits: 4 (TBQ4, 66-byte blocks) or 3 (TBQ3, 50-byte blocks).
+template <int kBits>
 __global__ void __launch_bounds__(kQThreads, 3)
 quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
                      const int32_t *__restrict__ start_pos, int64_t capacity, const SignTable sg,
                      const PageMap pm, uint8_t *__restrict__ cache) {
     extern __shared__ __align__(16) uint8_t qsm[];
+    constexpr int kBlk = kBits == 4 ? kBlockBytes : kBlockBytes3;
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     uint8_t *wsm = qsm + wib * kQWarpBytes;
     float4 *tile = reinterpret_cast<float4 *>(wsm);                          // [32][32]
@@ -108,9 +116,9 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
             } else if (pm.table) {
                 const int32_t pid = __ldg(pm.table + (int64_t)b * pm.max_pages + pos / pm.page_size);
                 if (pid < 0 || (int64_t)pid >= pm.n_pages) record_status(4u);
-                else doff = (((int64_t)pid * Hkv + h) * pm.page_size + pos % pm.page_size) * kBlockBytes;
+                else doff = (((int64_t)pid * Hkv + h) * pm.page_size + pos % pm.page_size) * kBlk;
             } else {
-                doff = (((int64_t)b * Hkv + h) * capacity + pos) * kBlockBytes;
+                doff = (((int64_t)b * Hkv + h) * capacity + pos) * kBlk;
             }
         }
         // load: row i, one 16-byte chunk per lane
@@ -159,31 +167,48 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
         uint16_t sb = __half_as_ushort(__float2half_rn(m));
         if ((sb & 0x7FFFu) == 0x7C00u) sb = 0x7BFFu;                 // saturate at 65504
         const float S = half_bits_to_float(sb);
-        uint16_t *mine = stage + lane * (kBlockBytes / 2);
+        uint16_t *mine = stage + lane * (kBlk / 2);
         mine[0] = sb;
         const float rs = S == 0.0f ? 0.0f : __frcp_rn(S);
-#pragma unroll
-        for (int w = 0; w < kD / 4; ++w) {                             // 4 nibbles per piece
-            uint32_t piece = 0;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float x = v[4 * w + k];
-                const float q0 = __fmul_rn(x, rs);
-                const float e = __fmaf_rn(-q0, S, x);
-                const float q = __fmaf_rn(e, rs, q0);               // x / S, correctly rounded
+        // x / S correctly rounded, then the codebook's index
+        auto index_of = [&](float x) -> uint32_t {
+            const float q0 = __fmul_rn(x, rs);
+            const float e = __fmaf_rn(-q0, S, x);
+            const float q = __fmaf_rn(e, rs, q0);
+            if constexpr (kBits == 4) {
                 const float u = __fadd_rn(__fmul_rn(q, 7.5f), 7.5f);
-                const uint32_t idx = S == 0.0f ? 8u : min(__float2uint_rn(u), 15u);
-                piece |= idx << (4 * k);
+                return S == 0.0f ? 8u : min(__float2uint_rn(u), 15u);
+            } else {
+                const float u = __fadd_rn(__fmul_rn(q, 3.5f), 3.5f);
+                return S == 0.0f ? 4u : min(__float2uint_rn(u), 7u);
             }
-            mine[1 + w] = (uint16_t)piece;
+        };
+        if constexpr (kBits == 4) {
+#pragma unroll
+            for (int w = 0; w < kD / 4; ++w) {                         // 4 nibbles per piece
+                uint32_t piece = 0;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) piece |= index_of(v[4 * w + k]) << (4 * k);
+                mine[1 + w] = (uint16_t)piece;
+            }
+        } else {
+#pragma unroll
+            for (int h2 = 0; h2 < kD / 16; ++h2) {                     // two 24-bit words
+                uint64_t wd = 0;                                       // = three pieces
+#pragma unroll
+                for (int k = 0; k < 16; ++k) wd |= (uint64_t)index_of(v[16 * h2 + k]) << (3 * k);
+                mine[1 + 3 * h2] = (uint16_t)wd;
+                mine[2 + 3 * h2] = (uint16_t)(wd >> 16);
+                mine[3 + 3 * h2] = (uint16_t)(wd >> 32);
+            }
         }
         doffs[lane] = doff;
         __syncwarp();
-        // store: the 32 blocks as 1,056 consecutive 16-bit pieces
+        // store: the 32 blocks as 32 x kBlk / 2 consecutive 16-bit pieces
 #pragma unroll
-        for (int k = 0; k < kBlockBytes / 2; ++k) {
+        for (int k = 0; k < kBlk / 2; ++k) {
             const int j = lane + 32 * k;
-            const int row = j / (kBlockBytes / 2), pc = j - row * (kBlockBytes / 2);
+            const int row = j / (kBlk / 2), pc = j - row * (kBlk / 2);
             const int64_t off = doffs[row];
             if (off >= 0) *reinterpret_cast<uint16_t *>(cache + off + 2 * pc) = stage[j];
         }

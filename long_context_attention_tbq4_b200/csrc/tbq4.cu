@@ -126,13 +126,17 @@ tbq4_status run_attention(AttnParams p, void *workspace, size_t ws_bytes,
     p.part_o = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.part_o);
     p.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) + w.part_ml);
     static bool attr_set[64] = {}, attr_paged[64] = {}, attr_mq[64] = {};  // once per device
+    static bool attr_3[64] = {};
     const bool mq = p.q_len > 1, paged = p.block_table != nullptr;
     if (mq && paged) return TBQ4_ERR_SHAPE;
+    if (p.tbq3 && (mq || paged || p.k_new)) return TBQ4_ERR_SHAPE;
     if (paged && p.split_tokens > kPidCap * kChunk) return TBQ4_ERR_SHAPE;
     if (mq ? !ensure_smem_attr((const void *)dmq::decode_mq_kernel, dmq::kSmemBytes, attr_mq)
            : paged ? !ensure_smem_attr((const void *)decode_tc_kernel<true>, kTcSmemBytesPaged,
                                        attr_paged)
-                   : !ensure_smem_attr((const void *)decode_tc_kernel<false>, kTcSmemBytes, attr_set))
+           : p.tbq3 ? !ensure_smem_attr((const void *)decode_tc_kernel<false, 3>, kTcSmemBytes,
+                                        attr_3)
+                    : !ensure_smem_attr((const void *)decode_tc_kernel<false>, kTcSmemBytes, attr_set))
         return TBQ4_ERR_LAUNCH;
     dim3 g1(p.n_splits, p.Hkv, p.nseq);
     if (g_ev_before) cudaEventRecord(g_ev_before, st);
@@ -140,6 +144,8 @@ tbq4_status run_attention(AttnParams p, void *workspace, size_t ws_bytes,
         dmq::decode_mq_kernel<<<g1, dmq::kThreads, dmq::kSmemBytes, st>>>(p);
     else if (paged)
         decode_tc_kernel<true><<<g1, kTcWarps * 32, kTcSmemBytesPaged, st>>>(p);
+    else if (p.tbq3)
+        decode_tc_kernel<false, 3><<<g1, kTcWarps * 32, kTcSmemBytes, st>>>(p);
     else
         decode_tc_kernel<false><<<g1, kTcWarps * 32, kTcSmemBytes, st>>>(p);
     // The combine is a programmatic dependent launch: its CTAs are placed as
@@ -209,7 +215,7 @@ namespace {
 
 tbq4_status quantize_impl(const float *src, int B, int n_new, int Hkv, const int32_t *start_pos,
                           int64_t capacity, uint64_t sign_seed, const PageMap &pm,
-                          uint8_t *cache, void *stream) {
+                          uint8_t *cache, void *stream, int bits = 4) {
     if (!src || !start_pos || !cache) return TBQ4_ERR_NULL;
     if (!aligned(src, 16) || !aligned(cache, 16) || !aligned(start_pos, 4))
         return TBQ4_ERR_ALIGN;
@@ -222,13 +228,18 @@ tbq4_status quantize_impl(const float *src, int B, int n_new, int Hkv, const int
     tbq4_signs(sign_seed, sg8);
     SignTable sg;
     for (int i = 0; i < kD; ++i) sg.s[i] = (float)sg8[i];
-    static bool attr_set[64] = {};    // set once per device
-    if (!ensure_smem_attr((const void *)quantize_rows_kernel, kQSmemBytes, attr_set))
-        return TBQ4_ERR_LAUNCH;
+    static bool attr4[64] = {}, attr3[64] = {};    // set once per device
+    const void *fn = bits == 3 ? (const void *)quantize_rows_kernel<3>
+                               : (const void *)quantize_rows_kernel<4>;
+    if (!ensure_smem_attr(fn, kQSmemBytes, bits == 3 ? attr3 : attr4)) return TBQ4_ERR_LAUNCH;
     int64_t blocks = ceil_div(rows, (int64_t)kQThreads);   // one row per thread
     if (blocks > (int64_t)kNumSMs * 3) blocks = (int64_t)kNumSMs * 3;
-    quantize_rows_kernel<<<(unsigned)blocks, kQThreads, kQSmemBytes, (cudaStream_t)stream>>>(
-        src, B, n_new, Hkv, start_pos, capacity, sg, pm, cache);
+    if (bits == 3)
+        quantize_rows_kernel<3><<<(unsigned)blocks, kQThreads, kQSmemBytes, (cudaStream_t)stream>>>(
+            src, B, n_new, Hkv, start_pos, capacity, sg, pm, cache);
+    else
+        quantize_rows_kernel<4><<<(unsigned)blocks, kQThreads, kQSmemBytes, (cudaStream_t)stream>>>(
+            src, B, n_new, Hkv, start_pos, capacity, sg, pm, cache);
     return launch_status();
 }
 
@@ -242,6 +253,21 @@ tbq4_status tbq4_quantize_append(const float *src, int B, int n_new, int Hkv,
     const PageMap contiguous = {nullptr, 0, 0, 0};
     return quantize_impl(src, B, n_new, Hkv, start_pos, capacity, sign_seed, contiguous, cache,
                          stream);
+}
+
+tbq4_status tbq3_quantize_append(const float *src, int B, int n_new, int Hkv,
+                                 const int32_t *start_pos, int64_t capacity,
+                                 uint64_t sign_seed, uint8_t *cache, void *stream) {
+    const PageMap contiguous = {nullptr, 0, 0, 0};
+    return quantize_impl(src, B, n_new, Hkv, start_pos, capacity, sign_seed, contiguous, cache,
+                         stream, 3);
+}
+
+size_t tbq3_block_bytes(void) { return kBlockBytes3; }
+
+size_t tbq3_cache_bytes(int batch, int n_kv_heads, int64_t capacity) {
+    if (batch <= 0 || n_kv_heads <= 0 || capacity <= 0) return 0;
+    return (size_t)batch * n_kv_heads * (size_t)capacity * kBlockBytes3;
 }
 
 tbq4_status tbq4_quantize_append_paged(const float *src, int B, int n_new, int Hkv,
@@ -297,7 +323,7 @@ tbq4_status decode_impl(const float *q, const uint8_t *k_cache, const uint8_t *v
                         int64_t capacity, float softmax_scale, uint64_t sign_seed,
                         int32_t split_tokens, void *workspace, size_t ws_bytes, uint16_t *out,
                         void *stream, const float *k_new, const float *v_new,
-                        const PagedArgs *pg = nullptr) {
+                        const PagedArgs *pg = nullptr, int bits = 4) {
     if (!q || !k_cache || !v_cache || !seq_lens || !workspace || !out)
         return TBQ4_ERR_NULL;
     if (pg) {
@@ -318,8 +344,9 @@ tbq4_status decode_impl(const float *q, const uint8_t *k_cache, const uint8_t *v
     p.q_bf16 = 0;
     p.k = k_cache;
     p.v = v_cache;
-    p.head_stride = capacity * kBlockBytes;
+    p.head_stride = capacity * (bits == 3 ? kBlockBytes3 : kBlockBytes);
     p.seq_stride = (int64_t)Hkv * p.head_stride;
+    p.tbq3 = bits == 3;
     p.seq_lens = seq_lens;
     p.max_len = max_len;
     p.capacity = capacity;
@@ -436,6 +463,15 @@ tbq4_status tbq4_attn_decode_paged(const float *q, const float *k_new, const flo
     const PagedArgs pg = {block_table, max_pages, page_size, n_pages};
     return decode_impl(q, k_pool, v_pool, seq_lens, max_len, B, Hq, Hkv, 0, softmax_scale,
                        sign_seed, 0, workspace, ws_bytes, out, stream, k_new, v_new, &pg);
+}
+
+tbq4_status tbq3_attn_decode(const float *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                             const int32_t *seq_lens, int32_t max_len, int B, int Hq, int Hkv,
+                             int64_t capacity, float softmax_scale, uint64_t sign_seed,
+                             void *workspace, size_t ws_bytes, uint16_t *out, void *stream) {
+    return decode_impl(q, k_cache, v_cache, seq_lens, max_len, B, Hq, Hkv, capacity,
+                       softmax_scale, sign_seed, 0, workspace, ws_bytes, out, stream, nullptr,
+                       nullptr, nullptr, 3);
 }
 
 tbq4_status tbq4_attn_decode(const float *q, const uint8_t *k_cache,

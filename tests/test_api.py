@@ -239,3 +239,35 @@ def test_page_table_generator():
         k = (n + 31) // 32
         assert (table[b, :k] >= 0).all() and (table[b, k:] == -1).all()
     assert np.array_equal(W.page_table(3, lens, 32, spare=2)[0], table)   # seeded
+
+
+def test_tbq3_rejects_bad_arguments(T):
+    from long_context_attention_tbq4_b200._lib import lib as L
+    assert L.tbq3_block_bytes() == 50
+    assert L.tbq3_cache_bytes(2, 4, 1024) == 2 * 4 * 1024 * 50
+    assert L.tbq3_cache_bytes(0, 4, 1024) == 0
+
+    def d(**kw):
+        a = dict(q=A, k=A, v=A, lens=A, max_len=64, B=1, Hq=8, Hkv=2, cap=64, scale=0.1,
+                 seed=0, ws=A2, ws_bytes=1 << 30, out=A, stream=None)
+        a.update(kw)
+        return L.tbq3_attn_decode(a["q"], a["k"], a["v"], a["lens"], a["max_len"], a["B"],
+                                  a["Hq"], a["Hkv"], a["cap"], a["scale"], a["seed"], a["ws"],
+                                  a["ws_bytes"], a["out"], a["stream"])
+    assert d(q=None) == 1
+    assert d(k=MIS) == 2
+    assert d(Hq=7) == 3
+    assert d(cap=60) == 4
+    assert d(max_len=65) == 4
+    assert d(ws_bytes=16) == 5
+
+    def q(**kw):
+        a = dict(src=A, B=1, n=4, Hkv=2, pos=A, cap=64, seed=0, cache=A, stream=None)
+        a.update(kw)
+        return L.tbq3_quantize_append(a["src"], a["B"], a["n"], a["Hkv"], a["pos"], a["cap"],
+                                      a["seed"], a["cache"], a["stream"])
+    assert q(src=None) == 1
+    assert q(cache=C.c_void_p(0x10002)) == 2
+    assert q(Hkv=0) == 3
+    assert q(cap=12) == 4
+    assert q(n=0) == 0
