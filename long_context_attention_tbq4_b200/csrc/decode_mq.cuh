@@ -52,6 +52,12 @@ constexpr int kMaxQLen = 4;
 constexpr uint32_t kSpin = 1u << 22;
 constexpr float kRescale = 8.0f;                        // log2 units
 constexpr int kQBits = 18;                              // |q_int| <= 2^18
+// Registers per thread after the prologue, per warpgroup: producer / MMA
+// (warps 0-3), dequantisation (4-7), softmax (8-23).  The sum over the 24
+// warps must fit in what the CTA was launched with, 768 threads x 80.
+constexpr uint32_t kRegsCtl = 24, kRegsDeq = 72, kRegsSoft = 96;
+static_assert(4 * kRegsCtl + 4 * kRegsDeq + 16 * kRegsSoft <= 24 * 80,
+              "register split exceeds the launch budget");
 
 // One operand buffer (double-buffered): K tile, V^T tile, P'^T tile, the
 // tile's S_k and S_v.  Offsets from a 1024-aligned base.
@@ -279,7 +285,9 @@ decode_mq_kernel(const AttnParams p) {
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_ptr;
 
-    if (warp == 0) {
+    if (warp < 4) {
+      tc::regs_dec<kRegsCtl>();
+      if (warp == 0) {
         // ======================= producer ====================================
         // Each tile's K and V rows go as 32-row pieces, one per lane, so the
         // copy engine has many requests in flight.
@@ -356,7 +364,9 @@ decode_mq_kernel(const AttnParams p) {
                 }
             }
         }
+      }
     } else if (warp >= kDeqWarp0 && warp < kDeqWarp0 + kDeqWarps) {
+        tc::regs_dec<kRegsDeq>();
         // ======================= dequantisation ==============================
         const int d = threadIdx.x - 32 * kDeqWarp0;     // 0..127
         for (int j = 0; j < n_tiles; ++j) {
@@ -430,6 +440,7 @@ decode_mq_kernel(const AttnParams p) {
             }
         }
     } else if (warp >= kSoftWarp0) {
+        tc::regs_inc<kRegsSoft>();
         // ======================= softmax =====================================
         const int ws = warp - kSoftWarp0;                   // 0..15
         const int wg = ws >> 2;                             // query rows 8 wg .. 8 wg + 7
