@@ -22,10 +22,9 @@
 // output errors of a few 1e-3 where one token dominates; 18 bits keep the
 // logit error below 1e-3 of a log2 unit even in the worst case.)
 // V operand: pairs of tokens are interleaved with PRMT so that one register
-// holds the same dimension of two tokens; the nibbles enter as fp16
-// subnormals, masked in place, and the odd level 2n - 15 is restored at the
-// end (see lvl_lo).  P' = p * S_v (the block scale of V), so O = sum_t p_t
-// S_v,t (2n-15) / 15.
+// holds the same dimension of two tokens; the levels enter as (n - 8) 2^-10
+// and the odd level 2n - 15 is restored at the end (see lvl_lo).  P' = p * S_v (the
+// block scale of V), so O = sum_t p_t S_v,t (2n-15) / 15.
 // Softmax runs in fp32 in the log2 domain; the running max is per head and
 // the accumulators are only rescaled when some logit exceeds it by 2^3
 // (tested with one vote per chunk; the chunk max is only formed then).
@@ -145,29 +144,32 @@ __device__ __forceinline__ float ld_half(const uint8_t *p) {
     return __half2float(*reinterpret_cast<const __half *>(p));
 }
 
-// V levels enter the tensor cores as fp16 subnormals, one LOP3 per register:
-// masking a nibble into the low mantissa bits of an fp16 with a zero
-// exponent field gives n 2^-24 (bits 0-3) or 16 n 2^-24 = n 2^-20 (bits
-// 4-7), exact, and the fp16 MMA takes subnormal operands exactly.  Products
-// with P' and their fp32 sums stay far above fp32's normal range limit.
-// The low nibbles (even dimensions) land in the rows r of an m-tile, the
-// high ones (odd dimensions) in the rows r + 8, so with R = sum_t P'_t (one
-// extra MMA per k-step with an all-ones A operand):
-//   even dimensions  sum_t P'_t (2n - 15) = 2^25 O_lo - 15 R
-//   odd dimensions   sum_t P'_t (2n - 15) = 2^21 O_hi - 15 R
-// The subtraction loses about 2^-24 * 15 R per accumulation, against
-// results of order R.
+// V levels enter the tensor cores as (n - 8) 2^-10, exact in fp16, from one
+// LOP3 and one HFMA2 per register: masking a nibble into the low mantissa
+// bits of an fp16 with a zero exponent field gives the subnormal n 2^-24
+// (bits 0-3) or 16 n 2^-24 (bits 4-7); fp16 arithmetic keeps subnormals, so
+// x 2^14 - 2^-7 (resp. x 2^10 - 2^-7) is (n - 8) 2^-10 with no rounding.
+// Since 2n - 15 = 2 (n - 8) + 1, O = 2^11 sum_t P'_t (n_t - 8) 2^-10 +
+// sum_t P'_t; the second sum (R) comes from one extra MMA per k-step with an
+// all-ones A operand.
+constexpr uint32_t kH2Pow14 = 0x74007400u;     // {2^14, 2^14}
+constexpr uint32_t kH2Pow10 = 0x64006400u;     // {2^10, 2^10}
+constexpr uint32_t kH2NegBias = 0xA000A000u;   // {-2^-7, -2^-7}
 constexpr uint32_t kH2Ones = 0x3C003C00u;      // {1, 1}
-constexpr float kLoLevelScale = 33554432.0f;   // 2 * 2^24
-constexpr float kHiLevelScale = 2097152.0f;    // 2 * 2^20
+constexpr float kVLevelScale = 2048.0f;        // 2 * 2^10
 
-// low nibbles of bytes 0 and 2 -> {n 2^-24, n 2^-24}
-__device__ __forceinline__ uint32_t lvl_lo(uint32_t v) {
-    return v & 0x000F000Fu;
+__device__ __forceinline__ uint32_t hfma2_u32(uint32_t x, uint32_t a, uint32_t b) {
+    __half2 r = __hfma2(*reinterpret_cast<__half2 *>(&x), *reinterpret_cast<__half2 *>(&a),
+                        *reinterpret_cast<__half2 *>(&b));
+    return *reinterpret_cast<uint32_t *>(&r);
 }
-// high nibbles of bytes 0 and 2 -> {n 2^-20, n 2^-20}
+// low nibbles of bytes 0 and 2 -> {(n - 8) 2^-10, (n - 8) 2^-10}
+__device__ __forceinline__ uint32_t lvl_lo(uint32_t v) {
+    return hfma2_u32(v & 0x000F000Fu, kH2Pow14, kH2NegBias);
+}
+// high nibbles of bytes 0 and 2 -> {(n - 8) 2^-10, (n - 8) 2^-10}
 __device__ __forceinline__ uint32_t lvl_hi(uint32_t v) {
-    return v & 0x00F000F0u;
+    return hfma2_u32(v & 0x00F000F0u, kH2Pow10, kH2NegBias);
 }
 
 // x = c0 + 256 c1 + 65536 c2 with c0, c1 in [-128, 127]
@@ -690,15 +692,14 @@ decode_tc_kernel(const AttnParams p) {
     float *wt = l_w + kTcWarps * kMaxGroup;                              // [W][8]
     float2 *ml_h = reinterpret_cast<float2 *>(wt + kTcWarps * kMaxGroup);  // [8]
     {
-        // sum_t P'_t (2n - 15): elements 0, 1 sit in rows r (even dimensions,
-        // low nibbles), elements 2, 3 in rows r + 8 (odd, high nibbles)
+        // sum_t P'_t (2n - 15) = 2^11 sum_t P'_t (n - 8) 2^-10 + sum_t P'_t
         float4 *mine = reinterpret_cast<float4 *>(o_w + (warp * 32 + lane) * kLaneStride);
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt)
-            mine[mt] = make_float4(fmaf(kLoLevelScale, o[mt][0], -15.0f * rr[0]),
-                                   fmaf(kLoLevelScale, o[mt][1], -15.0f * rr[1]),
-                                   fmaf(kHiLevelScale, o[mt][2], -15.0f * rr[2]),
-                                   fmaf(kHiLevelScale, o[mt][3], -15.0f * rr[3]));
+            mine[mt] = make_float4(fmaf(kVLevelScale, o[mt][0], rr[0]),
+                                   fmaf(kVLevelScale, o[mt][1], rr[1]),
+                                   fmaf(kVLevelScale, o[mt][2], rr[2]),
+                                   fmaf(kVLevelScale, o[mt][3], rr[3]));
     }
     if (r == 0) {
         m_w[warp * kMaxGroup + 2 * c] = m_a;
