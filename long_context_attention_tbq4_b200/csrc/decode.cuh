@@ -251,4 +251,28 @@ decode_combine_kernel(const AttnParams p) {
     }
 }
 
+
+// The same merge with one warp per output row (sequence or query position
+// s, query head h): for few splits per row and many rows, as in the chunked
+// prefill (a few key splits for each of n_new x Hq rows), where a 16-warp
+// CTA per row would mostly idle.  Each warp runs the log-sum-exp merge over
+// its row's splits, normalises, rotates back and stores.  Launched as a
+// programmatic dependent of the attention kernel.
+__global__ void __launch_bounds__(kCombineWarps * 32)
+combine_rows_kernel(const AttnParams p, int n_rows) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int lane = threadIdx.x & 31;
+    const int rowid = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+    if (rowid >= n_rows) return;
+    const int s = rowid / p.Hq, h = rowid - (rowid / p.Hq) * p.Hq;
+    const int used = used_splits(p, seq_length(p, s));
+    const int64_t row0 = ((int64_t)s * p.Hq + h) * p.n_splits;
+    float4 O;
+    float M, L;
+    merge_split_run(p, row0, used, 0, 1, lane, O, M, L);
+    const float inv = L > 0.f ? 1.0f / L : 0.f;
+    float v[4] = {O.x * inv, O.y * inv, O.z * inv, O.w * inv};
+    store_row(p, s, h, v, lane);
+}
+
 }  // namespace tbq4

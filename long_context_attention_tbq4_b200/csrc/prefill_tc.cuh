@@ -158,6 +158,8 @@ prefill_tc_kernel(const PrefillParams p) {
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = tc::smem_addr(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the dependent combine may be scheduled from now on (it waits for this grid)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // ---- work unit ---------------------------------------------------------
     const int split = blockIdx.x;

@@ -216,4 +216,50 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
     }
 }
 
+
+// Few rows (a prefill chunk, a decode step): one warp per row with the warp
+// encoder, so that even a few thousand rows spread over every SM instead of
+// the handful of blocks the thread-per-row kernel would fill.  The same
+// bytes as quantize_rows_kernel<4> (the same encoding steps in the same
+// order); rows are taken in source order (b, t, h), so the loads of
+// consecutive warps are contiguous.
+constexpr int kQWarpRowsPerBlock = 8;               // warps per block
+
+__global__ void __launch_bounds__(kQWarpRowsPerBlock * 32)
+quantize_warp_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
+                          const int32_t *__restrict__ start_pos, int64_t capacity,
+                          uint64_t sign_lo, uint64_t sign_hi, const PageMap pm,
+                          uint8_t *__restrict__ cache) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t rows = (uint32_t)B * (uint32_t)n_new * (uint32_t)Hkv;   // < 2^31 (host)
+    const uint32_t sbits = lane_sign_bits(sign_lo, sign_hi, lane);
+    for (uint32_t r = blockIdx.x * kQWarpRowsPerBlock + (threadIdx.x >> 5); r < rows;
+         r += gridDim.x * kQWarpRowsPerBlock) {
+        const uint32_t h = r % (uint32_t)Hkv, bt = r / (uint32_t)Hkv;
+        const uint32_t t = bt % (uint32_t)n_new, b = bt / (uint32_t)n_new;
+        const float4 x4 = __ldcs(reinterpret_cast<const float4 *>(src + (int64_t)r * kD) + lane);
+        float v[4] = {x4.x, x4.y, x4.z, x4.w};
+        uint16_t sb;
+        const uint32_t packed = encode_row(v, sbits, lane, &sb);
+        const int64_t pos = (int64_t)__ldg(start_pos + b) + t;
+        int64_t doff = -1;
+        if (pos >= 0 && pos < capacity) {
+            if (pm.table) {
+                const int32_t pid = __ldg(pm.table + (int64_t)b * pm.max_pages + pos / pm.page_size);
+                if (pid >= 0 && (int64_t)pid < pm.n_pages)
+                    doff = (((int64_t)pid * Hkv + h) * pm.page_size + pos % pm.page_size) * kBlockBytes;
+            } else {
+                doff = (((int64_t)b * Hkv + h) * capacity + pos) * kBlockBytes;
+            }
+        }
+        if (doff < 0) {
+            if (lane == 0) record_status(4u /* TBQ4_ERR_CAPACITY */);
+            continue;
+        }
+        uint8_t *dst = cache + doff;
+        reinterpret_cast<uint16_t *>(dst + 2)[lane] = (uint16_t)packed;
+        if (lane == 0) *reinterpret_cast<uint16_t *>(dst) = sb;
+    }
+}
+
 }  // namespace tbq4

@@ -213,6 +213,10 @@ void tbq4_signs(uint64_t seed, int8_t out[128]) {
 
 namespace {
 
+// Below this many rows the thread-per-row encoder fills too few blocks
+// (rows / 128) to keep the GPU busy; the warp-per-row encoder takes over.
+constexpr int64_t kSmallAppendRows = 16384;
+
 tbq4_status quantize_impl(const float *src, int B, int n_new, int Hkv, const int32_t *start_pos,
                           int64_t capacity, uint64_t sign_seed, const PageMap &pm,
                           uint8_t *cache, void *stream, int bits = 4) {
@@ -224,6 +228,17 @@ tbq4_status quantize_impl(const float *src, int B, int n_new, int Hkv, const int
     if (n_new == 0) return TBQ4_OK;
     const int64_t rows = (int64_t)B * n_new * Hkv;
     if (rows > 0x7FFFFFFFLL) return TBQ4_ERR_SHAPE;      // rows are indexed in 32 bits
+    if (bits == 4 && rows < kSmallAppendRows) {
+        // few rows: one warp per row over every SM
+        uint64_t lo, hi;
+        sign_words(sign_seed, &lo, &hi);
+        int64_t blocks = ceil_div(rows, (int64_t)kQWarpRowsPerBlock);
+        if (blocks > (int64_t)kNumSMs * 8) blocks = (int64_t)kNumSMs * 8;
+        quantize_warp_rows_kernel<<<(unsigned)blocks, kQWarpRowsPerBlock * 32, 0,
+                                    (cudaStream_t)stream>>>(src, B, n_new, Hkv, start_pos,
+                                                            capacity, lo, hi, pm, cache);
+        return launch_status();
+    }
     int8_t sg8[kD];
     tbq4_signs(sign_seed, sg8);
     SignTable sg;
@@ -578,7 +593,20 @@ tbq4_status tbq4_attn_prefill_chunk(const uint16_t *q, int n_new, int64_t n_cach
     c.part_ml = pp.part_ml;
     c.out = out;
     c.out_bf16 = 1;
-    decode_combine_kernel<<<dim3(Hq, n_new), kCombineWarps * 32, 0, st>>>(c);
+    // one warp per (position, head) row, a programmatic dependent launch
+    const int n_rows = n_new * Hq;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((n_rows + kCombineWarps - 1) / kCombineWarps));
+    cfg.blockDim = dim3(kCombineWarps * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, combine_rows_kernel, c, n_rows) != cudaSuccess)
+        return TBQ4_ERR_LAUNCH;
     return launch_status();
 }
 
