@@ -184,6 +184,22 @@ def flush_l2(buf):
     buf.sum()
 
 
+def capture_graph(torch, fn):
+    """fn captured as a CUDA graph, after one run on a side stream (the usual
+    warm-up before capture)."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
 def bench_decode(T, torch, case, N, step_bytes, kernel_bytes, steps, warmup, flush):
     dev = torch.device("cuda")
     cap = N
@@ -227,8 +243,25 @@ def bench_decode(T, torch, case, N, step_bytes, kernel_bytes, steps, warmup, flu
     T.tbq4_set_timing_events(None, None)
     torch.cuda.synchronize()
     barrier()
-    step_ms = [e0.elapsed_time(e1) for e0, e1, _, _ in ev]
+    eager_ms = [e0.elapsed_time(e1) for e0, e1, _, _ in ev]
     kern_ms = [k0.elapsed_time(k1) for _, _, k0, k1 in ev]
+
+    # The step as a serving loop runs it: captured once as a CUDA graph (the
+    # launch shape depends only on max_len, the lengths are read on the
+    # device) and replayed; each replay is the same two kernels.
+    g_step = capture_graph(torch, step)
+    ev = timing_events(torch, steps)
+    barrier()
+    torch.cuda.synchronize()
+    for e0, e1, _, _ in ev:
+        flush_l2(flush)
+        e0.record()
+        g_step.replay()
+        e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    step_ms = [e0.elapsed_time(e1) for e0, e1, _, _ in ev]
+    del g_step
 
     # end to end: the step's inputs from pinned host memory, the output back
     q_h = torch.from_numpy(case.q).pin_memory()
@@ -247,6 +280,7 @@ def bench_decode(T, torch, case, N, step_bytes, kernel_bytes, steps, warmup, flu
     for _ in range(warmup):
         e2e_step()
     torch.cuda.synchronize()
+    # (eager: captured in a graph, the pinned-memory copies ran slower)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(steps)]
     barrier()
@@ -261,8 +295,8 @@ def bench_decode(T, torch, case, N, step_bytes, kernel_bytes, steps, warmup, flu
     assert T.tbq4_get_device_status() == 0
     h2d = q_h.numel() * 4 + kn_h.numel() * 4 + vn_h.numel() * 4
     d2h = out_h.numel() * 2
-    return {"step_ms": step_ms, "kern_ms": kern_ms, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
-            "launches_per_step": 2, "out": out.float().cpu().numpy()}
+    return {"step_ms": step_ms, "eager_ms": eager_ms, "kern_ms": kern_ms, "e2e_ms": e2e_ms,
+            "h2d": h2d, "d2h": d2h, "launches_per_step": 2, "out": out.float().cpu().numpy()}
 
 
 def bench_prefill(T, torch, steps, warmup, flush):
@@ -517,8 +551,11 @@ def main():
                    "Hkv": case.Hkv, "head_dim": D, "kv_format": "tbq4 (66 B / 128 values)",
                    "l2": "flushed before every timed step: 512 MiB written, then read back "
                          "(no hits, no dirty lines left)",
+                   "launch": "each step is one replay of a CUDA graph captured once "
+                             "(decode kernel + combine); e2e launches eagerly",
                    "parallelism": "replicas" if world > 1 else "single"},
         "step_bytes": step_bytes,
+        "ms_per_step_eager": max_over_ranks(torch, float(np.mean(dec["eager_ms"]))),
         "pct_hbm_peak": value / world / peaks["hbm_gbs"],
         # the split kernel and its combine (a programmatic dependent launch,
         # no gap between them) are timed as one region
