@@ -51,7 +51,7 @@ def parse():
     ap.add_argument("--prefill-steps", type=int, default=5)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["decode", "prefill"], default=None,
+    ap.add_argument("--profile", choices=["decode", "prefill", "quantize"], default=None,
                     help="only run warm-up + steps of one workload's step, untimed, with "
                          "no flush buffer (a small footprint for ncu captures)")
     return ap.parse_args()
@@ -72,8 +72,10 @@ def measured_peaks():
 # Source files each profiled kernel is built from: a recorded ncu traffic
 # figure is only reported while these files are unchanged.
 KERNEL_SOURCES = {
-    "decode_tc_kernel": ["common.cuh", "quantize.cuh", "decode.cuh", "decode_tc.cuh"],
+    "decode_tc_kernel": ["common.cuh", "mbarrier.cuh", "quantize.cuh", "decode.cuh",
+                         "decode_tc.cuh"],
     "prefill_tc_kernel": ["common.cuh", "decode.cuh", "tcgen05.cuh", "prefill_tc.cuh"],
+    "quantize_rows_kernel": ["common.cuh", "mbarrier.cuh", "quantize.cuh"],
 }
 
 
@@ -420,6 +422,21 @@ def profile_prefill(T, torch, n_steps):
     return 0
 
 
+def profile_quantize(T, torch, case, N, n_steps):
+    """Bulk quantise-appends of the 262K K rows (1,048,576 rows, 537 MB in)
+    with nothing else on the device (for ncu)."""
+    dev = torch.device("cuda")
+    kc = T.empty_cache(1, case.Hkv, N)
+    src = torch.from_numpy(np.ascontiguousarray(case.k[0])[None]).to(dev)
+    zero = torch.zeros(1, dtype=torch.int32, device=dev)
+    for _ in range(n_steps):
+        T.tbq4_quantize_append(src, zero, kc, case.sign_seed)
+    torch.cuda.synchronize()
+    assert T.tbq4_get_device_status() == 0
+    print("profile: %d appends of %d rows" % (n_steps, N * case.Hkv))
+    return 0
+
+
 # ------------------------------------------------------------ CPU baseline
 def oracle_decode_sample(case, N, rows):
     """Oracle caches (built once, untimed) and a timed call on `rows`."""
@@ -540,6 +557,8 @@ def main():
         return profile_decode(T, torch, case, N, args.steps + args.warmup)
     if args.profile == "prefill":
         return profile_prefill(T, torch, args.steps + args.warmup)
+    if args.profile == "quantize":
+        return profile_quantize(T, torch, case, N, args.steps + args.warmup)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
     uuid = str(getattr(torch.cuda.get_device_properties(local), "uuid", "") or "")
     with Clocks(uuid) as clk:

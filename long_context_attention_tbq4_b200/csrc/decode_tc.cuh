@@ -31,6 +31,7 @@
 #pragma once
 #include "common.cuh"
 #include "decode.cuh"
+#include "mbarrier.cuh"
 #include "quantize.cuh"
 
 namespace tbq4 {
@@ -51,7 +52,6 @@ constexpr int kTcSmemBytes = kRingBytes + kBarBytes + kQScratchBytes + 128;
 constexpr int kPidCap = 4096;
 constexpr int kTcSmemBytesPaged = kTcSmemBytes + kPidCap * 4;
 static_assert(kTcSmemBytesPaged <= 227 * 1024, "shared memory per CTA");
-constexpr uint32_t kSpinLimit = 1u << 22;                  // bounded mbarrier wait
 constexpr int kQBits = 18;                                 // |q_int| <= 2^18
 
 static_assert(kStageBytes % 16 == 0, "stage must keep 16-byte alignment");
@@ -59,46 +59,6 @@ constexpr float kLazyRescale = 8.0f;                       // log2 units
 static_assert(kRingBytes >= kTcWarps * 32 * 36 * 4 + 3 * kTcWarps * kMaxGroup * 4 +
                                 kMaxGroup * 8,
               "merge buffers reuse the ring");
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Waits for the phase with the given parity; gives up after kSpinLimit
-// polls and returns false (warp-uniform).
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
-    bool ok = false;
-    for (uint32_t i = 0; i < kSpinLimit && !ok; ++i) ok = mbar_try_wait(bar, parity);
-    return __all_sync(kFull, ok);
-}
-
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
-                                         uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
 
 // The MMA wrappers are pure register operations (not volatile), so the
 // compiler may interleave them with the unpacking of the next operands.

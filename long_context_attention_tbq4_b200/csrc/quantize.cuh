@@ -9,6 +9,7 @@
 //                         the bulk append (HBM-bound: 512 bytes in, 66 out)
 #pragma once
 #include "common.cuh"
+#include "mbarrier.cuh"
 
 namespace tbq4 {
 
@@ -46,8 +47,9 @@ struct SignTable {
     float s[kD];
 };
 
-// One thread encodes one whole 128-value row (rows are independent, so a
-// thread per row keeps the transform in registers, with no shuffles):
+// Bulk append: one thread encodes one whole 128-value row (rows are
+// independent, so a thread per row keeps the transform in registers, with no
+// shuffles):
 //   rotation  the same butterflies in the same order as warp_fwht128 (stride
 //             1 first; lower = a + b, upper = a - b, each rounded on its own).
 //             The sign flip is exact, so the first stage is
@@ -58,12 +60,16 @@ struct SignTable {
 //             r = RN(1/S) once per row, q0 = RN(x r), e = x - q0 S (exact with
 //             FMA), q = RN(q0 + e r).  The conversion to unsigned saturates
 //             negative values to 0, which with min(., 15) is the clamp.
-// Memory: a warp takes 32 rows in head-major order (row = (b Hkv + h) n_new
-// + t), so its 32 blocks are contiguous in the cache.  The rows come in with
-// one 512-byte load per row across the warp into a shared tile (16-byte
-// chunk c of row i at position c ^ (i % 8), so the per-thread reads of a
-// whole row are free of bank conflicts), and the 32 blocks go out from a
-// shared staging area as consecutive 16-bit pieces.
+// Memory: rows go in groups of 32 in head-major order (row = (b Hkv + h)
+// n_new + t), so a group's 32 blocks are contiguous in the cache.  One CTA
+// of eight warps per SM, two warps per scheduler (so a thread can keep its
+// row's 128 values in registers: a scheduler's register file is a quarter
+// of the SM's).  Each warp owns one shared-memory stage: a group comes in as
+// one 512-byte cp.async.bulk per row (rows 528 bytes apart, so the
+// per-thread reads of a whole row are free of bank conflicts); once the
+// rows are in registers the warp sends its next group's copies into the
+// same stage, and they land while this group is encoded.  The blocks go out
+// from a per-warp staging area as consecutive 16-bit pieces.
 // Paged destination: row (b, pos) goes to page table[b][pos / page_size],
 // row pos % page_size, of a pool [n_pages][Hkv][page_size][66].  A null
 // table means the contiguous cache [B][Hkv][capacity][66].
@@ -73,43 +79,69 @@ struct PageMap {
     int64_t n_pages;
 };
 
-constexpr int kQRows = 32;                                   // rows per warp and step
-constexpr int kQWarpBytes = kQRows * 512 + kQRows * kBlockBytes + kQRows * 8;
 // The 3-bit variant (TBQ3): the same rotation and scale, 8 levels
 // (i - 3.5)/3.5 * S, index clamp(rne(fl32(fl32(x/S)*3.5)+3.5), 0, 7) (4 when
 // S == 0), indices 8g .. 8g+7 as one little-endian 24-bit word (index 8g+k
 // at bits 3k .. 3k+2): 2 + 48 = 50 bytes per block.
 constexpr int kBlockBytes3 = 50;
-constexpr int kQThreads = 128;
-constexpr int kQSmemBytes = (kQThreads / 32) * kQWarpBytes;
 
-// kBits: 4 (TBQ4, 66-byte blocks) or 3 (TBQ3, 50-byte blocks).
+constexpr int kQRows = 32;                                   // rows per group
+constexpr int kQWarps = 8;                                   // warps per CTA
+constexpr int kQRowStride = 512 + 16;                        // bytes between staged rows
+constexpr int kQStageBytes = kQRows * kQRowStride;
+constexpr int kQOutBytes = kQRows * kBlockBytes + kQRows * 8;   // blocks + destinations
+constexpr int kQThreads = kQWarps * 32;
+constexpr int kQRingBytes = kQWarps * kQStageBytes;
+constexpr int kQSmemBytes = kQRingBytes + kQWarps * kQOutBytes + kQWarps * 8;
+static_assert(kQSmemBytes <= 227 * 1024, "shared memory per CTA");
+static_assert(kQStageBytes % 16 == 0 && kQRowStride % 16 == 0 && kQOutBytes % 16 == 0,
+              "bulk copies and staged rows stay 16-byte aligned");
+
+// kBits: 4 (TBQ4, 66-byte blocks) or 3 (TBQ3, 50-byte blocks).  Group k of a
+// CTA is group blockIdx.x + k gridDim.x, encoded by warp k % kQWarps.
 template <int kBits>
-__global__ void __launch_bounds__(kQThreads, 3)
+__global__ void __launch_bounds__(kQThreads, 1)
 quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
                      const int32_t *__restrict__ start_pos, int64_t capacity, const SignTable sg,
                      const PageMap pm, uint8_t *__restrict__ cache) {
-    extern __shared__ __align__(16) uint8_t qsm[];
+    extern __shared__ __align__(128) uint8_t qsm[];
     constexpr int kBlk = kBits == 4 ? kBlockBytes : kBlockBytes3;
-    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-    uint8_t *wsm = qsm + wib * kQWarpBytes;
-    float4 *tile = reinterpret_cast<float4 *>(wsm);                          // [32][32]
-    uint16_t *stage = reinterpret_cast<uint16_t *>(wsm + kQRows * 512);      // [32][33]
-    int64_t *doffs = reinterpret_cast<int64_t *>(wsm + kQRows * 512 + kQRows * kBlockBytes);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t rows = (uint32_t)B * (uint32_t)n_new * (uint32_t)Hkv;    // < 2^31 (host)
     const uint32_t groups = (rows + kQRows - 1) / kQRows;
-    const uint32_t wstride = gridDim.x * (kQThreads / 32);
-    for (uint32_t gi = blockIdx.x * (kQThreads / 32) + wib; gi < groups; gi += wstride) {
-        // this lane's row and its source and destination
+    const uint32_t bar = smem_u32(qsm + kQRingBytes + kQWarps * kQOutBytes) + 8 * warp;
+    uint8_t *stg = qsm + warp * kQStageBytes;
+    uint8_t *wout = qsm + kQRingBytes + warp * kQOutBytes;
+    uint16_t *stage = reinterpret_cast<uint16_t *>(wout);                      // [32][kBlk/2]
+    int64_t *doffs = reinterpret_cast<int64_t *>(wout + kQRows * kBlockBytes);  // [32]
+    // the 32 rows of group gi into this warp's stage, one bulk copy per lane
+    // (tail lanes repeat the last row; nothing of theirs is stored)
+    auto load_group = [&](uint32_t gi) {
+        const uint32_t r = min(gi * kQRows + lane, rows - 1);
+        const uint32_t t = r % (uint32_t)n_new, bh = r / (uint32_t)n_new;
+        const uint32_t h = bh % (uint32_t)Hkv, b = bh / (uint32_t)Hkv;
+        const float *srow = src + (((int64_t)b * n_new + t) * Hkv + h) * kD;
+        if (lane == 0) mbar_expect_tx(bar, kQRows * 512);
+        __syncwarp();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        bulk_g2s(smem_u32(stg + lane * kQRowStride), srow, 512, bar);
+    };
+    if (lane == 0) {
+        mbar_init(bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    uint32_t gi = blockIdx.x + warp * gridDim.x;
+    if (gi < groups) load_group(gi);
+    for (uint32_t phase = 0; gi < groups; phase ^= 1u) {
+        const uint32_t gnext = gi + kQWarps * gridDim.x;
+        // this lane's row and its destination, while the rows load
         const uint32_t r = gi * kQRows + lane;
         const bool live = r < rows;
-        const uint32_t rr = live ? r : rows - 1;
-        const uint32_t t = rr % (uint32_t)n_new, bh = rr / (uint32_t)n_new;
-        const uint32_t h = bh % (uint32_t)Hkv, b = bh / (uint32_t)Hkv;
-        const float4 *srow =
-            reinterpret_cast<const float4 *>(src + (((int64_t)b * n_new + t) * Hkv + h) * kD);
         int64_t doff = -1;          // -1: nothing stored (tail lane or bad position)
         if (live) {
+            const uint32_t t = r % (uint32_t)n_new, bh = r / (uint32_t)n_new;
+            const uint32_t h = bh % (uint32_t)Hkv, b = bh / (uint32_t)Hkv;
             const int64_t pos = (int64_t)__ldg(start_pos + b) + t;
             if (pos < 0 || pos >= capacity) {
                 record_status(4u /* TBQ4_ERR_CAPACITY */);
@@ -121,23 +153,24 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
                 doff = (((int64_t)b * Hkv + h) * capacity + pos) * kBlk;
             }
         }
-        // load: row i, one 16-byte chunk per lane
-#pragma unroll 8
-        for (int i = 0; i < kQRows; ++i) {
-            const float4 *pi = reinterpret_cast<const float4 *>(
-                __shfl_sync(kFull, reinterpret_cast<uintptr_t>(srow), i));
-            tile[i * 32 + (lane ^ (i & 7))] = __ldcs(pi + lane);
+        if (!mbar_wait_bounded(bar, phase)) {
+            if (lane == 0) record_status(7u /* TBQ4_ERR_DEVICE_TIMEOUT */);
+            break;
+        }
+        float v[kD];
+        {
+            const float4 *row = reinterpret_cast<const float4 *>(stg + lane * kQRowStride);
+#pragma unroll
+            for (int c = 0; c < kD / 4; ++c) {
+                const float4 x = row[c];
+                v[4 * c] = x.x;
+                v[4 * c + 1] = x.y;
+                v[4 * c + 2] = x.z;
+                v[4 * c + 3] = x.w;
+            }
         }
         __syncwarp();
-        float v[kD];
-#pragma unroll
-        for (int c = 0; c < kD / 4; ++c) {
-            const float4 x = tile[lane * 32 + (c ^ (lane & 7))];
-            v[4 * c] = x.x;
-            v[4 * c + 1] = x.y;
-            v[4 * c + 2] = x.z;
-            v[4 * c + 3] = x.w;
-        }
+        if (gnext < groups) load_group(gnext);              // lands while this group encodes
         // stage 1 with the signs folded in
 #pragma unroll
         for (int j = 0; j < kD; j += 2) {
@@ -188,7 +221,7 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
             for (int w = 0; w < kD / 4; ++w) {                         // 4 nibbles per piece
                 uint32_t piece = 0;
 #pragma unroll
-                for (int k = 0; k < 4; ++k) piece |= index_of(v[4 * w + k]) << (4 * k);
+                for (int k4 = 0; k4 < 4; ++k4) piece |= index_of(v[4 * w + k4]) << (4 * k4);
                 mine[1 + w] = (uint16_t)piece;
             }
         } else {
@@ -196,7 +229,8 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
             for (int h2 = 0; h2 < kD / 16; ++h2) {                     // two 24-bit words
                 uint64_t wd = 0;                                       // = three pieces
 #pragma unroll
-                for (int k = 0; k < 16; ++k) wd |= (uint64_t)index_of(v[16 * h2 + k]) << (3 * k);
+                for (int k16 = 0; k16 < 16; ++k16)
+                    wd |= (uint64_t)index_of(v[16 * h2 + k16]) << (3 * k16);
                 mine[1 + 3 * h2] = (uint16_t)wd;
                 mine[2 + 3 * h2] = (uint16_t)(wd >> 16);
                 mine[3 + 3 * h2] = (uint16_t)(wd >> 32);
@@ -206,13 +240,14 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
         __syncwarp();
         // store: the 32 blocks as 32 x kBlk / 2 consecutive 16-bit pieces
 #pragma unroll
-        for (int k = 0; k < kBlk / 2; ++k) {
-            const int j = lane + 32 * k;
+        for (int k2 = 0; k2 < kBlk / 2; ++k2) {
+            const int j = lane + 32 * k2;
             const int row = j / (kBlk / 2), pc = j - row * (kBlk / 2);
             const int64_t off = doffs[row];
             if (off >= 0) *reinterpret_cast<uint16_t *>(cache + off + 2 * pc) = stage[j];
         }
         __syncwarp();
+        gi = gnext;
     }
 }
 

@@ -247,8 +247,10 @@ tbq4_status quantize_impl(const float *src, int B, int n_new, int Hkv, const int
     const void *fn = bits == 3 ? (const void *)quantize_rows_kernel<3>
                                : (const void *)quantize_rows_kernel<4>;
     if (!ensure_smem_attr(fn, kQSmemBytes, bits == 3 ? attr3 : attr4)) return TBQ4_ERR_LAUNCH;
-    int64_t blocks = ceil_div(rows, (int64_t)kQThreads);   // one row per thread
-    if (blocks > (int64_t)kNumSMs * 3) blocks = (int64_t)kNumSMs * 3;
+    // one CTA per SM (the ring takes most of shared memory), each over a
+    // strided share of the 32-row groups
+    int64_t blocks = ceil_div(rows, (int64_t)kQRows);
+    if (blocks > (int64_t)kNumSMs) blocks = (int64_t)kNumSMs;
     if (bits == 3)
         quantize_rows_kernel<3><<<(unsigned)blocks, kQThreads, kQSmemBytes, (cudaStream_t)stream>>>(
             src, B, n_new, Hkv, start_pos, capacity, sg, pm, cache);

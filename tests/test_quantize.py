@@ -100,3 +100,31 @@ def test_bytes_bit_exact_workloads(T, case):
         for b, x in enumerate(seqs):
             n = len(x)
             assert np.array_equal(got[b, :, :n], want[b, :, :n]), (case, b)
+
+
+def test_bulk_path_ragged_groups_and_positions(T):
+    # 3 x 2,731 x 3 = 24,579 rows: the bulk encoder (16,384 rows or more), a
+    # group count that the CTA count does not divide, a 3-row tail group, and
+    # a different start position per sequence
+    rng = np.random.default_rng(21)
+    B, n_new, Hkv, cap = 3, 2731, 3, 4096
+    src = (rng.standard_t(4, (B, n_new, Hkv, 128)) * 3).astype(np.float32)
+    src[1, 100] = 0.0                                 # zero rows inside the bulk path
+    start = [0, 1000, 1365]
+    got = _gpu_append(T, src, start, cap, 5)
+    want = _oracle_append(src, start, cap, 5)
+    assert np.array_equal(got, want)
+
+
+def test_bulk_path_out_of_range_rows_are_skipped_and_flagged(T):
+    import torch
+    rng = np.random.default_rng(22)
+    src = rng.standard_normal((1, 20000, 1, 128)).astype(np.float32)
+    cache = T.empty_cache(1, 1, 16384)
+    cache.fill_(0xAB)
+    T.tbq4_quantize_append(torch.from_numpy(src).cuda(),
+                           torch.tensor([100], dtype=torch.int32, device="cuda"), cache)
+    assert T.tbq4_get_device_status() == 4           # rows past the capacity
+    assert T.tbq4_get_device_status() == 0
+    want = _oracle_append(src, [100], 16384, 0)
+    assert np.array_equal(cache.cpu().numpy(), want)
