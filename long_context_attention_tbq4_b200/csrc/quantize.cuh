@@ -58,8 +58,9 @@ struct SignTable {
 //   index     clamp(rne(fl32(fl32(x/S) * 7.5) + 7.5), 0, 15), 8 when S == 0.
 //             The quotient is the correctly rounded x/S by Markstein's method:
 //             r = RN(1/S) once per row, q0 = RN(x r), e = x - q0 S (exact with
-//             FMA), q = RN(q0 + e r).  The conversion to unsigned saturates
-//             negative values to 0, which with min(., 15) is the clamp.
+//             FMA), q = RN(q0 + e r).  rint is an add of 1.5 * 2^23 on the
+//             FMA pipe; the clamp is needed only for rows whose fp16 scale is
+//             zero, subnormal or saturated, and is applied to x for those.
 // Memory: rows go in groups of 32 in head-major order (row = (b Hkv + h)
 // n_new + t), so a group's 32 blocks are contiguous in the cache.  One CTA
 // of eight warps per SM, two warps per scheduler (so a thread can keep its
@@ -202,19 +203,30 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
         const float S = half_bits_to_float(sb);
         uint16_t *mine = stage + lane * (kBlk / 2);
         mine[0] = sb;
-        const float rs = S == 0.0f ? 0.0f : __frcp_rn(S);
-        // x / S correctly rounded, then the codebook's index
+        // A normal, unsaturated fp16 scale is within 2^-11 of max|x|, so
+        // |x/S| <= 1 + 2^-11 and u = fl(fl(x/S) * 7.5) + 7.5 lies in
+        // [-0.004, 15.004]: rint(u) is already in [0, 15] (3-bit: [0, 7]) and
+        // needs no clamp.  A zero, subnormal or saturated scale: x is clamped
+        // to [-S, S] first, which gives the same index (the index is monotone
+        // in x, and -S, S give 0 and 15), and S = 0 divides by 1 instead, so
+        // every u is 7.5 (3.5): index 8 (4).
+        const uint32_t sabs = sb & 0x7FFFu;
+        if (sabs < 0x0400u || sabs == 0x7BFFu) {
+#pragma unroll
+            for (int j = 0; j < kD; ++j) v[j] = fminf(fmaxf(v[j], -S), S);
+        }
+        const float Sd = S == 0.0f ? 1.0f : S;
+        const float rs = __frcp_rn(Sd);
+        // x / S correctly rounded, then the codebook's index: rint by adding
+        // 1.5 * 2^23 (the sum's ulp is 1 for |u| < 2^22, and its low bits are
+        // rint(u), ties to even)
         auto index_of = [&](float x) -> uint32_t {
             const float q0 = __fmul_rn(x, rs);
-            const float e = __fmaf_rn(-q0, S, x);
+            const float e = __fmaf_rn(-q0, Sd, x);
             const float q = __fmaf_rn(e, rs, q0);
-            if constexpr (kBits == 4) {
-                const float u = __fadd_rn(__fmul_rn(q, 7.5f), 7.5f);
-                return S == 0.0f ? 8u : min(__float2uint_rn(u), 15u);
-            } else {
-                const float u = __fadd_rn(__fmul_rn(q, 3.5f), 3.5f);
-                return S == 0.0f ? 4u : min(__float2uint_rn(u), 7u);
-            }
+            constexpr float kL = kBits == 4 ? 7.5f : 3.5f;
+            const float u = __fadd_rn(__fmul_rn(q, kL), kL);
+            return __float_as_uint(__fadd_rn(u, 12582912.0f)) & (kBits == 4 ? 0xFu : 0x7u);
         };
         if constexpr (kBits == 4) {
 #pragma unroll

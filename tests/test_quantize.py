@@ -128,3 +128,28 @@ def test_bulk_path_out_of_range_rows_are_skipped_and_flagged(T):
     assert T.tbq4_get_device_status() == 0
     want = _oracle_append(src, [100], 16384, 0)
     assert np.array_equal(cache.cpu().numpy(), want)
+
+
+def test_bulk_path_extreme_scales(T):
+    """20,480 rows through the bulk encoder, every 32-row group mixing rows
+    whose fp16 scale is zero (max |x_rot| below 2^-25), subnormal, near the
+    smallest normal, ordinary, or saturated at 65,504 (the rows that take the
+    clamp), for both the 4-bit and the 3-bit encoder."""
+    import torch
+    rng = np.random.default_rng(23)
+    B, n_new, Hkv, cap = 2, 2560, 4, 2560
+    src = rng.standard_normal((B, n_new, Hkv, 128)).astype(np.float32)
+    gains = np.array([1.0, 1e-6, 1e-9, 3e-5, 1.0, 7e4, 1e-7, 250.0], np.float32)
+    src *= gains[np.arange(n_new) % 8][None, :, None, None]
+    src[:, 4::8, :, 5] = 1e9                          # one huge value: a saturated scale
+    zero = np.zeros(B, np.int32)
+    got = _gpu_append(T, src, zero, cap, 3)
+    want = _oracle_append(src, zero, cap, 3)
+    assert np.array_equal(got, want)
+    got3 = T.empty_cache3(B, Hkv, cap)
+    got3.fill_(0xAB)
+    T.tbq3_quantize_append(torch.from_numpy(src).cuda(), torch.from_numpy(zero).cuda(), got3, 3)
+    assert T.tbq4_get_device_status() == 0
+    want3 = np.full((B, Hkv, cap, 50), 0xAB, np.uint8)
+    oracle.quantize_append3(src, zero, cap, 3, want3)
+    assert np.array_equal(got3.cpu().numpy(), want3)
