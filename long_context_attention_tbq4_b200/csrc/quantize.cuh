@@ -5,8 +5,9 @@
 //   encode_row            one warp per row (four values per lane, the
 //                         transform over shuffles); the decode kernel uses it
 //                         to append the current token
-//   quantize_rows_kernel  one thread per row, the transform in registers;
-//                         the bulk append (HBM-bound: 512 bytes in, 66 out)
+//   quantize_rows_kernel  four threads per row, the transform in registers
+//                         and two shuffle stages; the bulk append (512
+//                         bytes in, 66 out per row)
 #pragma once
 #include "common.cuh"
 #include "mbarrier.cuh"
@@ -41,19 +42,15 @@ __device__ __forceinline__ uint32_t encode_row(float v[4], uint32_t sbits, int l
     return i0 | (i1 << 4) | (i2 << 8) | (i3 << 12);
 }
 
-// The +-1 sign diagonal as floats, passed by value: a kernel parameter is a
-// constant-bank operand, so the signs fold into the first butterfly stage.
-struct SignTable {
-    float s[kD];
-};
-
-// Bulk append: one thread encodes one whole 128-value row (rows are
-// independent, so a thread per row keeps the transform in registers, with no
-// shuffles):
+// Bulk append: four threads per 128-value row, each holding a quarter of it
+// (32 consecutive values) in registers.
 //   rotation  the same butterflies in the same order as warp_fwht128 (stride
 //             1 first; lower = a + b, upper = a - b, each rounded on its own).
-//             The sign flip is exact, so the first stage is
-//             fma(v_j, s_j, s_k v_k) and fma(v_j, s_j, -s_k v_k).
+//             Strides 1 .. 16 stay inside a quarter; strides 32 and 64 pair
+//             quarters q and q ^ 1, q and q ^ 2 (lanes 8 and 16 apart), the
+//             upper one computing fma(own, -1, partner) = partner - own.  The
+//             sign flip is exact, so the first stage is fma(v_j, s_j, s_k v_k)
+//             and fma(v_j, s_j, -s_k v_k).
 //   scale     S = fp16(max |x_rot|), saturated at 65504.
 //   index     clamp(rne(fl32(fl32(x/S) * 7.5) + 7.5), 0, 15), 8 when S == 0.
 //             The quotient is the correctly rounded x/S by Markstein's method:
@@ -61,16 +58,15 @@ struct SignTable {
 //             FMA), q = RN(q0 + e r).  rint is an add of 1.5 * 2^23 on the
 //             FMA pipe; the clamp is needed only for rows whose fp16 scale is
 //             zero, subnormal or saturated, and is applied to x for those.
-// Memory: rows go in groups of 32 in head-major order (row = (b Hkv + h)
-// n_new + t), so a group's 32 blocks are contiguous in the cache.  One CTA
-// of eight warps per SM, two warps per scheduler (so a thread can keep its
-// row's 128 values in registers: a scheduler's register file is a quarter
-// of the SM's).  Each warp owns one shared-memory stage: a group comes in as
-// one 512-byte cp.async.bulk per row (rows 528 bytes apart, so the
-// per-thread reads of a whole row are free of bank conflicts); once the
-// rows are in registers the warp sends its next group's copies into the
-// same stage, and they land while this group is encoded.  The blocks go out
-// from a per-warp staging area as consecutive 16-bit pieces.
+// Memory: rows go in groups of 8 in head-major order (row = (b Hkv + h)
+// n_new + t), so a group's 8 blocks are contiguous in the cache.  Lane l
+// takes row l % 8 of its warp's group and quarter l / 8 of that row.  One
+// CTA of 16 warps per SM; each warp streams its groups through a ring of
+// kQDepth shared-memory stages, one 512-byte cp.async.bulk per row (rows 528
+// bytes apart, so the eight lanes of a 16-byte read phase hit eight
+// different bank groups), and sends the copies of a later group into a stage
+// as soon as the rows are in registers.  The blocks go out from a per-warp
+// staging area as consecutive 16-bit pieces.
 // Paged destination: row (b, pos) goes to page table[b][pos / page_size],
 // row pos % page_size, of a pool [n_pages][Hkv][page_size][66].  A null
 // table means the contiguous cache [B][Hkv][capacity][66].
@@ -86,83 +82,103 @@ struct PageMap {
 // at bits 3k .. 3k+2): 2 + 48 = 50 bytes per block.
 constexpr int kBlockBytes3 = 50;
 
-constexpr int kQRows = 32;                                   // rows per group
-constexpr int kQWarps = 8;                                   // warps per CTA
+constexpr int kQRows = 8;                                    // rows per group
+constexpr int kQWarps = 16;                                  // warps per CTA
+constexpr int kQDepth = 2;                                   // stages per warp
 constexpr int kQRowStride = 512 + 16;                        // bytes between staged rows
 constexpr int kQStageBytes = kQRows * kQRowStride;
-constexpr int kQOutBytes = kQRows * kBlockBytes + kQRows * 8;   // blocks + destinations
+constexpr int kQOutBytes = kQRows * kBlockBytes + 16 + kQRows * 8;   // blocks, pad, destinations
 constexpr int kQThreads = kQWarps * 32;
-constexpr int kQRingBytes = kQWarps * kQStageBytes;
-constexpr int kQSmemBytes = kQRingBytes + kQWarps * kQOutBytes + kQWarps * 8;
+constexpr int kQRingBytes = kQWarps * kQDepth * kQStageBytes;
+constexpr int kQSmemBytes = kQRingBytes + kQWarps * kQOutBytes + kD * 4 + kQWarps * kQDepth * 8;
 static_assert(kQSmemBytes <= 227 * 1024, "shared memory per CTA");
 static_assert(kQStageBytes % 16 == 0 && kQRowStride % 16 == 0 && kQOutBytes % 16 == 0,
               "bulk copies and staged rows stay 16-byte aligned");
 
 // kBits: 4 (TBQ4, 66-byte blocks) or 3 (TBQ3, 50-byte blocks).  Group k of a
-// CTA is group blockIdx.x + k gridDim.x, encoded by warp k % kQWarps.
+// CTA is group blockIdx.x + k gridDim.x, taken by warp k % kQWarps.
 template <int kBits>
 __global__ void __launch_bounds__(kQThreads, 1)
 quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
-                     const int32_t *__restrict__ start_pos, int64_t capacity, const SignTable sg,
-                     const PageMap pm, uint8_t *__restrict__ cache) {
+                     const int32_t *__restrict__ start_pos, int64_t capacity, uint64_t sign_lo,
+                     uint64_t sign_hi, const PageMap pm, uint8_t *__restrict__ cache) {
     extern __shared__ __align__(128) uint8_t qsm[];
     constexpr int kBlk = kBits == 4 ? kBlockBytes : kBlockBytes3;
+    constexpr int kPieces = kBlk / 2;                         // 16-bit pieces per block
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int rho = lane & 7, qq = lane >> 3;                 // row of the group, quarter
     const uint32_t rows = (uint32_t)B * (uint32_t)n_new * (uint32_t)Hkv;    // < 2^31 (host)
     const uint32_t groups = (rows + kQRows - 1) / kQRows;
-    const uint32_t bar = smem_u32(qsm + kQRingBytes + kQWarps * kQOutBytes) + 8 * warp;
-    uint8_t *stg = qsm + warp * kQStageBytes;
+    uint8_t *ring = qsm + warp * kQDepth * kQStageBytes;
     uint8_t *wout = qsm + kQRingBytes + warp * kQOutBytes;
-    uint16_t *stage = reinterpret_cast<uint16_t *>(wout);                      // [32][kBlk/2]
-    int64_t *doffs = reinterpret_cast<int64_t *>(wout + kQRows * kBlockBytes);  // [32]
-    // the 32 rows of group gi into this warp's stage, one bulk copy per lane
-    // (tail lanes repeat the last row; nothing of theirs is stored)
-    auto load_group = [&](uint32_t gi) {
-        const uint32_t r = min(gi * kQRows + lane, rows - 1);
-        const uint32_t t = r % (uint32_t)n_new, bh = r / (uint32_t)n_new;
-        const uint32_t h = bh % (uint32_t)Hkv, b = bh / (uint32_t)Hkv;
-        const float *srow = src + (((int64_t)b * n_new + t) * Hkv + h) * kD;
-        if (lane == 0) mbar_expect_tx(bar, kQRows * 512);
-        __syncwarp();
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        bulk_g2s(smem_u32(stg + lane * kQRowStride), srow, 512, bar);
-    };
+    uint16_t *stage = reinterpret_cast<uint16_t *>(wout);                     // [8][kPieces]
+    int64_t *doffs = reinterpret_cast<int64_t *>(wout + kQRows * kBlockBytes + 16);   // [8]
+    float *sgn = reinterpret_cast<float *>(qsm + kQRingBytes + kQWarps * kQOutBytes);  // [128]
+    const uint32_t bar0 = smem_u32(sgn + kD) + warp * kQDepth * 8;
+    if (threadIdx.x < kD) {
+        const int i = threadIdx.x;
+        const uint64_t w = i < 64 ? sign_lo : sign_hi;
+        sgn[i] = ((w >> (i & 63)) & 1u) ? -1.0f : 1.0f;
+    }
     if (lane == 0) {
-        mbar_init(bar, 1);
+        for (int d = 0; d < kQDepth; ++d) mbar_init(bar0 + 8 * d, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    __syncwarp();
-    uint32_t gi = blockIdx.x + warp * gridDim.x;
-    if (gi < groups) load_group(gi);
-    for (uint32_t phase = 0; gi < groups; phase ^= 1u) {
-        const uint32_t gnext = gi + kQWarps * gridDim.x;
-        // this lane's row and its destination, while the rows load
-        const uint32_t r = gi * kQRows + lane;
-        const bool live = r < rows;
-        int64_t doff = -1;          // -1: nothing stored (tail lane or bad position)
-        if (live) {
+    __syncthreads();
+    // the 8 rows of group gi into stage d, one bulk copy per lane 0..7 (rows
+    // past the end repeat the last row; nothing of theirs is stored)
+    auto load_group = [&](uint32_t gi, int d) {
+        if (lane == 0) mbar_expect_tx(bar0 + 8 * d, kQRows * 512);
+        __syncwarp();
+        if (lane < kQRows) {
+            const uint32_t r = min(gi * kQRows + lane, rows - 1);
             const uint32_t t = r % (uint32_t)n_new, bh = r / (uint32_t)n_new;
             const uint32_t h = bh % (uint32_t)Hkv, b = bh / (uint32_t)Hkv;
-            const int64_t pos = (int64_t)__ldg(start_pos + b) + t;
-            if (pos < 0 || pos >= capacity) {
-                record_status(4u /* TBQ4_ERR_CAPACITY */);
-            } else if (pm.table) {
-                const int32_t pid = __ldg(pm.table + (int64_t)b * pm.max_pages + pos / pm.page_size);
-                if (pid < 0 || (int64_t)pid >= pm.n_pages) record_status(4u);
-                else doff = (((int64_t)pid * Hkv + h) * pm.page_size + pos % pm.page_size) * kBlk;
-            } else {
-                doff = (((int64_t)b * Hkv + h) * capacity + pos) * kBlk;
-            }
+            const float *srow = src + (((int64_t)b * n_new + t) * Hkv + h) * kD;
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            bulk_g2s(smem_u32(ring + d * kQStageBytes + lane * kQRowStride), srow, 512,
+                     bar0 + 8 * d);
         }
-        if (!mbar_wait_bounded(bar, phase)) {
+    };
+    const uint32_t gstride = kQWarps * gridDim.x;
+    uint32_t gi = blockIdx.x + warp * gridDim.x;
+#pragma unroll
+    for (int d = 0; d < kQDepth; ++d)
+        if (gi + d * gstride < groups) load_group(gi + d * gstride, d);
+    const float neg = (qq & 1) ? -1.0f : 1.0f, neg2 = (qq & 2) ? -1.0f : 1.0f;
+    for (uint32_t it = 0; gi < groups; ++it, gi += gstride) {
+        const int d = (int)(it % kQDepth);
+        // this row's destination, while the rows load (one lane per row)
+        if (qq == 0) {
+            const uint32_t r = gi * kQRows + rho;
+            int64_t doff = -1;      // -1: nothing stored (past the end or a bad position)
+            if (r < rows) {
+                const uint32_t t = r % (uint32_t)n_new, bh = r / (uint32_t)n_new;
+                const uint32_t h = bh % (uint32_t)Hkv, b = bh / (uint32_t)Hkv;
+                const int64_t pos = (int64_t)__ldg(start_pos + b) + t;
+                if (pos < 0 || pos >= capacity) {
+                    record_status(4u /* TBQ4_ERR_CAPACITY */);
+                } else if (pm.table) {
+                    const int32_t pid =
+                        __ldg(pm.table + (int64_t)b * pm.max_pages + pos / pm.page_size);
+                    if (pid < 0 || (int64_t)pid >= pm.n_pages) record_status(4u);
+                    else doff = (((int64_t)pid * Hkv + h) * pm.page_size + pos % pm.page_size) * kBlk;
+                } else {
+                    doff = (((int64_t)b * Hkv + h) * capacity + pos) * kBlk;
+                }
+            }
+            doffs[rho] = doff;
+        }
+        if (!mbar_wait_bounded(bar0 + 8 * d, (it / kQDepth) & 1u)) {
             if (lane == 0) record_status(7u /* TBQ4_ERR_DEVICE_TIMEOUT */);
             break;
         }
-        float v[kD];
+        float v[32];
         {
-            const float4 *row = reinterpret_cast<const float4 *>(stg + lane * kQRowStride);
+            const float4 *row = reinterpret_cast<const float4 *>(ring + d * kQStageBytes +
+                                                                 rho * kQRowStride + qq * 128);
 #pragma unroll
-            for (int c = 0; c < kD / 4; ++c) {
+            for (int c = 0; c < 8; ++c) {
                 const float4 x = row[c];
                 v[4 * c] = x.x;
                 v[4 * c + 1] = x.y;
@@ -171,38 +187,60 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
             }
         }
         __syncwarp();
-        if (gnext < groups) load_group(gnext);              // lands while this group encodes
-        // stage 1 with the signs folded in
+        if (gi + kQDepth * gstride < groups) load_group(gi + kQDepth * gstride, d);
+        // stride 1 with the signs folded in
+        {
+            const float4 *s4 = reinterpret_cast<const float4 *>(sgn + 32 * qq);
 #pragma unroll
-        for (int j = 0; j < kD; j += 2) {
-            const float bb = __fmul_rn(v[j + 1], sg.s[j + 1]);
-            const float lo = __fmaf_rn(v[j], sg.s[j], bb);
-            const float hi = __fmaf_rn(v[j], sg.s[j], -bb);
-            v[j] = lo;
-            v[j + 1] = hi;
+            for (int c = 0; c < 8; ++c) {
+                const float4 sv = s4[c];
+                const float sj[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+                for (int e = 0; e < 4; e += 2) {
+                    const int j = 4 * c + e;
+                    const float bb = __fmul_rn(v[j + 1], sj[e + 1]);
+                    const float lo = __fmaf_rn(v[j], sj[e], bb);
+                    const float hi = __fmaf_rn(v[j], sj[e], -bb);
+                    v[j] = lo;
+                    v[j + 1] = hi;
+                }
+            }
         }
+        // strides 2 .. 16 inside the quarter
 #pragma unroll
-        for (int hs = 2; hs < kD; hs <<= 1) {
+        for (int hs = 2; hs < 32; hs <<= 1) {
 #pragma unroll
-            for (int j = 0; j < kD; ++j) {
+            for (int j = 0; j < 32; ++j) {
                 if (j & hs) continue;
                 const float a = v[j], c = v[j + hs];
                 v[j] = __fadd_rn(a, c);
                 v[j + hs] = __fsub_rn(a, c);
             }
         }
+        // strides 32 and 64 across quarters: the lower quarter adds the
+        // partner's value, the upper one subtracts its own from it
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const float p = __shfl_xor_sync(kFull, v[j], 8);
+            v[j] = __fmaf_rn(v[j], neg, p);
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const float p = __shfl_xor_sync(kFull, v[j], 16);
+            v[j] = __fmaf_rn(v[j], neg2, p);
+        }
         const float cr = rot_c();
         float m = 0.f;
 #pragma unroll
-        for (int j = 0; j < kD; ++j) {
+        for (int j = 0; j < 32; ++j) {
             v[j] = __fmul_rn(v[j], cr);
             m = fmaxf(m, fabsf(v[j]));
         }
+        m = fmaxf(m, __shfl_xor_sync(kFull, m, 8));
+        m = fmaxf(m, __shfl_xor_sync(kFull, m, 16));
         uint16_t sb = __half_as_ushort(__float2half_rn(m));
         if ((sb & 0x7FFFu) == 0x7C00u) sb = 0x7BFFu;                 // saturate at 65504
         const float S = half_bits_to_float(sb);
-        uint16_t *mine = stage + lane * (kBlk / 2);
-        mine[0] = sb;
         // A normal, unsaturated fp16 scale is within 2^-11 of max|x|, so
         // |x/S| <= 1 + 2^-11 and u = fl(fl(x/S) * 7.5) + 7.5 lies in
         // [-0.004, 15.004]: rint(u) is already in [0, 15] (3-bit: [0, 7]) and
@@ -213,7 +251,7 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
         const uint32_t sabs = sb & 0x7FFFu;
         if (sabs < 0x0400u || sabs == 0x7BFFu) {
 #pragma unroll
-            for (int j = 0; j < kD; ++j) v[j] = fminf(fmaxf(v[j], -S), S);
+            for (int j = 0; j < 32; ++j) v[j] = fminf(fmaxf(v[j], -S), S);
         }
         const float Sd = S == 0.0f ? 1.0f : S;
         const float rs = __frcp_rn(Sd);
@@ -228,45 +266,51 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
             const float u = __fadd_rn(__fmul_rn(q, kL), kL);
             return __float_as_uint(__fadd_rn(u, 12582912.0f)) & (kBits == 4 ? 0xFu : 0x7u);
         };
+        uint16_t *mine = stage + rho * kPieces;
+        if (qq == 0) mine[0] = sb;
         if constexpr (kBits == 4) {
+            // values 32 qq .. 32 qq + 31: nibble bytes 16 qq .. 16 qq + 15,
+            // pieces 1 + 8 qq .. 8 + 8 qq
 #pragma unroll
-            for (int w = 0; w < kD / 4; ++w) {                         // 4 nibbles per piece
+            for (int w = 0; w < 8; ++w) {
                 uint32_t piece = 0;
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) piece |= index_of(v[4 * w + k4]) << (4 * k4);
-                mine[1 + w] = (uint16_t)piece;
+                mine[1 + 8 * qq + w] = (uint16_t)piece;
             }
         } else {
+            // values 32 qq .. 32 qq + 31: four 24-bit words, bytes 12 qq ..
+            // 12 qq + 11, pieces 1 + 6 qq .. 6 + 6 qq
 #pragma unroll
-            for (int h2 = 0; h2 < kD / 16; ++h2) {                     // two 24-bit words
-                uint64_t wd = 0;                                       // = three pieces
+            for (int h2 = 0; h2 < 2; ++h2) {                           // two words = three pieces
+                uint64_t wd = 0;
 #pragma unroll
                 for (int k16 = 0; k16 < 16; ++k16)
                     wd |= (uint64_t)index_of(v[16 * h2 + k16]) << (3 * k16);
-                mine[1 + 3 * h2] = (uint16_t)wd;
-                mine[2 + 3 * h2] = (uint16_t)(wd >> 16);
-                mine[3 + 3 * h2] = (uint16_t)(wd >> 32);
+                mine[1 + 6 * qq + 3 * h2] = (uint16_t)wd;
+                mine[2 + 6 * qq + 3 * h2] = (uint16_t)(wd >> 16);
+                mine[3 + 6 * qq + 3 * h2] = (uint16_t)(wd >> 32);
             }
         }
-        doffs[lane] = doff;
         __syncwarp();
-        // store: the 32 blocks as 32 x kBlk / 2 consecutive 16-bit pieces
+        // store: the 8 blocks as 8 x kPieces consecutive 16-bit pieces
 #pragma unroll
-        for (int k2 = 0; k2 < kBlk / 2; ++k2) {
+        for (int k2 = 0; k2 < (kQRows * kPieces + 31) / 32; ++k2) {
             const int j = lane + 32 * k2;
-            const int row = j / (kBlk / 2), pc = j - row * (kBlk / 2);
-            const int64_t off = doffs[row];
-            if (off >= 0) *reinterpret_cast<uint16_t *>(cache + off + 2 * pc) = stage[j];
+            if (j < kQRows * kPieces) {
+                const int row = j / kPieces, pc = j - row * kPieces;
+                const int64_t off = doffs[row];
+                if (off >= 0) *reinterpret_cast<uint16_t *>(cache + off + 2 * pc) = stage[j];
+            }
         }
         __syncwarp();
-        gi = gnext;
     }
 }
 
 
 // Few rows (a prefill chunk, a decode step): one warp per row with the warp
 // encoder, so that even a few thousand rows spread over every SM instead of
-// the handful of blocks the thread-per-row kernel would fill.  The same
+// a few hundred 8-row groups of the bulk kernel.  The same
 // bytes as quantize_rows_kernel<4> (the same encoding steps in the same
 // order); rows are taken in source order (b, t, h), so the loads of
 // consecutive warps are contiguous.

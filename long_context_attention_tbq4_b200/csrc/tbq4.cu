@@ -213,8 +213,8 @@ void tbq4_signs(uint64_t seed, int8_t out[128]) {
 
 namespace {
 
-// Below this many rows the thread-per-row encoder fills too few blocks
-// (rows / 128) to keep the GPU busy; the warp-per-row encoder takes over.
+// Below this many rows the bulk encoder has too few 8-row groups to keep
+// the GPU busy; the warp-per-row encoder takes over.
 constexpr int64_t kSmallAppendRows = 16384;
 
 tbq4_status quantize_impl(const float *src, int B, int n_new, int Hkv, const int32_t *start_pos,
@@ -239,24 +239,21 @@ tbq4_status quantize_impl(const float *src, int B, int n_new, int Hkv, const int
                                                             capacity, lo, hi, pm, cache);
         return launch_status();
     }
-    int8_t sg8[kD];
-    tbq4_signs(sign_seed, sg8);
-    SignTable sg;
-    for (int i = 0; i < kD; ++i) sg.s[i] = (float)sg8[i];
+    uint64_t lo, hi;
+    sign_words(sign_seed, &lo, &hi);
     static bool attr4[64] = {}, attr3[64] = {};    // set once per device
     const void *fn = bits == 3 ? (const void *)quantize_rows_kernel<3>
                                : (const void *)quantize_rows_kernel<4>;
     if (!ensure_smem_attr(fn, kQSmemBytes, bits == 3 ? attr3 : attr4)) return TBQ4_ERR_LAUNCH;
-    // one CTA per SM (the ring takes most of shared memory), each over a
-    // strided share of the 32-row groups
+    // one CTA per SM, each over a strided share of the 8-row groups
     int64_t blocks = ceil_div(rows, (int64_t)kQRows);
     if (blocks > (int64_t)kNumSMs) blocks = (int64_t)kNumSMs;
     if (bits == 3)
         quantize_rows_kernel<3><<<(unsigned)blocks, kQThreads, kQSmemBytes, (cudaStream_t)stream>>>(
-            src, B, n_new, Hkv, start_pos, capacity, sg, pm, cache);
+            src, B, n_new, Hkv, start_pos, capacity, lo, hi, pm, cache);
     else
         quantize_rows_kernel<4><<<(unsigned)blocks, kQThreads, kQSmemBytes, (cudaStream_t)stream>>>(
-            src, B, n_new, Hkv, start_pos, capacity, sg, pm, cache);
+            src, B, n_new, Hkv, start_pos, capacity, lo, hi, pm, cache);
     return launch_status();
 }
 

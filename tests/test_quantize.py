@@ -131,7 +131,7 @@ def test_bulk_path_out_of_range_rows_are_skipped_and_flagged(T):
 
 
 def test_bulk_path_extreme_scales(T):
-    """20,480 rows through the bulk encoder, every 32-row group mixing rows
+    """20,480 rows through the bulk encoder, every 8-row group mixing rows
     whose fp16 scale is zero (max |x_rot| below 2^-25), subnormal, near the
     smallest normal, ordinary, or saturated at 65,504 (the rows that take the
     clamp), for both the 4-bit and the 3-bit encoder."""
