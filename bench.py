@@ -481,7 +481,22 @@ def cpu_baseline(case, N, step_bytes, sample_rows=24, reps=5):
 
 
 # ------------------------------------------------------------- distributed
-_dist = None
+_dist = None             # torch.distributed once a process group is up (N > 1)
+_dist_device = "cuda"    # where the max-over-ranks reduction runs: "cuda" (nccl), "cpu" (gloo)
+
+
+def init_distributed(torch, backend, local):
+    """One process group for the N independent replicas: nccl on the GPUs,
+    gloo for the CPU tests of the same host logic.  The timeout is short so
+    that a rank that never arrives ends the others' next collective with an
+    error."""
+    global _dist, _dist_device
+    import datetime
+    import torch.distributed as dist
+    kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    _dist = dist
+    _dist_device = "cuda" if backend == "nccl" else "cpu"
 
 
 def barrier():
@@ -492,9 +507,24 @@ def barrier():
 def max_over_ranks(torch, x):
     if _dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_dist_device)
     _dist.all_reduce(t, op=_dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_totals(torch, dec, steps, world, step_bytes):
+    """Whole-job figures of `world` independent replicas, each rank having
+    timed `steps` decode steps (dec: per-step device times in ms).  Every time
+    is the max over ranks; the value counts the bytes of all ranks.  Every
+    rank makes the same three reductions in the same order."""
+    total_ms = max_over_ranks(torch, float(np.sum(dec["step_ms"])))
+    ms_per_step = total_ms / steps
+    e2e_ms = max_over_ranks(torch, float(np.mean(dec["e2e_ms"])))
+    eager_ms = max_over_ranks(torch, float(np.mean(dec["eager_ms"])))
+    return {"ms_per_step": ms_per_step,
+            "value": world * step_bytes / (ms_per_step * 1e-3) / 1e9,
+            "e2e_ms": e2e_ms, "e2e_value": world * step_bytes / (e2e_ms * 1e-3) / 1e9,
+            "eager_ms": eager_ms}
 
 
 # -------------------------------------------------------------------- main
@@ -533,7 +563,6 @@ def run_reference(args):
 
 
 def main():
-    global _dist
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
@@ -544,11 +573,7 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-        _dist = dist
+        init_distributed(torch, "nccl", local)
     import long_context_attention_tbq4_b200 as T
 
     peaks = measured_peaks()
@@ -568,10 +593,8 @@ def main():
                                                          min(args.warmup, 3), flush)
     clocks = clk.summary()
 
-    total_ms = max_over_ranks(torch, float(np.sum(dec["step_ms"])))
-    ms_per_step = total_ms / args.steps
-    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
-    e2e_ms = max_over_ranks(torch, float(np.mean(dec["e2e_ms"])))
+    tot = replica_totals(torch, dec, args.steps, world, step_bytes)
+    ms_per_step, value, e2e_ms = tot["ms_per_step"], tot["value"], tot["e2e_ms"]
     kern_ms = float(np.mean(dec["kern_ms"]))
     achieved = kernel_bytes / (kern_ms * 1e-3) / 1e9
     traffic = recorded_traffic("decode_tc_kernel")
@@ -588,7 +611,7 @@ def main():
                              "(decode kernel + combine); e2e launches eagerly",
                    "parallelism": "replicas" if world > 1 else "single"},
         "step_bytes": step_bytes,
-        "ms_per_step_eager": max_over_ranks(torch, float(np.mean(dec["eager_ms"]))),
+        "ms_per_step_eager": tot["eager_ms"],
         "pct_hbm_peak": value / world / peaks["hbm_gbs"],
         # the split kernel and its combine (a programmatic dependent launch,
         # no gap between them) are timed as one region
@@ -598,7 +621,7 @@ def main():
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                      "algorithmic_bytes": kernel_bytes, "kernel_ms": kern_ms,
                      "peak_source": peaks["source"]},
-        "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        "e2e": {"value": tot["e2e_value"], "unit": "GB/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": dec["h2d"],
                 "d2h_bytes_per_step": dec["d2h"]},
         "gpu_launches": dec["launches_per_step"] * args.steps,
