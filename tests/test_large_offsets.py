@@ -111,3 +111,33 @@ def test_page_pool_past_4gb(T):
     check_decode(got.float().cpu().numpy(), want)
     del kp, vp
     torch.cuda.empty_cache()
+
+
+def test_prefill_past_4gb(T):
+    """Chunked prefill over one sequence whose last KV head starts past 2^32
+    (two caches of [4][21,692,416][66], 5.7 GB each): the chunk's append and
+    the attention's tile copies use 64-bit offsets."""
+    import torch
+    from helpers import PREFILL_REL_L2, capacity_for, gpu_caches, rel_l2
+    n_cached, n_new, Hq, Hkv, cap = 1000, 130, 24, 4, 21_692_416
+    assert (Hkv - 1) * cap * 66 > GB4
+    case = W.prefill_case("prefill_past_4gb", 96, n_cached, n_new, Hq, Hkv)
+    kc = gpu_caches([case.k[:n_cached]], Hkv, cap, case.sign_seed)[0]
+    vc = gpu_caches([case.v[:n_cached]], Hkv, cap, case.sign_seed)[0]
+    start = torch.tensor([n_cached], dtype=torch.int32, device="cuda")
+    for cache, x in ((kc, case.k), (vc, case.v)):
+        chunk = torch.from_numpy(np.ascontiguousarray(x[n_cached:])[None]).cuda()
+        T.tbq4_quantize_append(chunk, start, cache[None], sign_seed=case.sign_seed)
+    q = torch.from_numpy(case.q_bf16.view(np.int16)).cuda().view(torch.bfloat16)
+    got = T.tbq4_attn_prefill_chunk(q, n_cached, kc, vc, case.softmax_scale, case.sign_seed)
+    assert T.tbq4_get_device_status() == 0
+    small = capacity_for(n_cached + n_new)
+    ko = oracle_caches([case.k], Hkv, small, case.sign_seed)[0]
+    vo = oracle_caches([case.v], Hkv, small, case.sign_seed)[0]
+    n = n_cached + n_new
+    assert np.array_equal(kc[:, :n].cpu().numpy(), ko[:, :n])
+    assert np.array_equal(vc[:, :n].cpu().numpy(), vo[:, :n])
+    want = oracle.attn_prefill(case.q, n_cached, ko, vo, case.softmax_scale, case.sign_seed)
+    assert rel_l2(got.float().cpu().numpy(), want) <= PREFILL_REL_L2
+    del kc, vc
+    torch.cuda.empty_cache()
