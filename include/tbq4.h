@@ -320,9 +320,12 @@ TBQ4_API tbq4_status tbq4_attn_prefill_chunk(const uint16_t *q, int n_new,
                                     void *stream);
 
 /* Profiling hook: while set, every attention call records `before` on its
- * stream just before its main (split) kernel and `after` just after it, so
- * a caller can time that kernel alone with cudaEventElapsedTime.  Both are
- * cudaEvent_t created by the caller; pass NULLs to stop recording.  Not
+ * stream just before its attention kernel and `after` just after it, so a
+ * caller can time the attention alone with cudaEventElapsedTime.  Decode:
+ * the events bracket the split kernel and its combine (a programmatic
+ * dependent launch that starts while the split kernel drains, so the pair is
+ * one region); prefill: the attention kernel alone, not its combine.  Both
+ * are cudaEvent_t created by the caller; pass NULLs to stop recording.  Not
  * thread-safe: meant for benchmarks. */
 TBQ4_API void tbq4_set_timing_events(void *before, void *after);
 
