@@ -10,7 +10,10 @@ Written straight from the definitions, with no numpy and no shared code with
 * nearest_level_index3, unpack3, dequant3: the same for the 3-bit variant
   (8 levels S*(2i-7)/7; a 50-byte block read as a little-endian bit stream);
 * attention: softmax(scale * q_rot . k) v with math.fsum, in the rotated
-  domain, then rotated back with the explicit Hadamard entries.
+  domain, then rotated back with the explicit Hadamard entries;
+* rotate_f32_stages: the binary32 rotation as whole-vector numpy stages (the
+  one function here that uses numpy), which pins the butterfly order of the
+  C oracle bit for bit.
 """
 import math
 from fractions import Fraction
@@ -115,3 +118,24 @@ def attend(q, k_blocks, v_blocks, scale, s, deq=dequant) -> list:
     o_rot = [math.fsum(p[t] * vs[t][i] for t in range(len(vs))) / l
              for i in range(len(q_rot))]
     return unrotate(o_rot, s)
+
+
+def rotate_f32_stages(x, s):
+    """The binary32 rotation of the codebook, stage by stage on whole numpy
+    float32 vectors: z = s * x; for stride h = 1, 2, 4, ..., 64 split z into
+    blocks of 2h, the first half a and the second half b of each block
+    becoming a + b and a - b (numpy rounds each add and subtract to binary32
+    and never contracts them); finally one binary32 multiply by
+    fl32(1/sqrt(128)) = 0x3DB504F3.  Any other stride order or association
+    rounds differently on general inputs, so equality with the C oracle on
+    random vectors fixes its order."""
+    import numpy as np
+    z = np.asarray(x, np.float32) * np.asarray(s, np.float32)
+    n = z.shape[-1]
+    h = 1
+    while h < n:
+        blk = z.reshape(n // (2 * h), 2, h)
+        a, b = blk[:, 0, :], blk[:, 1, :]
+        z = np.stack([a + b, a - b], axis=1).reshape(n)
+        h *= 2
+    return z * np.array(0x3DB504F3, np.uint32).view(np.float32)

@@ -67,16 +67,22 @@ def half_ulp_fp16(x):
 
 
 def check_decode(got, want):
-    """max-abs <= 2e-3 beyond the fp16 output rounding, rel-L2 <= 1e-3.
+    """Per element |gpu - oracle| <= max(2e-3, half an fp16 ulp of the oracle
+    value), and rel-L2 <= 1e-3 over the whole tensor.
 
-    The decode output is fp16, so even an exact kernel is off by up to half
-    an fp16 ulp of the true value (1.95e-3 at |o| in [4, 8)); the absolute
-    bound is applied on top of that allowance."""
+    The decode output is fp16.  Below |o| = 8 half an fp16 ulp is at most
+    2^-10 < 2e-3, so there the bound is the plain 2e-3; only where fp16
+    itself cannot come within 2e-3 of the true value (|o| >= 8, half an ulp
+    >= 3.9e-3) is the bound half an ulp, what correct rounding of the exact
+    value allows.  Returns (raw max-abs, rel-L2)."""
     got = np.asarray(got, np.float64)
     want = np.asarray(want, np.float64)
-    excess = np.abs(got - want) - half_ulp_fp16(want)
-    ma, rl = float(excess.max()), rel_l2(got, want)
-    assert ma <= DECODE_MAX_ABS and rl <= DECODE_REL_L2, (ma, max_abs(got, want), rl)
+    err = np.abs(got - want)
+    bound = np.maximum(DECODE_MAX_ABS, half_ulp_fp16(want))
+    worst = int(np.argmax(err - bound))
+    ma, rl = float(err.max()), rel_l2(got, want)
+    assert err.flat[worst] <= bound.flat[worst] and rl <= DECODE_REL_L2, (
+        ma, float(err.flat[worst]), float(want.flat[worst]), rl)
     return ma, rl
 
 

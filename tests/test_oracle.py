@@ -173,6 +173,49 @@ def test_rotate_f32_close_to_exact_rotation():
         assert np.all(np.abs(got - exact) <= bound)
 
 
+def test_rotate_f32_butterfly_order_is_pinned_bitwise():
+    # Random and heavy-tailed vectors round differently under any other
+    # stride order or association; the C oracle must equal the stage-wise
+    # float32 restatement of the codebook's order bit for bit.
+    from oracle import brute
+    for seed in (0, 1, 12345):
+        s = oracle.signs(seed)
+        for t in range(100):
+            kind = t % 4
+            if kind == 0:
+                x = RNG.standard_normal(D)
+            elif kind == 1:
+                x = RNG.standard_t(4, D) * 10.0
+            elif kind == 2:
+                x = RNG.standard_normal(D) * np.exp(RNG.uniform(-20, 20, D))
+            else:
+                x = RNG.uniform(-1, 1, D) * 65504.0
+            x = x.astype(np.float32)
+            got = oracle.rotate_f32(x, s)
+            want = brute.rotate_f32_stages(x, s)
+            assert np.array_equal(got.view(np.uint32), want.view(np.uint32)), (seed, t)
+
+
+def test_rotate_f32_stages_detects_a_reordered_transform():
+    # the pin is sensitive: descending strides give different bits on
+    # random inputs
+    from oracle import brute
+    s = oracle.signs(0)
+    diff = 0
+    for _ in range(50):
+        x = RNG.standard_normal(D).astype(np.float32)
+        z = x * s.astype(np.float32)
+        h = D // 2
+        while h >= 1:
+            blk = z.reshape(D // (2 * h), 2, h)
+            a, b = blk[:, 0, :], blk[:, 1, :]
+            z = np.stack([a + b, a - b], axis=1).reshape(D)
+            h //= 2
+        z = z * np.array(0x3DB504F3, np.uint32).view(np.float32)
+        diff += not np.array_equal(z.view(np.uint32), brute.rotate_f32_stages(x, s).view(np.uint32))
+    assert diff > 25
+
+
 # ------------------------------------------------------------- quantiser
 def test_level_index_is_nearest_level():
     # away from midpoints the binary32 index formula picks the nearest of the

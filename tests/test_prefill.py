@@ -1,7 +1,11 @@
 """GPU chunked prefill against the fp64 oracle (rel-L2 <= 1e-2).
 
 The chunk's K/V are quantise-appended by the GPU before attention, as the
-prefill workload does; the oracle quantises the same rows itself.
+prefill workload does; the oracle quantises the same rows itself.  Every
+output row is compared: the bar is the pooled rel-L2 over the whole output,
+and each (position, head) row must also stay within PREFILL_ROW_REL_L2, so
+that one wrong head, M-tile or split boundary cannot hide in the pooled norm
+(such a row is off by order one).
 """
 import numpy as np
 import pytest
@@ -12,6 +16,26 @@ from long_context_attention_tbq4_b200 import workloads as W
 from helpers import PREFILL_REL_L2, capacity_for, gpu_caches, oracle_caches, rel_l2
 
 pytestmark = pytest.mark.gpu
+
+PREFILL_ROW_REL_L2 = 5e-2
+
+
+def check_prefill(got, want):
+    """Pooled rel-L2 <= 1e-2 and every row's rel-L2 <= PREFILL_ROW_REL_L2;
+    returns (pooled, worst row, its index)."""
+    got = np.asarray(got, np.float64).reshape(-1, 128)
+    want = np.asarray(want, np.float64).reshape(-1, 128)
+    assert np.isfinite(got).all()
+    pooled = rel_l2(got, want)
+    num = np.linalg.norm(got - want, axis=1)
+    den = np.maximum(np.linalg.norm(want, axis=1), 1e-300)
+    rows = num / den
+    worst = int(np.argmax(rows))
+    print(f"prefill rel-L2 pooled {pooled:.3e}, worst row {rows[worst]:.3e} (row {worst} "
+          f"of {len(rows)}), median row {float(np.median(rows)):.3e}")
+    assert pooled <= PREFILL_REL_L2, pooled
+    assert rows[worst] <= PREFILL_ROW_REL_L2, (worst, rows[worst])
+    return pooled, float(rows[worst]), worst
 
 
 @pytest.fixture(scope="module")
@@ -53,16 +77,29 @@ def test_prefill_small(T, n_cached, n_new, Hq, Hkv):
     cap = capacity_for(n_cached + n_new)
     got, _, _ = gpu_prefill(T, case, cap)
     want = oracle_prefill(case, cap)
-    assert rel_l2(got, want) <= PREFILL_REL_L2
+    check_prefill(got, want)
 
 
-def test_prefill_131k_sampled_rows(T):
+def test_prefill_131k_every_row(T):
+    # 512 new tokens over 131,072 cached, 24/4 heads: all 12,288 output rows
+    # against the oracle over every key each row sees
     case = W.prefill_131k()
     cap = W.round_capacity(case.n_cached + case.n_new)
     got, _, _ = gpu_prefill(T, case, cap)
-    qi = [0, 1, 2, 127, 128, 255, 256, 383, 510, 511]
-    rows = np.array([i * case.Hq + h for i in qi for h in range(0, case.Hq, 5)], np.int32)
-    want = oracle_prefill(case, cap, rows=rows).reshape(-1, 128)[rows]
-    sel = got.reshape(-1, 128)[rows]
-    assert rel_l2(sel, want) <= PREFILL_REL_L2
-    assert np.isfinite(got).all()
+    want = oracle_prefill(case, cap)
+    check_prefill(got, want)
+
+
+def test_prefill_deterministic(T):
+    # two calls on the same caches give the same bits (fixed split plan and
+    # merge order; the combine is a programmatic dependent launch)
+    import torch
+    case = W.prefill_case("det", 71, 5000, 300, 24, 4)
+    cap = capacity_for(case.n_cached + case.n_new)
+    first, kc, vc = gpu_prefill(T, case, cap)
+    q = torch.from_numpy(case.q_bf16.view(np.int16)).cuda().view(torch.bfloat16)
+    for _ in range(2):
+        again = T.tbq4_attn_prefill_chunk(q, case.n_cached, kc, vc, case.softmax_scale,
+                                          case.sign_seed)
+        assert T.tbq4_get_device_status() == 0
+        assert np.array_equal(again.float().cpu().numpy(), first)
