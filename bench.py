@@ -148,8 +148,46 @@ class Clocks:
 
 
 # ---------------------------------------------------------------- workloads
+def load_workloads():
+    """The seeded input generators, loaded by file path: importing them
+    through the package would run its __init__, which maps libtbq4.so, and
+    the reference (oracle) arm must not map the product library."""
+    import importlib.util
+    name = "_tbq4_workloads"
+    if name in sys.modules:
+        return sys.modules[name]
+    path = os.path.join(ROOT, "long_context_attention_tbq4_b200", "workloads.py")
+    spec = importlib.util.spec_from_file_location(name, path)
+    mod = importlib.util.module_from_spec(spec)
+    sys.modules[name] = mod
+    spec.loader.exec_module(mod)
+    return mod
+
+
+# What the decode path computes in: the arithmetic type of each stage.
+DECODE_DTYPE = ("u8 x s8 integer QK (q_rot as an 18-bit integer, exact int32 sums), "
+                "f16 PV operands with f32 accumulation, f32 softmax, f16 output")
+PREFILL_DTYPE = "bf16 QK and PV on tcgen05 with f32 TMEM accumulators, f32 softmax, bf16 output"
+
+
+def decode_config(case, N, world):
+    """The config both arms print (the product and the oracle reference)."""
+    return {"workload": "decode_262k", "batch": case.B, "ctx": N, "Hq": case.Hq,
+            "Hkv": case.Hkv, "head_dim": D, "kv_format": "tbq4 (66 B / 128 values)",
+            "step": "append the new token's K/V rows, then decode attention over all keys "
+                    "(split kernel + log-sum-exp combine with the inverse rotation)",
+            "l2": L2_NOTE, "launch": LAUNCH_NOTE,
+            "parallelism": "replicas" if world > 1 else "single"}
+
+
+L2_NOTE = ("flushed before every timed step: 512 MiB written, then read back "
+           "(no hits, no dirty lines left)")
+LAUNCH_NOTE = ("each step is one replay of a CUDA graph captured once (decode kernel + "
+               "combine); e2e launches eagerly")
+
+
 def decode_workload():
-    from long_context_attention_tbq4_b200 import workloads as W
+    W = load_workloads()
     case = W.decode_262k()
     N = int(case.seq_lens[0])
     bytes_kv = 2 * case.Hkv * N * BLOCK
@@ -302,7 +340,7 @@ def bench_decode(T, torch, case, N, step_bytes, kernel_bytes, steps, warmup, flu
 
 
 def bench_prefill(T, torch, steps, warmup, flush):
-    from long_context_attention_tbq4_b200 import workloads as W
+    W = load_workloads()
     c = W.prefill_131k()
     dev = torch.device("cuda")
     cap = W.round_capacity(c.n_cached + c.n_new)
@@ -396,7 +434,7 @@ def profile_decode(T, torch, case, N, n_steps):
 def profile_prefill(T, torch, n_steps):
     """Chunked-prefill steps (append the chunk, attend) with nothing else on
     the device (for ncu)."""
-    from long_context_attention_tbq4_b200 import workloads as W
+    W = load_workloads()
     c = W.prefill_131k()
     dev = torch.device("cuda")
     cap = W.round_capacity(c.n_cached + c.n_new)
@@ -554,10 +592,10 @@ def run_reference(args):
               f"{N} keys per step plus the new token's append; time scaled by {scale:g}")
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64 (the oracle's arithmetic; the encoder in f32 as the codebook fixes)",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": "decode_262k", "batch": 1, "ctx": N, "Hq": case.Hq,
-                       "Hkv": case.Hkv, "head_dim": D},
+            "config": decode_config(case, N, int(os.environ.get("WORLD_SIZE", "1"))),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.get_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -606,14 +644,8 @@ def main():
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic",
-        "config": {"workload": "decode_262k", "batch": 1, "ctx": N, "Hq": case.Hq,
-                   "Hkv": case.Hkv, "head_dim": D, "kv_format": "tbq4 (66 B / 128 values)",
-                   "l2": "flushed before every timed step: 512 MiB written, then read back "
-                         "(no hits, no dirty lines left)",
-                   "launch": "each step is one replay of a CUDA graph captured once "
-                             "(decode kernel + combine); e2e launches eagerly",
-                   "parallelism": "replicas" if world > 1 else "single"},
+        "dtype": DECODE_DTYPE, "data": "synthetic",
+        "config": decode_config(case, N, world),
         "step_bytes": step_bytes,
         "ms_per_step_eager": tot["eager_ms"],
         "pct_hbm_peak": value / world / peaks["hbm_gbs"],
@@ -633,6 +665,7 @@ def main():
     }
     if pre is not None:
         pk = peaks["bf16_tflops"]
+        pre["dtype"] = PREFILL_DTYPE
         pre["roofline"] = {"bound": "tensor", "achieved": pre["attn_kernel_tflops"],
                            "peak": pk, "unit": "TFLOP/s",
                            "frac": pre["attn_kernel_tflops"] / pk,
