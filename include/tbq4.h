@@ -74,11 +74,18 @@ typedef enum {
     TBQ4_ERR_DEVICE_TIMEOUT = 7   /* a bounded wait inside a kernel gave up */
 } tbq4_status;
 
-/* Bytes of one block (66) and of one cache (B*Hkv*capacity*66). */
+/* Bytes of one block (66: the 2-byte scale and 64 bytes of 4-bit indices,
+ * trefon.com, "Kontekst 262K na jednej RTX 4090", section "Od czego
+ * zaczalem") and of one cache (B*Hkv*capacity*66; K and V are separate
+ * caches, section "Konfiguracja", -ctk/-ctv).  0 for non-positive sizes. */
 TBQ4_API size_t tbq4_block_bytes(void);
 TBQ4_API size_t tbq4_cache_bytes(int batch, int n_kv_heads, int64_t capacity);
 
-/* Host: the +-1 diagonal for `seed`, written to out[128] (host memory). */
+/* Host: the +-1 diagonal for `seed`, written to out[128] (host memory).
+ * It is the sign step of the Hadamard rotation that defines the stored
+ * domain (page section "Od czego zaczalem": the cache and attention live in
+ * the Hadamard-rotated domain; the signs themselves are this library's
+ * codebook, above).  No error path. */
 TBQ4_API void tbq4_signs(uint64_t seed, int8_t out[128]);
 
 /*
@@ -100,7 +107,14 @@ TBQ4_API tbq4_status tbq4_quantize_append(const float *src, int B, int n_new, in
 /*
  * Decode attention (one query token per sequence) over TBQ4 caches, split
  * over the context and merged by log-sum-exp; grouped-query heads share
- * one KV stream (q head h reads KV head h / (Hq/Hkv)).
+ * one KV stream (q head h reads KV head h / (Hq/Hkv)).  This is the page's
+ * flash-attention kernel that reads the raw TBQ4 blocks from global memory
+ * and dequantises them in its inner loop, in the rotated domain, with no F16
+ * buffer (trefon.com, "Kontekst 262K na jednej RTX 4090", section "Od czego
+ * zaczalem"; enabled there by --flash-attn on with -ctk/-ctv tbq4_0, section
+ * "Konfiguracja").  q is rotated once, the output rotated back once per row.
+ * tbq4_decode_workspace_bytes returns the scratch this call needs for its
+ * split partials (0 for invalid sizes).
  *   q          device, fp32 [B][Hq][128], 16-byte aligned
  *   k_cache,
  *   v_cache    device, uint8 [B][Hkv][capacity][66], 16-byte aligned
@@ -115,6 +129,10 @@ TBQ4_API tbq4_status tbq4_quantize_append(const float *src, int B, int n_new, in
  *              bytes, 256-byte aligned; its contents need no initialisation.
  *   out        device, fp16 [B][Hq][128] (round to nearest even).
  * Constraints: Hq % Hkv == 0, Hq/Hkv <= 8, B >= 1.
+ * Errors: TBQ4_ERR_NULL, TBQ4_ERR_ALIGN (q, caches 16 bytes, workspace 256
+ * bytes), TBQ4_ERR_SHAPE (head counts, B), TBQ4_ERR_CAPACITY (capacity not a
+ * multiple of 8, or max_len > capacity), TBQ4_ERR_WORKSPACE (ws_bytes too
+ * small), TBQ4_ERR_LAUNCH.
  */
 TBQ4_API size_t tbq4_decode_workspace_bytes(int B, int Hq, int Hkv, int32_t max_len);
 TBQ4_API tbq4_status tbq4_attn_decode(const float *q, const uint8_t *k_cache,
@@ -249,10 +267,13 @@ TBQ4_API tbq4_status tbq4_attn_decode_mq(const float *q, const uint8_t *k_cache,
                                          uint64_t sign_seed, void *workspace, size_t ws_bytes,
                                          uint16_t *out, void *stream);
 
-/* As tbq4_attn_decode, with the context split into pieces of
+/* As tbq4_attn_decode (the page's decode kernel over raw blocks, section
+ * "Od czego zaczalem"), with the context split into pieces of
  * `split_tokens` keys (a multiple of 32; 0 = automatic).  The result does
  * not depend on the split beyond fp32 rounding.  Workspace requirement:
- * tbq4_decode_workspace_bytes_split(). */
+ * tbq4_decode_workspace_bytes_split() (0 for invalid sizes).  Errors as
+ * tbq4_attn_decode, plus TBQ4_ERR_SHAPE for a split that is not a multiple
+ * of 32. */
 TBQ4_API size_t tbq4_decode_workspace_bytes_split(int B, int Hq, int Hkv,
                                          int32_t max_len, int32_t split_tokens);
 TBQ4_API tbq4_status tbq4_attn_decode_split(const float *q, const uint8_t *k_cache,
@@ -282,8 +303,11 @@ TBQ4_API tbq4_status tbq4_attn_decode_split(const float *q, const uint8_t *k_cac
  *     Hkv, max_len), exceeds 8 MiB, it returns TBQ4_ERR_WORKSPACE and
  *     launches nothing.
  *   - The first call on a device looks up the device address of the array
- *     (cudaGetSymbolAddress, with that device current) and keeps it; make
- *     that first call before any stream capture.
+ *     (cudaGetSymbolAddress, with that device current) and keeps it for the
+ *     rest of the process; make that first call before any stream capture.
+ *     A cudaDeviceReset of that device invalidates the kept address, and
+ *     this library cannot see the reset: do not call this entry point on a
+ *     device again after resetting it in the same process.
  *   - All calls share the one array, which keeps what the previous call
  *     wrote.  Nothing in it needs clearing (each partial is written before
  *     it is read), but calls whose kernels overlap on the GPU, for example
@@ -301,13 +325,23 @@ TBQ4_API tbq4_status tbq4_attn_decode_noalloc(const float *q, const uint8_t *k_c
  * Chunked prefill attention for one sequence: n_new query tokens at
  * absolute positions n_cached .. n_cached+n_new-1, each attending causally
  * to keys 0 .. its own position, over TBQ4 caches that already hold the
- * chunk's K/V (call tbq4_quantize_append on the chunk first).
+ * chunk's K/V (call tbq4_quantize_append on the chunk first).  It is the
+ * same flash-attention over raw TBQ4 blocks in the rotated domain (trefon.com,
+ * "Kontekst 262K na jednej RTX 4090", section "Od czego zaczalem"; the
+ * page's server processes prompts in chunks of -ub tokens into the same
+ * cache, section "Konfiguracja"), with QK^T and PV as dense tensor-core
+ * contractions over tiles dequantised to bf16.
+ * tbq4_prefill_workspace_bytes returns its scratch size (0 for invalid
+ * sizes).
  *   q          device, bf16 bits [n_new][Hq][128], 16-byte aligned
  *   k_cache,
  *   v_cache    device, uint8 [Hkv][capacity][66] (one sequence), 16-byte
  *              aligned; n_cached + n_new <= capacity
  *   workspace  device scratch of tbq4_prefill_workspace_bytes(...) bytes
  *   out        device, bf16 bits [n_new][Hq][128] (round to nearest even)
+ * Errors: TBQ4_ERR_NULL, TBQ4_ERR_ALIGN, TBQ4_ERR_SHAPE (Hq % Hkv, G > 8,
+ * n_new outside [1, 65535]), TBQ4_ERR_CAPACITY (n_cached + n_new above
+ * capacity), TBQ4_ERR_WORKSPACE, TBQ4_ERR_LAUNCH.
  */
 TBQ4_API size_t tbq4_prefill_workspace_bytes(int n_new, int Hq, int Hkv,
                                     int64_t n_cached);
@@ -319,7 +353,8 @@ TBQ4_API tbq4_status tbq4_attn_prefill_chunk(const uint16_t *q, int n_new,
                                     size_t ws_bytes, uint16_t *out,
                                     void *stream);
 
-/* Profiling hook: while set, every attention call records `before` on its
+/* Profiling hook (the page has no counterpart; it serves the measurement
+ * of the kernels above): while set, every attention call records `before` on its
  * stream just before its attention kernel and `after` just after it, so a
  * caller can time the attention alone with cudaEventElapsedTime.  Decode:
  * the events bracket the split kernel and its combine (a programmatic
@@ -331,10 +366,25 @@ TBQ4_API void tbq4_set_timing_events(void *before, void *after);
 
 /* Synchronises `stream`, returns the first error code a kernel of this
  * library recorded on the current device since the last call (TBQ4_OK if
- * none) and clears it. */
+ * none) and clears it.  The device-side checks it reports (positions and
+ * lengths against the capacity, bounded waits) guard the kernels above; the
+ * page describes no counterpart.  TBQ4_ERR_LAUNCH if the synchronisation
+ * or the read fails. */
 TBQ4_API tbq4_status tbq4_get_device_status(void *stream);
 
-/* Static description of a status code. */
+/* Self-test of the device-side failure path (no counterpart on the page;
+ * it checks this library's own guard).  Launches one warp on `stream` that
+ * waits on a shared-memory barrier nothing will ever complete, with no copy
+ * in flight, using the same bounded wait as every kernel here; after `polls`
+ * polls (1 .. 65536) it gives up, records TBQ4_ERR_DEVICE_TIMEOUT in the
+ * device status and returns, leaving the context usable.  Returns
+ * TBQ4_ERR_SHAPE for a poll count outside that range, TBQ4_ERR_LAUNCH if the
+ * launch fails, else TBQ4_OK (the timeout itself is reported by
+ * tbq4_get_device_status). */
+TBQ4_API tbq4_status tbq4_selftest_bounded_wait(uint32_t polls, void *stream);
+
+/* Static description of a status code (this library's error codes, above;
+ * no counterpart on the page).  Never NULL. */
 TBQ4_API const char *tbq4_status_string(tbq4_status s);
 
 #ifdef __cplusplus

@@ -26,7 +26,8 @@ __all__ = [
     "tbq4_decode_workspace_bytes", "tbq4_attn_decode", "tbq4_attn_decode_append",
     "tbq4_decode_mq_workspace_bytes", "tbq4_attn_decode_mq",
     "tbq4_prefill_workspace_bytes", "tbq4_attn_prefill_chunk",
-    "tbq4_set_timing_events", "tbq4_get_device_status", "empty_cache",
+    "tbq4_set_timing_events", "tbq4_get_device_status", "tbq4_selftest_bounded_wait",
+    "empty_cache",
     "empty_pool", "tbq4_quantize_append_paged", "tbq4_attn_decode_paged",
     "BLOCK_BYTES3", "empty_cache3", "tbq3_quantize_append", "tbq3_attn_decode",
 ]
@@ -338,3 +339,11 @@ def tbq4_set_timing_events(before=None, after=None):
 def tbq4_get_device_status(stream=None) -> int:
     """Synchronises the stream and returns (and clears) the device error code."""
     return int(lib.tbq4_get_device_status(_stream(stream)))
+
+
+def tbq4_selftest_bounded_wait(polls=256, stream=None) -> None:
+    """Launches the bounded-wait self-test: one warp waits on a barrier that
+    nothing completes, gives up after `polls` polls and records
+    TBQ4_ERR_DEVICE_TIMEOUT (read it with tbq4_get_device_status)."""
+    check(lib.tbq4_selftest_bounded_wait(C.c_uint32(int(polls)), _stream(stream)),
+          "tbq4_selftest_bounded_wait")

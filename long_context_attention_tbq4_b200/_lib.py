@@ -43,6 +43,7 @@ SIGNATURES = {
                                      _u64, _p, _sz, _p, _p]),
     "tbq4_set_timing_events": (None, [_p, _p]),
     "tbq4_get_device_status": (_i, [_p]),
+    "tbq4_selftest_bounded_wait": (_i, [C.c_uint32, _p]),
     "tbq4_status_string": (C.c_char_p, [_i]),
 }
 

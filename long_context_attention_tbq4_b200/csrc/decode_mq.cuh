@@ -162,7 +162,7 @@ decode_mq_kernel(const AttnParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    const uint32_t sbase = tc::smem_addr(smem);
+    const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // the dependent combine kernel may be scheduled from now on
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -199,23 +199,23 @@ decode_mq_kernel(const AttnParams p) {
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kRawStages; ++i) {
-            tc::bar_init(raw_full(i), 1);
-            tc::bar_init(raw_empty(i), kDeqWarps);
+            mbar_init(raw_full(i), 1);
+            mbar_init(raw_empty(i), kDeqWarps);
         }
         for (int b = 0; b < 2; ++b) {
-            tc::bar_init(op_full(b), kDeqWarps);
-            tc::bar_init(s_full(b), 1);
-            tc::bar_init(s_empty(b), kSoftWarps);
-            tc::bar_init(p_full(b), kSoftWarps);
-            tc::bar_init(tile_free(b), 1);
-            for (int w = 0; w < kSoftGroups; ++w) tc::bar_init(vote(b, w), 4);
+            mbar_init(op_full(b), kDeqWarps);
+            mbar_init(s_full(b), 1);
+            mbar_init(s_empty(b), kSoftWarps);
+            mbar_init(p_full(b), kSoftWarps);
+            mbar_init(tile_free(b), 1);
+            for (int w = 0; w < kSoftGroups; ++w) mbar_init(vote(b, w), 4);
         }
-        for (int w = 0; w < kSoftGroups; ++w) tc::bar_init(mx_bar(w), 4);
-        tc::bar_init(fin_bar, kSoftWarps);
-        tc::fence_barrier_init();
+        for (int w = 0; w < kSoftGroups; ++w) mbar_init(mx_bar(w), 4);
+        mbar_init(fin_bar, kSoftWarps);
+        fence_barrier_init();
     }
     if (warp == 1) {
-        tc::tmem_alloc(tc::smem_addr(tmem_ptr), kTmemCols);
+        tc::tmem_alloc(smem_u32(tmem_ptr), kTmemCols);
         tc::tmem_relinquish();
     }
     // zero B_q (rows of absent query rows stay 0) and the P' tiles (rows of
@@ -279,7 +279,7 @@ decode_mq_kernel(const AttnParams p) {
             qpar[2 * c + 1] = 0.f;
         }
     }
-    tc::fence_proxy_async();                // B_q and the zeroed P' rows are read by the MMAs
+    fence_proxy_async();                // B_q and the zeroed P' rows are read by the MMAs
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -294,7 +294,7 @@ decode_mq_kernel(const AttnParams p) {
         for (int j = 0; j < n_tiles; ++j) {
             const int st = j % kRawStages;
             if (j >= kRawStages &&
-                !tc::bar_wait_warp(raw_empty(st), ((j / kRawStages) - 1) & 1, kSpin)) {
+                !mbar_wait_bounded(raw_empty(st), ((j / kRawStages) - 1) & 1, kSpin)) {
                 record_status(7u);
                 break;
             }
@@ -303,8 +303,8 @@ decode_mq_kernel(const AttnParams p) {
             const int rows = (min(kTile, t1 - tj) + 7) & ~7;
             const uint32_t dst = sbase + kOffRaw + st * kRawStageBytes;
             if (lane == 0) {
-                tc::fence_proxy_async();
-                tc::bar_expect_tx(raw_full(st), 2u * (uint32_t)rows * kBlockBytes);
+                fence_proxy_async();
+                mbar_expect_tx(raw_full(st), 2u * (uint32_t)rows * kBlockBytes);
             }
             __syncwarp();
             const int piece = lane >> 1, kv = lane & 1;
@@ -312,7 +312,7 @@ decode_mq_kernel(const AttnParams p) {
             if (piece < kTile / kPieceRows && r0 < rows) {
                 const uint32_t nb = (uint32_t)(min(kPieceRows, rows - r0)) * kBlockBytes;
                 const uint8_t *src = (kv ? vb : kb) + (int64_t)(tj + r0) * kBlockBytes;
-                tc::bulk_g2s(dst + kv * kRawBytes + r0 * kBlockBytes, src, nb, raw_full(st));
+                bulk_g2s(dst + kv * kRawBytes + r0 * kBlockBytes, src, nb, raw_full(st));
             }
         }
     } else if (warp == 1) {
@@ -326,8 +326,8 @@ decode_mq_kernel(const AttnParams p) {
                 bool moved = false;
                 if (jq < n_tiles && jq <= jp + 1) {
                     const int b = jq & 1;
-                    if (tc::bar_test(op_full(b), (jq >> 1) & 1) &&
-                        (jq < 2 || tc::bar_test(s_empty(b), ((jq >> 1) - 1) & 1))) {
+                    if (mbar_test(op_full(b), (jq >> 1) & 1) &&
+                        (jq < 2 || mbar_test(s_empty(b), ((jq >> 1) - 1) & 1))) {
                         tc::fence_after_sync();
                         const uint32_t kt = sbase + kOffBuf + b * kBufBytes + kKTile;
 #pragma unroll
@@ -341,7 +341,7 @@ decode_mq_kernel(const AttnParams p) {
                 }
                 if (jp < jq) {
                     const int b = jp & 1;
-                    if (tc::bar_test(p_full(b), (jp >> 1) & 1)) {
+                    if (mbar_test(p_full(b), (jp >> 1) & 1)) {
                         tc::fence_after_sync();
                         const uint32_t vt = sbase + kOffBuf + b * kBufBytes + kVTile;
                         const uint32_t pt = sbase + kOffBuf + b * kBufBytes + kPTile;
@@ -371,8 +371,8 @@ decode_mq_kernel(const AttnParams p) {
         const int d = threadIdx.x - 32 * kDeqWarp0;     // 0..127
         for (int j = 0; j < n_tiles; ++j) {
             const int st = j % kRawStages, b = j & 1;
-            if (!tc::bar_wait_warp(raw_full(st), (j / kRawStages) & 1, kSpin)) { record_status(7u); break; }
-            if (j >= 2 && !tc::bar_wait_warp(tile_free(b), ((j >> 1) - 1) & 1, kSpin)) {
+            if (!mbar_wait_bounded(raw_full(st), (j / kRawStages) & 1, kSpin)) { record_status(7u); break; }
+            if (j >= 2 && !mbar_wait_bounded(tile_free(b), ((j >> 1) - 1) & 1, kSpin)) {
                 record_status(7u);
                 break;
             }
@@ -432,11 +432,11 @@ decode_mq_kernel(const AttnParams p) {
                 for (int e = 0; e < 4; ++e)
                     sts128(vt + sw128(4 * bp + e, 16 * tg, 16384), o[e][0], o[e][1], o[e][2], o[e][3]);
             }
-            tc::fence_proxy_async();            // the tiles are read by the tensor core
+            fence_proxy_async();            // the tiles are read by the tensor core
             __syncwarp();
             if (lane == 0) {
-                tc::bar_arrive(op_full(b));
-                tc::bar_arrive(raw_empty(st));
+                mbar_arrive(op_full(b));
+                mbar_arrive(raw_empty(st));
             }
         }
     } else if (warp >= kSoftWarp0) {
@@ -467,7 +467,7 @@ decode_mq_kernel(const AttnParams p) {
         for (int j = 0; j < n_tiles; ++j) {
             const int b = j & 1;
             const uint32_t par = (j >> 1) & 1;
-            if (!tc::bar_wait_warp(s_full(b), par, kSpin) || !tc::bar_wait_warp(op_full(b), par, kSpin)) {
+            if (!mbar_wait_bounded(s_full(b), par, kSpin) || !mbar_wait_bounded(op_full(b), par, kSpin)) {
                 record_status(7u);
                 ok = false;
                 break;
@@ -480,11 +480,11 @@ decode_mq_kernel(const AttnParams p) {
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::bar_arrive(s_empty(b));
+            if (lane == 0) mbar_arrive(s_empty(b));
 
             if (8 * wg >= NQ) {                 // no query row of this warpgroup is in use
                 __syncwarp();
-                if (lane == 0) tc::bar_arrive(p_full(b));
+                if (lane == 0) mbar_arrive(p_full(b));
                 continue;
             }
             const float *sig = reinterpret_cast<const float *>(smem + kOffBuf + b * kBufBytes + kSig);
@@ -505,8 +505,8 @@ decode_mq_kernel(const AttnParams p) {
             const bool wgrow = __any_sync(kFull, grow);
             if (lane == 0) flags[kSoftWarps * b + ws] = wgrow ? 1 : 0;
             __syncwarp();
-            if (lane == 0) tc::bar_arrive(vote(b, wg));
-            if (!tc::bar_wait_warp(vote(b, wg), par, kSpin)) { record_status(7u); ok = false; break; }
+            if (lane == 0) mbar_arrive(vote(b, wg));
+            if (!mbar_wait_bounded(vote(b, wg), par, kSpin)) { record_status(7u); ok = false; break; }
             int any = 0;
 #pragma unroll
             for (int w = 0; w < 4; ++w) any |= flags[kSoftWarps * b + 4 * wg + w];
@@ -520,8 +520,8 @@ decode_mq_kernel(const AttnParams p) {
                     if (lane == 0) xch[kCols * q4 + 8 * wg + k] = wm;
                 }
                 __syncwarp();
-                if (lane == 0) tc::bar_arrive(mx_bar(wg));
-                if (!tc::bar_wait_warp(mx_bar(wg), mx_phase, kSpin)) { record_status(7u); ok = false; break; }
+                if (lane == 0) mbar_arrive(mx_bar(wg));
+                if (!mbar_wait_bounded(mx_bar(wg), mx_phase, kSpin)) { record_status(7u); ok = false; break; }
                 mx_phase ^= 1u;
                 uint32_t cs[8];
 #pragma unroll
@@ -541,7 +541,7 @@ decode_mq_kernel(const AttnParams p) {
                 // O holds PV up to tile j-1: wait for it, scale this lane's
                 // columns of this warpgroup's rows
                 if (j >= 1) {
-                    if (!tc::bar_wait_warp(tile_free((j - 1) & 1), ((j - 1) >> 1) & 1, kSpin)) {
+                    if (!mbar_wait_bounded(tile_free((j - 1) & 1), ((j - 1) >> 1) & 1, kSpin)) {
                         record_status(7u);
                         ok = false;
                         break;
@@ -570,16 +570,16 @@ decode_mq_kernel(const AttnParams p) {
                     sts16(pt + sw128(c, 2 * t, kPAtom), __half_as_ushort(ph));
                 }
             }
-            tc::fence_proxy_async();            // P' is read by the tensor core
+            fence_proxy_async();            // P' is read by the tensor core
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::bar_arrive(p_full(b));
+            if (lane == 0) mbar_arrive(p_full(b));
         }
 
         // ---- partials: thread = dimension t of O --------------------------
         uint32_t ov[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
         if (ok && n_tiles > 0) {
-            if (tc::bar_wait_warp(tile_free((n_tiles - 1) & 1), ((n_tiles - 1) >> 1) & 1, kSpin)) {
+            if (mbar_wait_bounded(tile_free((n_tiles - 1) & 1), ((n_tiles - 1) >> 1) & 1, kSpin)) {
                 tc::fence_after_sync();
                 tc::tmem_ld8(t_lane + kTmemO + 8 * wg, ov);
                 tc::tmem_wait_ld();
@@ -597,8 +597,8 @@ decode_mq_kernel(const AttnParams p) {
             }
         }
         __syncwarp();
-        if (lane == 0) tc::bar_arrive(fin_bar);
-        if (tc::bar_wait_warp(fin_bar, 0, kSpin)) {
+        if (lane == 0) mbar_arrive(fin_bar);
+        if (mbar_wait_bounded(fin_bar, 0, kSpin)) {
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const int c = 8 * wg + k;

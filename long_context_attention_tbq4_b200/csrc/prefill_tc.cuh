@@ -156,7 +156,7 @@ prefill_tc_kernel(const PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    const uint32_t sbase = tc::smem_addr(smem);
+    const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // the dependent combine may be scheduled from now on (it waits for this grid)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -191,17 +191,17 @@ prefill_tc_kernel(const PrefillParams p) {
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + kOffTmemPtr);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kRawStages; ++s) { tc::bar_init(raw_full(s), 1); tc::bar_init(raw_empty(s), 4); }
-        for (int s = 0; s < kSlots; ++s) { tc::bar_init(slot_full(s), 4); tc::bar_init(slot_empty(s), 1); }
+        for (int s = 0; s < kRawStages; ++s) { mbar_init(raw_full(s), 1); mbar_init(raw_empty(s), 4); }
+        for (int s = 0; s < kSlots; ++s) { mbar_init(slot_full(s), 4); mbar_init(slot_empty(s), 1); }
         for (int a = 0; a < 2; ++a) {
-            tc::bar_init(s_full(a), 1);
-            tc::bar_init(p_full(a), 4);
-            tc::bar_init(o_done(a), 1);
+            mbar_init(s_full(a), 1);
+            mbar_init(p_full(a), 4);
+            mbar_init(o_done(a), 1);
         }
-        tc::fence_barrier_init();
+        fence_barrier_init();
     }
     if (warp == 1) {
-        tc::tmem_alloc(tc::smem_addr(tmem_ptr), 512);
+        tc::tmem_alloc(smem_u32(tmem_ptr), 512);
         tc::tmem_relinquish();
     }
 
@@ -227,7 +227,7 @@ prefill_tc_kernel(const PrefillParams p) {
                   *reinterpret_cast<uint32_t *>(&b01), *reinterpret_cast<uint32_t *>(&b23));
         }
     }
-    tc::fence_proxy_async();                // Q tiles are read by the tensor core
+    fence_proxy_async();                // Q tiles are read by the tensor core
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -241,7 +241,7 @@ prefill_tc_kernel(const PrefillParams p) {
             for (int j = 0; j < n_tiles; ++j) {
                 const int st = j % kRawStages;
                 if (j >= kRawStages &&
-                    !tc::bar_wait_lazy(raw_empty(st), ((j / kRawStages) - 1) & 1, kSpin, kLazyNs)) {
+                    !mbar_wait_lazy(raw_empty(st), ((j / kRawStages) - 1) & 1, kSpin, kLazyNs)) {
                     record_status(7u);
                     break;
                 }
@@ -249,10 +249,10 @@ prefill_tc_kernel(const PrefillParams p) {
                 const int64_t ntok = min((int64_t)kTile, keys_total - t0);
                 const uint32_t bytes = (uint32_t)((ntok + 7) & ~7LL) * kBlockBytes;
                 const uint32_t dst = sbase + kOffRaw + st * kRawStageBytes;
-                tc::fence_proxy_async();
-                tc::bar_expect_tx(raw_full(st), 2 * bytes);
-                tc::bulk_g2s(dst, p.k + head_off + t0 * kBlockBytes, bytes, raw_full(st));
-                tc::bulk_g2s(dst + kRawBytes, p.v + head_off + t0 * kBlockBytes, bytes,
+                fence_proxy_async();
+                mbar_expect_tx(raw_full(st), 2 * bytes);
+                bulk_g2s(dst, p.k + head_off + t0 * kBlockBytes, bytes, raw_full(st));
+                bulk_g2s(dst + kRawBytes, p.v + head_off + t0 * kBlockBytes, bytes,
                              raw_full(st));
             }
         }
@@ -266,7 +266,7 @@ prefill_tc_kernel(const PrefillParams p) {
             auto wait = [&](uint32_t bar, uint32_t par) {
                 bool got = false;
                 for (uint32_t i = 0; ok && i < kSpin && !got; ++i) {
-                    got = tc::bar_test(bar, par);
+                    got = mbar_test(bar, par);
                     if (!got) __nanosleep(20);
                 }
                 if (ok && !got) { ok = false; record_status(7u); }
@@ -329,14 +329,14 @@ prefill_tc_kernel(const PrefillParams p) {
             const int st = j % kRawStages;
             const uint32_t raw = sbase + kOffRaw + st * kRawStageBytes;
             const int64_t t0 = (int64_t)(tile_begin + j) * kTile;
-            if (!tc::bar_wait_lazy_warp(raw_full(st), (j / kRawStages) & 1, kSpin, kLazyNs)) { record_status(7u); break; }
+            if (!mbar_wait_lazy_warp(raw_full(st), (j / kRawStages) & 1, kSpin, kLazyNs)) { record_status(7u); break; }
             // K tile: token t -> row t, dims contiguous, each level times the
             // token's factor S_k * scale * log2(e) / 15 rounded once (so S
             // leaves the MMA in log2 units); 0 past the cache end, where the
             // raw bytes are stale
             {
                 const int u = 2 * j, slot = u % kSlots;
-                if (u >= kSlots && !tc::bar_wait_lazy_warp(slot_empty(slot), ((u / kSlots) - 1) & 1, kSpin, kLazyNs)) {
+                if (u >= kSlots && !mbar_wait_lazy_warp(slot_empty(slot), ((u / kSlots) - 1) & 1, kSpin, kLazyNs)) {
                     record_status(7u);
                     break;
                 }
@@ -359,15 +359,15 @@ prefill_tc_kernel(const PrefillParams p) {
                            __byte_perm(l1, h1, 0x5410), __byte_perm(l0, h0, 0x7632),
                            __byte_perm(l1, h1, 0x7632));
                 }
-                tc::fence_proxy_async();
+                fence_proxy_async();
                 __syncwarp();
-                if (lane == 0) tc::bar_arrive(slot_full(slot));
+                if (lane == 0) mbar_arrive(slot_full(slot));
             }
             // V^T tile: dim d -> row d, keys contiguous; thread = token pair
             // (2pp, 2pp+1) x dims [64 hf, 64 hf + 64)
             {
                 const int u = 2 * j + 1, slot = u % kSlots;
-                if (u >= kSlots && !tc::bar_wait_lazy_warp(slot_empty(slot), ((u / kSlots) - 1) & 1, kSpin, kLazyNs)) {
+                if (u >= kSlots && !mbar_wait_lazy_warp(slot_empty(slot), ((u / kSlots) - 1) & 1, kSpin, kLazyNs)) {
                     record_status(7u);
                     break;
                 }
@@ -400,12 +400,12 @@ prefill_tc_kernel(const PrefillParams p) {
                         sts32(dst + sw128_off(d + 3, ta), v_scaled(X >> 12, s2, s1));
                     }
                 }
-                tc::fence_proxy_async();
+                fence_proxy_async();
                 __syncwarp();
-                if (lane == 0) tc::bar_arrive(slot_full(slot));
+                if (lane == 0) mbar_arrive(slot_full(slot));
             }
             __syncwarp();
-            if (lane == 0) tc::bar_arrive(raw_empty(st));
+            if (lane == 0) mbar_arrive(raw_empty(st));
         }
     } else {
         tc::regs_inc<kRegsSoft>();
@@ -420,7 +420,7 @@ prefill_tc_kernel(const PrefillParams p) {
         float m = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < n_tiles && active; ++j) {
-            if (!tc::bar_wait_warp(s_full(a), j & 1, kSpin)) {
+            if (!mbar_wait_bounded(s_full(a), j & 1, kSpin)) {
                 record_status(7u);
                 ok = false;
                 break;
@@ -498,7 +498,7 @@ prefill_tc_kernel(const PrefillParams p) {
                 if (__any_sync(kFull, need)) {
                     const float corr = (m == -INFINITY) ? 0.f : tc::ex2(m - m_new);
                     if (j > 0) {
-                        if (!tc::bar_wait_warp(o_done(a), (j - 1) & 1, kSpin)) {
+                        if (!mbar_wait_bounded(o_done(a), (j - 1) & 1, kSpin)) {
                             record_status(7u);
                             ok = false;
                             break;
@@ -546,7 +546,7 @@ prefill_tc_kernel(const PrefillParams p) {
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::bar_arrive(p_full(a));
+            if (lane == 0) mbar_arrive(p_full(a));
         }
         // ---- partial (O unnormalised, m, l) for this split -----------------
         const int h = 2 * pair + a;
@@ -554,7 +554,7 @@ prefill_tc_kernel(const PrefillParams p) {
         const int64_t prow =
             (((int64_t)(i0 + row) * p.Hq + g * p.G + h) * p.n_splits + split);
         if (active && n_tiles > 0 && ok &&
-            tc::bar_wait_warp(o_done(a), (n_tiles - 1) & 1, kSpin)) {
+            mbar_wait_bounded(o_done(a), (n_tiles - 1) & 1, kSpin)) {
             tc::fence_after_sync();
 #pragma unroll 1
             for (int ch = 0; ch < 4; ++ch) {

@@ -146,7 +146,9 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
     for (int d = 0; d < kQDepth; ++d)
         if (gi + d * gstride < groups) load_group(gi + d * gstride, d);
     const float neg = (qq & 1) ? -1.0f : 1.0f, neg2 = (qq & 2) ? -1.0f : 1.0f;
-    for (uint32_t it = 0; gi < groups; ++it, gi += gstride) {
+    bool aborted = false;
+    uint32_t it = 0;
+    for (; gi < groups; ++it, gi += gstride) {
         const int d = (int)(it % kQDepth);
         // this row's destination, while the rows load (one lane per row)
         if (qq == 0) {
@@ -171,6 +173,7 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
         }
         if (!mbar_wait_bounded(bar0 + 8 * d, (it / kQDepth) & 1u)) {
             if (lane == 0) record_status(7u /* TBQ4_ERR_DEVICE_TIMEOUT */);
+            aborted = true;
             break;
         }
         float v[32];
@@ -304,6 +307,19 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
             }
         }
         __syncwarp();
+    }
+    // After a give-up, the copies this warp still has queued (the stage it
+    // gave up on and the groups issued ahead of it) must land before the
+    // warp leaves: a CTA must not exit with bulk copies writing its shared
+    // memory.  Each gets one more bounded wait.
+    if (aborted) {
+#pragma unroll
+        for (int k = 0; k < kQDepth; ++k) {
+            if (gi + (uint32_t)k * gstride >= groups) break;
+            const uint32_t ik = it + (uint32_t)k;
+            if (!mbar_wait_bounded(bar0 + 8 * (ik % kQDepth), (ik / kQDepth) & 1u) && lane == 0)
+                record_status(7u);
+        }
     }
 }
 

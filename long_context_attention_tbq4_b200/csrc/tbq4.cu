@@ -11,6 +11,7 @@
 #include "decode_tc.cuh"
 #include "decode_mq.cuh"
 #include "prefill_tc.cuh"
+#include "selftest.cuh"
 
 #include <algorithm>
 #include <cmath>
@@ -624,6 +625,12 @@ tbq4_status tbq4_get_device_status(void *stream) {
             return TBQ4_ERR_LAUNCH;
     }
     return (tbq4_status)v;
+}
+
+tbq4_status tbq4_selftest_bounded_wait(uint32_t polls, void *stream) {
+    if (polls == 0 || polls > (1u << 16)) return TBQ4_ERR_SHAPE;
+    bounded_wait_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(polls);
+    return launch_status();
 }
 
 const char *tbq4_status_string(tbq4_status s) {

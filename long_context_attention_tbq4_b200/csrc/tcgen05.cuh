@@ -1,5 +1,6 @@
 // tcgen05.cuh -- thin inline-PTX wrappers for Blackwell (sm_100a) tensor
-// memory, UMMA and mbarrier operations used by the tcgen05 kernels.
+// memory and UMMA operations used by the tcgen05 kernels (their mbarriers,
+// bulk copies and proxy fences come from mbarrier.cuh).
 //
 // Encodings (PTX ISA, tcgen05 "shared memory descriptor" and "instruction
 // descriptor"; the same bit fields CUTLASS's UMMA::SmemDescriptor and
@@ -13,91 +14,10 @@
 #pragma once
 #include <stdint.h>
 
+#include "mbarrier.cuh"
+
 namespace tbq4 {
 namespace tc {
-
-__device__ __forceinline__ uint32_t smem_addr(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// ---- mbarrier ---------------------------------------------------------------
-__device__ __forceinline__ void bar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void bar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void bar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool bar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Non-blocking test of a phase (try_wait may suspend the thread for a while,
-// which a thread polling several barriers must avoid).
-__device__ __forceinline__ bool bar_test(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait for one thread: false after `limit` polls.
-__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, uint32_t limit) {
-    for (uint32_t i = 0; i < limit; ++i)
-        if (bar_try_wait(bar, parity)) return true;
-    return false;
-}
-
-// Bounded wait that sleeps `ns` nanoseconds between polls, for a thread
-// that runs ahead of its consumers: a polling warp takes issue slots from
-// the warps it shares a scheduler with.  False after `limit` polls.
-__device__ __forceinline__ bool bar_wait_lazy(uint32_t bar, uint32_t parity, uint32_t limit,
-                                              uint32_t ns) {
-    for (uint32_t i = 0; i < limit; ++i) {
-        if (bar_try_wait(bar, parity)) return true;
-        __nanosleep(ns);
-    }
-    return false;
-}
-__device__ __forceinline__ bool bar_wait_lazy_warp(uint32_t bar, uint32_t parity, uint32_t limit,
-                                                   uint32_t ns) {
-    const bool ok = bar_wait_lazy(bar, parity, limit, ns);
-    return __all_sync(0xffffffffu, ok);
-}
-
-// Bounded wait by a whole warp: every lane polls, and the result is the
-// same in every lane (a warp never splits on a timeout).
-__device__ __forceinline__ bool bar_wait_warp(uint32_t bar, uint32_t parity, uint32_t limit) {
-    const bool ok = bar_wait(bar, parity, limit);
-    return __all_sync(0xffffffffu, ok);
-}
-
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
-                                         uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void fence_barrier_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
 
 // ---- tensor memory ----------------------------------------------------------
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {

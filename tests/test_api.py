@@ -22,7 +22,7 @@ def T():
 
 def declared_symbols():
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"TBQ4_API[^;(]*?\b(tbq4_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"TBQ4_API[^;(]*?\b(tbq[34]_\w+)\s*\(", text)))
 
 
 def test_header_declares_the_boundary():
@@ -34,7 +34,7 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(T):
     out = subprocess.run(["nm", "-D", "--defined-only", T.LIB_PATH], check=True,
                          capture_output=True, text=True).stdout
-    exported = set(re.findall(r"\bT (tbq4_\w+)", out))
+    exported = set(re.findall(r"\bT (tbq[34]_\w+)", out))
     from long_context_attention_tbq4_b200 import _lib
     for n in declared_symbols():
         assert n in exported, n
@@ -130,6 +130,13 @@ def test_prefill_rejects_bad_arguments(T):
     assert p(n=0) == 3
     assert p(nc=120) == 4                            # n_cached + n_new > capacity
     assert p(ws_bytes=8) == 5
+
+
+def test_selftest_rejects_bad_poll_counts(T):
+    # refused on the host, before any launch
+    from long_context_attention_tbq4_b200._lib import lib as L
+    assert L.tbq4_selftest_bounded_wait(0, None) == 3
+    assert L.tbq4_selftest_bounded_wait((1 << 16) + 1, None) == 3
 
 
 def test_status_strings(T):
