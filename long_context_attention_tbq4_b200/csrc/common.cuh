@@ -81,6 +81,19 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+// Exact arithmetic on powers of two x = 2^e (normal binary32, e in
+// [-126, 127]) through the exponent field: 1/x, a/b, and the largest power
+// of two <= y (y > 0 normal).
+__device__ __forceinline__ float pow2_inv(float x) {
+    return __uint_as_float(0x7F000000u - __float_as_uint(x));
+}
+__device__ __forceinline__ float pow2_ratio(float a, float b) {
+    return __uint_as_float(__float_as_uint(a) - __float_as_uint(b) + 0x3F800000u);
+}
+__device__ __forceinline__ float pow2_floor(float y) {
+    return __uint_as_float(__float_as_uint(y) & 0xFF800000u);
+}
+
 __device__ __forceinline__ float half_bits_to_float(uint16_t h) {
     return __half2float(__ushort_as_half(h));
 }

@@ -187,8 +187,12 @@ decode_combine_kernel(const AttnParams p) {
     const int used = used_splits(p, len);
     const int64_t row0 = ((int64_t)s * p.Hq + h) * p.n_splits;
     // Launched as a programmatic dependent of the split kernel: wait for all
-    // of its partials (a no-op under an ordinary launch).
+    // of its partials (a no-op under an ordinary launch).  Then the next
+    // decode step's split kernel may start: its caches were complete before
+    // this wait returned, and it reads its own inputs and writes the
+    // workspace only after its own wait, i.e. after this grid has finished.
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (used > kCombineWarps * kCombineFast) {
         float4 O;

@@ -13,8 +13,9 @@
 // raw nibble bytes | the same & 0x0F]; B_q rows 32 pc + c = piece pc of the
 // 18-bit weights u = q_odd (raw bytes) and w = 16 q_even - q_odd (low
 // nibbles) of query row c, so S column 32 pc + c is piece pc of 16 sum_d
-// n_d q_int,d (exact); V^T holds (n - 8) 2^-10 exactly in fp16; P' = p S_v
-// 2^-8; O = 2^11 O'' + R with R = sum P'.  Query row c = i G + h is query
+// n_d q_int,d (exact); V^T holds (2n - 15) 2^-11 exactly in fp16; P' = p S_v
+// ps with ps a power of two fitted to the V scales, as two fp16 terms hi + lo
+// (N = 64: 32 rows each); O = 2^11 O''.  Query row c = i G + h is query
 // token i (of q_len) for head h of the KV group; token i sits at position
 // len - q_len + i and sees keys [0, len - q_len + i] (bottom-right causal,
 // as the chunked prefill of the same pages: trefon.com, "Kontekst 262K na
@@ -41,7 +42,7 @@ namespace dmq {
 constexpr int kThreads = 768;
 constexpr int kTile = 128;                              // tokens per tile
 constexpr int kRawBytes = kTile * kBlockBytes;          // 8448
-constexpr int kRawStages = 5;
+constexpr int kRawStages = 4;
 constexpr int kPieceRows = 32;                          // rows per bulk copy (2,112 B)
 constexpr int kRawStageBytes = 2 * kRawBytes + 16;      // K | V | pad
 constexpr int kDeqWarp0 = 4, kDeqWarps = 4;
@@ -63,8 +64,9 @@ static_assert(4 * kRegsCtl + 4 * kRegsDeq + 16 * kRegsSoft <= 24 * 80,
 // tile's S_k and S_v.  Offsets from a 1024-aligned base.
 constexpr int kKTile = 0;                               // 128 rows x 128 B, 1 atom
 constexpr int kVTile = kKTile + kTile * 128;            // 128 rows x 256 B, 2 atoms
-constexpr int kPTile = kVTile + kTile * 256;            // 32 rows x 256 B, 2 atoms
-constexpr int kPAtom = kCols * 128;                     // 4 KB
+constexpr int kPTile = kVTile + kTile * 256;            // 64 rows x 256 B, 2 atoms
+constexpr int kPRows = 2 * kCols;                       // P' as hi (rows c), lo (kCols + c)
+constexpr int kPAtom = kPRows * 128;                    // 8 KB
 constexpr int kSig = kPTile + 2 * kPAtom;               // S_k[128], S_v[128] floats
 constexpr int kBufBytes = kSig + 2 * kTile * 4;         // 58,368
 static_assert(kVTile % 1024 == 0 && kPTile % 1024 == 0 && kBufBytes % 1024 == 0, "align");
@@ -76,15 +78,19 @@ constexpr int kOffQPar = kOffRaw + kRawStages * kRawStageBytes;   // [32][2] flo
 constexpr int kOffFlags = kOffQPar + kCols * 2 * 4;               // [2][16] ints
 constexpr int kOffXch = kOffFlags + 2 * kSoftWarps * 4;           // [4][32] floats
 constexpr int kOffXfin = kOffXch + 4 * kCols * 4;                 // [4][64] floats
-constexpr int kOffBar = kOffXfin + 4 * 2 * kCols * 4;
+constexpr int kOffDsv = kOffXfin + 4 * 2 * kCols * 4;             // [2][4] floats
+constexpr int kOffTps = kOffDsv + 2 * 4 * 4;                       // [2][2] floats
+constexpr int kOffBar = kOffTps + 2 * 2 * 4;
 constexpr int kSoftGroups = kSoftWarps / 4;            // warpgroups, 8 query rows each
-constexpr int kNumBars = 2 * kRawStages + 5 * 2 + 3 * kSoftGroups + 1;   // + vote, max per group, final
+constexpr int kNumBars = 2 * kRawStages + 5 * 2 + 3 * kSoftGroups + 1 + 2;   // + vote, max per
+                                                                            // group, final, S_v max
 constexpr int kOffTmemPtr = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffTmemPtr + 16 + 1024;     // + alignment slack
 static_assert(kOffBuf % 1024 == 0 && kOffRaw % 16 == 0 && kOffBar % 8 == 0, "align");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-// tensor memory columns: S buffers at 0 and 96 (s32), O at 192 (32 x f32)
+// tensor memory columns: S buffers at 0 and 96 (s32), O at 192 (64 x f32: the
+// products with P' hi at 192 + c, with P' lo at 224 + c)
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kTmemO = 2 * kSCols;
 
@@ -92,10 +98,10 @@ constexpr uint32_t kTmemO = 2 * kSCols;
 // [4,6) D format, [7,10) A format, [10,13) B format, [15]/[16] A/B major
 // (0 = K-major), [17,23) N >> 3, [24,29) M >> 4.
 //   kind::i8:  D s32 (2), A u8 (0), B s8 (1), M = 128, N = 96
-//   kind::f16: D f32 (1), A f16 (0), B f16 (0), M = 128, N = 32
+//   kind::f16: D f32 (1), A f16 (0), B f16 (0), M = 128, N = 64 (P' hi and lo)
 constexpr uint32_t kIdescQK = (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(kSCols >> 3) << 17) |
                               ((128u >> 4) << 24);
-constexpr uint32_t kIdescPV = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(kCols >> 3) << 17) |
+constexpr uint32_t kIdescPV = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(kPRows >> 3) << 17) |
                               ((128u >> 4) << 24);
 
 __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -135,19 +141,20 @@ __device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint3
                  : "memory");
 }
 
-// V levels (n - 8) 2^-10 in fp16 from nibbles in bits 0-3 (lo) or 4-7 (hi)
+// V levels (2n - 15) 2^-11 in fp16 from nibbles in bits 0-3 (lo) or 4-7 (hi)
 // of bytes 0 and 2: the masked halves are the subnormals n 2^-24 and
-// 16 n 2^-24, scaled and shifted by one exact HFMA2.
+// 16 n 2^-24, scaled and shifted by one exact HFMA2 (the results are normal
+// fp16 numbers with at most 4 significant bits).
 __device__ __forceinline__ uint32_t hfma2u(uint32_t x, uint32_t a, uint32_t b) {
     __half2 r = __hfma2(*reinterpret_cast<__half2 *>(&x), *reinterpret_cast<__half2 *>(&a),
                         *reinterpret_cast<__half2 *>(&b));
     return *reinterpret_cast<uint32_t *>(&r);
 }
 __device__ __forceinline__ uint32_t vlo(uint32_t v) {
-    return hfma2u(v & 0x000F000Fu, 0x74007400u /* 2^14 */, 0xA000A000u /* -2^-7 */);
+    return hfma2u(v & 0x000F000Fu, 0x74007400u /* 2^14 */, 0x9F809F80u /* -15 2^-11 */);
 }
 __device__ __forceinline__ uint32_t vhi(uint32_t v) {
-    return hfma2u(v & 0x00F000F0u, 0x64006400u /* 2^10 */, 0xA000A000u);
+    return hfma2u(v & 0x00F000F0u, 0x64006400u /* 2^10 */, 0x9F809F80u);
 }
 
 __device__ __forceinline__ void split3(int x, int &c0, int &c1, int &c2) {
@@ -194,6 +201,7 @@ decode_mq_kernel(const AttnParams p) {
     auto vote = [&](int b, int wgi) { return bx + 8 * (10 + 2 * wgi + b); };   // grow flags
     auto mx_bar = [&](int wgi) { return bx + 8 * (10 + 2 * kSoftGroups + wgi); }; // tile maxima
     const uint32_t fin_bar = bx + 8 * (10 + 3 * kSoftGroups);                 // final sums
+    auto sv_bar = [&](int b) { return bx + 8 * (11 + 3 * kSoftGroups + b); }; // dequant S_v max
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + kOffTmemPtr);
     float *qpar = reinterpret_cast<float *>(smem + kOffQPar);
 
@@ -212,6 +220,7 @@ decode_mq_kernel(const AttnParams p) {
         }
         for (int w = 0; w < kSoftGroups; ++w) mbar_init(mx_bar(w), 4);
         mbar_init(fin_bar, kSoftWarps);
+        for (int b = 0; b < 2; ++b) mbar_init(sv_bar(b), kDeqWarps);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -369,6 +378,17 @@ decode_mq_kernel(const AttnParams p) {
         tc::regs_dec<kRegsDeq>();
         // ======================= dequantisation ==============================
         const int d = threadIdx.x - 32 * kDeqWarp0;     // 0..127
+        // P' = p S_v ps (fp16) with ps a power of two, the largest that keeps
+        // P' <= 2^15 for every V scale seen so far (p <= 2^8): S_v ps <= 2^7.
+        // A fixed ps = 2^-8 (room for S_v = 65504) would leave the weights of
+        // most tokens among the fp16 subnormals, whose absolute spacing costs
+        // the output up to 1e-3.  These warps see every tile's scales first:
+        // they keep ps, hand the softmax S_v ps per token and, per tile, the
+        // factor by which ps shrank (the softmax rescales O and R by it) and
+        // the tile's ps.  0 until a nonzero S_v arrives.
+        float ps = 0.f;
+        float *dsv = reinterpret_cast<float *>(smem + kOffDsv);      // [2][4] warp maxima
+        float *tps = reinterpret_cast<float *>(smem + kOffTps);      // [2] x (factor, ps)
         for (int j = 0; j < n_tiles; ++j) {
             const int st = j % kRawStages, b = j & 1;
             if (!mbar_wait_bounded(raw_full(st), (j / kRawStages) & 1, kSpin)) { record_status(7u); break; }
@@ -400,11 +420,33 @@ decode_mq_kernel(const AttnParams p) {
                     sts128(kt + sw128(t, 64 + 32 * hh + 16, 0), x[4] & m4, x[5] & m4, x[6] & m4,
                            x[7] & m4);
                 }
-                // the token's block scales S_k and S_v
+                // the token's block scales S_k and S_v (tokens past the
+                // split's end count as S_v = 0)
                 float *sig = reinterpret_cast<float *>(smem + kOffBuf + b * kBufBytes + kSig);
                 sig[t] = __half2float(__ushort_as_half((uint16_t)lds16(raw + t * kBlockBytes)));
-                sig[kTile + t] =
-                    __half2float(__ushort_as_half((uint16_t)lds16(raw + kRawBytes + t * kBlockBytes)));
+                const float sv = t0 + j * kTile + t < t1
+                    ? __half2float(__ushort_as_half((uint16_t)lds16(raw + kRawBytes + t * kBlockBytes)))
+                    : 0.f;
+                // the tile's largest S_v, over the four dequantisation warps
+                const float wmx = warp_max(sv);
+                if (lane == 0) {
+                    dsv[4 * b + (warp - kDeqWarp0)] = wmx;
+                    mbar_arrive(sv_bar(b));
+                }
+                if (!mbar_wait_bounded(sv_bar(b), (j >> 1) & 1, kSpin)) {
+                    record_status(7u);
+                    break;
+                }
+                const float smx = fmaxf(fmaxf(dsv[4 * b], dsv[4 * b + 1]),
+                                        fmaxf(dsv[4 * b + 2], dsv[4 * b + 3]));
+                float f = 1.f;
+                if (ps == 0.f ? smx > 0.f : smx * ps > 128.0f) {
+                    const float nps = pow2_floor(__fdividef(128.0f, smx));
+                    f = ps == 0.f ? 1.f : pow2_ratio(nps, ps);
+                    ps = nps;
+                }
+                sig[kTile + t] = sv * ps;
+                if (d == 0) { tps[2 * b] = f; tps[2 * b + 1] = ps; }
             }
             // V^T tile, row = dim, tokens along K; unit = (tokens 8 tg .. +7,
             // nibble bytes 2 bp, 2 bp + 1 = dims 4 bp .. +3).  Two tokens' bytes
@@ -450,7 +492,7 @@ decode_mq_kernel(const AttnParams p) {
         int *flags = reinterpret_cast<int *>(smem + kOffFlags);       // [2][16]
         float *xch = reinterpret_cast<float *>(smem + kOffXch);       // [4][32]
         float *xfin = reinterpret_cast<float *>(smem + kOffXfin);     // [4][64]
-        float f2[8], bh[8], m[8], lp[8], rp[8];
+        float f2[8], bh[8], m[8], lp[8];
         int32_t lim[8];                                     // keys of row c: [0, lim)
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -459,7 +501,6 @@ decode_mq_kernel(const AttnParams p) {
             bh[k] = qpar[2 * c + 1];
             m[k] = -INFINITY;
             lp[k] = 0.f;
-            rp[k] = 0.f;
             lim[k] = c < NQ ? len - QL + c / G + 1 : 0;
         }
         uint32_t mx_phase = 0;
@@ -489,7 +530,7 @@ decode_mq_kernel(const AttnParams p) {
             }
             const float *sig = reinterpret_cast<const float *>(smem + kOffBuf + b * kBufBytes + kSig);
             const int32_t ta = t0 + j * kTile + t;            // absolute token
-            const float sk = sig[t], sv = ta < t1 ? sig[kTile + t] : 0.f;
+            const float sk = sig[t], sv = ta < t1 ? sig[kTile + t] : 0.f;   // sv: S_v ps
             float tt[8], x[8];
             bool grow = false;
 #pragma unroll
@@ -510,7 +551,9 @@ decode_mq_kernel(const AttnParams p) {
             int any = 0;
 #pragma unroll
             for (int w = 0; w < 4; ++w) any |= flags[kSoftWarps * b + 4 * wg + w];
-            if (any) {
+            // ps shrank by fsv (a power of two) on this tile: O and R move with it
+            const float fsv = reinterpret_cast<const float *>(smem + kOffTps)[2 * b];
+            if (any || fsv != 1.f) {
                 // move the maxima to the tile's (where larger) and rescale
                 float lg[8];
 #pragma unroll
@@ -534,8 +577,7 @@ decode_mq_kernel(const AttnParams p) {
                     if (nm == -INFINITY) cc = 1.f;
                     m[k] = nm;
                     lp[k] *= cc;
-                    rp[k] *= cc;
-                    cs[k] = __float_as_uint(cc);
+                    cs[k] = __float_as_uint(cc * fsv);
                     x[k] = lg[k] == -INFINITY ? -INFINITY : lg[k] - nm;
                 }
                 // O holds PV up to tile j-1: wait for it, scale this lane's
@@ -547,17 +589,24 @@ decode_mq_kernel(const AttnParams p) {
                         break;
                     }
                     tc::fence_after_sync();
-                    uint32_t ov[8];
-                    tc::tmem_ld8(t_lane + kTmemO + 8 * wg, ov);
-                    tc::tmem_wait_ld();
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {     // the P' hi and lo products
+                        uint32_t ov[8];
+                        tc::tmem_ld8(t_lane + kTmemO + kCols * half + 8 * wg, ov);
+                        tc::tmem_wait_ld();
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        ov[k] = __float_as_uint(__uint_as_float(ov[k]) * __uint_as_float(cs[k]));
-                    tc::tmem_st8(t_lane + kTmemO + 8 * wg, ov);
+                        for (int k = 0; k < 8; ++k)
+                            ov[k] = __float_as_uint(__uint_as_float(ov[k]) * __uint_as_float(cs[k]));
+                        tc::tmem_st8(t_lane + kTmemO + kCols * half + 8 * wg, ov);
+                    }
                     tc::tmem_wait_st();
                 }
             }
-            // p, P' = p S_v 2^-8 (fp16) into row c of the P'^T tile
+            // p, P' = p S_v ps as two fp16 terms, hi = fp16(P') into row c and
+            // lo = fp16(P' - hi) into row kCols + c of the P'^T tile: one fp16
+            // term rounds each weight by up to 2^-12 relative, which moves an
+            // output made of a few comparable tokens with distant values by up
+            // to about 1e-3; the pair carries about 22 significant bits
             const uint32_t pt = sbase + kOffBuf + b * kBufBytes + kPTile;
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
@@ -565,9 +614,11 @@ decode_mq_kernel(const AttnParams p) {
                 if (c < NQ) {
                     const float pv = tc::ex2(x[k]);
                     lp[k] += pv;
-                    const __half ph = __float2half_rn(pv * sv * (1.0f / 256.0f));
-                    rp[k] += __half2float(ph);
+                    const float y = pv * sv;
+                    const __half ph = __float2half_rn(y);
+                    const __half pl = __float2half_rn(y - __half2float(ph));
                     sts16(pt + sw128(c, 2 * t, kPAtom), __half_as_ushort(ph));
+                    sts16(pt + sw128(kCols + c, 2 * t, kPAtom), __half_as_ushort(pl));
                 }
             }
             fence_proxy_async();            // P' is read by the tensor core
@@ -577,24 +628,27 @@ decode_mq_kernel(const AttnParams p) {
         }
 
         // ---- partials: thread = dimension t of O --------------------------
-        uint32_t ov[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        // the last tile's ps: 2^11 / (15 ps) restores p S_v / 15 from the
+        // (2n - 15) 2^-11 levels
+        const float ps_end = n_tiles > 0
+            ? reinterpret_cast<const float *>(smem + kOffTps)[2 * ((n_tiles - 1) & 1) + 1] : 0.f;
+        const float ips15 = (ps_end > 0.f ? pow2_inv(ps_end) : 1.0f) * (2048.0f / 15.0f);
+        uint32_t ov[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u}, ovl[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
         if (ok && n_tiles > 0) {
             if (mbar_wait_bounded(tile_free((n_tiles - 1) & 1), ((n_tiles - 1) >> 1) & 1, kSpin)) {
                 tc::fence_after_sync();
                 tc::tmem_ld8(t_lane + kTmemO + 8 * wg, ov);
+                tc::tmem_ld8(t_lane + kTmemO + kCols + 8 * wg, ovl);
                 tc::tmem_wait_ld();
             } else {
                 record_status(7u);
             }
         }
-        // l and R of each row: warp sums, then across the four lane quarters
+        // l of each row: warp sums, then across the four lane quarters
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-            const float ls = warp_sum(lp[k]), rs = warp_sum(rp[k]);
-            if (lane == 0) {
-                xfin[2 * kCols * q4 + 8 * wg + k] = ls;
-                xfin[2 * kCols * q4 + kCols + 8 * wg + k] = rs;
-            }
+            const float ls = warp_sum(lp[k]);
+            if (lane == 0) xfin[2 * kCols * q4 + 8 * wg + k] = ls;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(fin_bar);
@@ -603,18 +657,15 @@ decode_mq_kernel(const AttnParams p) {
             for (int k = 0; k < 8; ++k) {
                 const int c = 8 * wg + k;
                 if (c < NQ) {
-                    float L = 0.f, R = 0.f;
+                    float L = 0.f;
 #pragma unroll
-                    for (int qq = 0; qq < 4; ++qq) {
-                        L += xfin[2 * kCols * qq + c];
-                        R += xfin[2 * kCols * qq + kCols + c];
-                    }
+                    for (int qq = 0; qq < 4; ++qq) L += xfin[2 * kCols * qq + c];
                     const int i = c / G, h = c - (c / G) * G;
                     const int64_t row =
                         (((int64_t)s * QL + i) * p.Hq + g * G + h) * p.n_splits + split;
-                    // sum_t P'_t (2n - 15) = 2^11 O'' + R; 2^8 / 15 restores p S_v / 15
+                    // sum_t P'_t (2n - 15) = 2^11 (O''_hi + O''_lo)
                     p.part_o[row * kD + t] =
-                        fmaf(2048.0f, __uint_as_float(ov[k]), R) * (256.0f / 15.0f);
+                        (__uint_as_float(ov[k]) + __uint_as_float(ovl[k])) * ips15;
                     if (t == 0) p.part_ml[row] = make_float2(m[k], L);
                 }
             }

@@ -23,8 +23,10 @@
 // logit error below 1e-3 of a log2 unit even in the worst case.)
 // V operand: pairs of tokens are interleaved with PRMT so that one register
 // holds the same dimension of two tokens; the levels enter as (n - 8) 2^-10
-// and the odd level 2n - 15 is restored at the end (see lvl_lo).  P' = p * S_v (the
-// block scale of V), so O = sum_t p_t S_v,t (2n-15) / 15.
+// and enter as (2n - 15) 2^-11 (see lvl_lo).  P' = p * S_v * ps (S_v the
+// block scale of V, ps a per-warp power of two that keeps P' a normal fp16)
+// enters as two fp16 terms hi + lo, so O = sum_t p_t S_v,t (2n-15) / 15 once
+// 1 / ps is applied.
 // Softmax runs in fp32 in the log2 domain; the running max is per head and
 // the accumulators are only rescaled when some logit exceeds it by 2^3
 // (tested with one vote per chunk; the chunk max is only formed then).
@@ -104,30 +106,28 @@ __device__ __forceinline__ float ld_half(const uint8_t *p) {
     return __half2float(*reinterpret_cast<const __half *>(p));
 }
 
-// V levels enter the tensor cores as (n - 8) 2^-10, exact in fp16, from one
-// LOP3 and one HFMA2 per register: masking a nibble into the low mantissa
-// bits of an fp16 with a zero exponent field gives the subnormal n 2^-24
-// (bits 0-3) or 16 n 2^-24 (bits 4-7); fp16 arithmetic keeps subnormals, so
-// x 2^14 - 2^-7 (resp. x 2^10 - 2^-7) is (n - 8) 2^-10 with no rounding.
-// Since 2n - 15 = 2 (n - 8) + 1, O = 2^11 sum_t P'_t (n_t - 8) 2^-10 +
-// sum_t P'_t; the second sum (R) comes from one extra MMA per k-step with an
-// all-ones A operand.
+// V levels enter the tensor cores as (n - 7.5) 2^-10 = (2n - 15) 2^-11,
+// exact in fp16 (normal numbers, at most 4 significant bits), from one LOP3
+// and one HFMA2 per register: masking a nibble into the low mantissa bits of
+// an fp16 with a zero exponent field gives the subnormal n 2^-24 (bits 0-3)
+// or 16 n 2^-24 (bits 4-7); fp16 arithmetic keeps subnormals, so x 2^14 -
+// 15 2^-11 (resp. x 2^10 - 15 2^-11) is (2n - 15) 2^-11 with no rounding,
+// and O = 2^11 sum_t P'_t (2n_t - 15) 2^-11.
 constexpr uint32_t kH2Pow14 = 0x74007400u;     // {2^14, 2^14}
 constexpr uint32_t kH2Pow10 = 0x64006400u;     // {2^10, 2^10}
-constexpr uint32_t kH2NegBias = 0xA000A000u;   // {-2^-7, -2^-7}
-constexpr uint32_t kH2Ones = 0x3C003C00u;      // {1, 1}
-constexpr float kVLevelScale = 2048.0f;        // 2 * 2^10
+constexpr uint32_t kH2NegBias = 0x9F809F80u;   // {-15 2^-11, -15 2^-11}
+constexpr float kVLevelScale = 2048.0f;        // 2^11
 
 __device__ __forceinline__ uint32_t hfma2_u32(uint32_t x, uint32_t a, uint32_t b) {
     __half2 r = __hfma2(*reinterpret_cast<__half2 *>(&x), *reinterpret_cast<__half2 *>(&a),
                         *reinterpret_cast<__half2 *>(&b));
     return *reinterpret_cast<uint32_t *>(&r);
 }
-// low nibbles of bytes 0 and 2 -> {(n - 8) 2^-10, (n - 8) 2^-10}
+// low nibbles of bytes 0 and 2 -> {(2n - 15) 2^-11, (2n - 15) 2^-11}
 __device__ __forceinline__ uint32_t lvl_lo(uint32_t v) {
     return hfma2_u32(v & 0x000F000Fu, kH2Pow14, kH2NegBias);
 }
-// high nibbles of bytes 0 and 2 -> {(n - 8) 2^-10, (n - 8) 2^-10}
+// high nibbles of bytes 0 and 2 -> {(2n - 15) 2^-11, (2n - 15) 2^-11}
 __device__ __forceinline__ uint32_t lvl_hi(uint32_t v) {
     return hfma2_u32(v & 0x00F000F0u, kH2Pow10, kH2NegBias);
 }
@@ -172,13 +172,6 @@ decode_tc_kernel(const AttnParams p) {
     const int r = lane >> 2, c = lane & 3;
     const int split = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
     const int G = p.G;
-    // q first: these loads must not queue behind the bulk copies issued below
-    float qv[4] = {0.f, 0.f, 0.f, 0.f};
-    if (warp < G) {
-        const int64_t base = ((int64_t)s * p.Hq + g * G + warp) * kD + 4 * lane;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) qv[k] = load_q(p, base + k);
-    }
     // The first chunks are copied before the length is known, bounded by
     // max_len (<= capacity): the split's end under the largest length.
     const int32_t t0 = split * p.split_tokens;
@@ -269,6 +262,21 @@ decode_tc_kernel(const AttnParams p) {
     int q0 = warp < n_chunks_max ? warp : -1;
     int q1 = warp + kTcWarps < n_chunks_max ? warp + kTcWarps : -1;
     int q2 = warp + 2 * kTcWarps < n_chunks_max ? warp + 2 * kTcWarps : -1;
+    // Launched as a programmatic dependent of the kernel before it (the
+    // previous decode step's combine, which triggers once its own inputs are
+    // complete): everything above touches only the caches, bounded by the
+    // host's max_len, and this CTA's shared memory.  q, the lengths and the
+    // new rows, which that kernel's predecessors may produce, are read after
+    // the wait, and so are the partials written (the combine before may still
+    // be reading the workspace until the wait returns).  Under an ordinary
+    // launch the wait returns at once.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    float qv[4] = {0.f, 0.f, 0.f, 0.f};
+    if (warp < G) {
+        const int64_t base = ((int64_t)s * p.Hq + g * G + warp) * kD + 4 * lane;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) qv[k] = load_q(p, base + k);
+    }
     const int32_t len = seq_length(p, s);
     const int32_t t1 = min(len, t1_max);
     const int n_chunks = t1 > t0 ? (t1 - t0 + kChunk - 1) / kChunk : 0;
@@ -372,8 +380,15 @@ decode_tc_kernel(const AttnParams p) {
     for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
         for (int k = 0; k < 4; ++k) o[mt][k] = 0.f;
-    float rr[4] = {0.f, 0.f, 0.f, 0.f};        // sum_t P'_t for heads 2c, 2c+1
     float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+    // P' = p S_v ps in fp16, with ps a power of two per warp: the largest one
+    // that keeps P' <= 2^15 for every V scale S_v this warp has seen (p <=
+    // 2^8 under the lazy rescale), i.e. S_v <= s_lim = 2^7 / ps.  A fixed
+    // ps = 2^-8 (room for S_v = 65504) would put the weights of most tokens
+    // among the fp16 subnormals, whose absolute spacing 2^-24 costs the
+    // output up to 1e-3; with ps fitted to the data they stay normal.  ps = 0
+    // until the first chunk with a nonzero S_v.
+    float ps = 0.f, s_lim = 0.f;
     const uint32_t hsel = (r & 1) ? 0x7632u : 0x5410u;          // half of head n = r
     const int src0 = 4 * (2 * c) + (r >> 1), src1 = 4 * (2 * c + 1) + (r >> 1);
     bool aborted = false;
@@ -498,14 +513,32 @@ decode_tc_kernel(const AttnParams p) {
             for (int u = 0; u < 4; ++u)
                 if (8 * u + r >= valid) { xa[u] = -INFINITY; xb[u] = -INFINITY; sv[u] = 0.f; }
         }
-        bool grow = false;
+        bool grow = false, sgrow = false;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) grow |= (xa[u] > kLazyRescale) | (xb[u] > kLazyRescale);
+        for (int u = 0; u < 4; ++u) {
+            grow |= (xa[u] > kLazyRescale) | (xb[u] > kLazyRescale);
+            sgrow |= sv[u] > s_lim;
+        }
         // The running max is only moved (and the accumulators rescaled)
         // when some logit exceeds it by more than 2^3; otherwise
-        // p = 2^(logit - m) <= 2^8, and P' carries a factor 2^-8 so that
-        // fp16 P' = p * S_v * 2^-8 stays <= S_v <= 65504.
-        if (__any_sync(kFull, grow)) {
+        // p = 2^(logit - m) <= 2^8.  ps only shrinks, when a V scale above
+        // s_lim arrives; both are rare after the first chunks.
+        if (__any_sync(kFull, grow | sgrow)) {
+          if (__any_sync(kFull, sgrow)) {
+            float smx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+#pragma unroll
+            for (int msk = 4; msk < 32; msk <<= 1) smx = fmaxf(smx, __shfl_xor_sync(kFull, smx, msk));
+            // the largest power of two <= 2^7 / smx (smx > s_lim >= 0)
+            const float nps = pow2_floor(__fdividef(128.0f, smx));
+            const float f = ps == 0.f ? 1.f : pow2_ratio(nps, ps);    // a power of two, < 1
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                o[mt][0] *= f; o[mt][1] *= f; o[mt][2] *= f; o[mt][3] *= f;
+            }
+            ps = nps;
+            s_lim = 128.0f * pow2_inv(nps);
+          }
+          if (__any_sync(kFull, grow)) {
             float mxa = -INFINITY, mxb = -INFINITY;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -529,28 +562,40 @@ decode_tc_kernel(const AttnParams p) {
             for (int mt = 0; mt < 8; ++mt) {
                 o[mt][0] *= ca; o[mt][1] *= cb; o[mt][2] *= ca; o[mt][3] *= cb;
             }
-            rr[0] *= ca; rr[1] *= cb; rr[2] *= ca; rr[3] *= cb;
 #pragma unroll
             for (int u = 0; u < 4; ++u) { xa[u] -= m_a; xb[u] -= m_b; }
+          }
         }
-        uint32_t p2[4];
+        // P' = hi + lo, two fp16 terms: hi = fp16(P'), lo = fp16(P' - hi)
+        // (the difference is exact in fp32).  One fp16 term rounds each weight
+        // by up to 2^-12 relative, which moves an output made of a few
+        // comparable tokens with distant values by up to about 1e-3; the pair
+        // carries about 22 significant bits.
+        uint32_t p2[4], p2l[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const float pa = fast_ex2(xa[u]), pb = fast_ex2(xb[u]);
             l_a += pa;
             l_b += pb;
-            const float svs = sv[u] * (1.0f / 256.0f);
-            __half2 h = __floats2half2_rn(pa * svs, pb * svs);
+            const float svs = sv[u] * ps;
+            const float ya = pa * svs, yb = pb * svs;
+            __half2 h = __floats2half2_rn(ya, yb);
+            const float2 hf = __half22float2(h);
+            __half2 hl = __floats2half2_rn(ya - hf.x, yb - hf.y);
             p2[u] = *reinterpret_cast<uint32_t *>(&h);
+            p2l[u] = *reinterpret_cast<uint32_t *>(&hl);
         }
         // P'^T B fragments: thread (n = r, c) needs head n, tokens
         // 16ks + {2c, 2c+1} (b0) and 16ks + 8 + {2c, 2c+1} (b1).
-        uint32_t pb[2][2];
+        uint32_t pb[2][2], pbl[2][2];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const uint32_t x = __shfl_sync(kFull, p2[u], src0);
             const uint32_t y = __shfl_sync(kFull, p2[u], src1);
             pb[u >> 1][u & 1] = __byte_perm(x, y, hsel);
+            const uint32_t xl = __shfl_sync(kFull, p2l[u], src0);
+            const uint32_t yl = __shfl_sync(kFull, p2l[u], src1);
+            pbl[u >> 1][u & 1] = __byte_perm(xl, yl, hsel);
         }
 
         // ---- O^T += V^T P'^T ---------------------------------------------
@@ -590,11 +635,13 @@ decode_tc_kernel(const AttnParams p) {
                 const uint32_t Xs = X >> 8, Ys = Y >> 8;
                 // dims 16r+4q4+{0,1} -> m-tile 2q4, rows r / r+8;
                 // dims 16r+4q4+{2,3} -> m-tile 2q4+1
-                mma16816(o[2 * q4], lvl_lo(X), lvl_hi(X), lvl_lo(Y), lvl_hi(Y), pb[ks][0], pb[ks][1]);
-                mma16816(o[2 * q4 + 1], lvl_lo(Xs), lvl_hi(Xs), lvl_lo(Ys), lvl_hi(Ys), pb[ks][0],
-                         pb[ks][1]);
+                const uint32_t a0 = lvl_lo(X), a1 = lvl_hi(X), a2 = lvl_lo(Y), a3 = lvl_hi(Y);
+                const uint32_t e0 = lvl_lo(Xs), e1 = lvl_hi(Xs), e2 = lvl_lo(Ys), e3 = lvl_hi(Ys);
+                mma16816(o[2 * q4], a0, a1, a2, a3, pb[ks][0], pb[ks][1]);
+                mma16816(o[2 * q4 + 1], e0, e1, e2, e3, pb[ks][0], pb[ks][1]);
+                mma16816(o[2 * q4], a0, a1, a2, a3, pbl[ks][0], pbl[ks][1]);
+                mma16816(o[2 * q4 + 1], e0, e1, e2, e3, pbl[ks][0], pbl[ks][1]);
             }
-            mma16816(rr, kH2Ones, kH2Ones, kH2Ones, kH2Ones, pb[ks][0], pb[ks][1]);
         }
 
         __syncwarp();
@@ -652,14 +699,14 @@ decode_tc_kernel(const AttnParams p) {
     float *wt = l_w + kTcWarps * kMaxGroup;                              // [W][8]
     float2 *ml_h = reinterpret_cast<float2 *>(wt + kTcWarps * kMaxGroup);  // [8]
     {
-        // sum_t P'_t (2n - 15) = 2^11 sum_t P'_t (n - 8) 2^-10 + sum_t P'_t
+        // sum_t P'_t (2n - 15) = 2^11 sum_t P'_t (2n - 15) 2^-11, and 1 / ps
+        // (a power of two, exact) puts every warp's rows in the units of
+        // p S_v before the warps are merged
+        const float osc = kVLevelScale * (ps > 0.f ? pow2_inv(ps) : 1.0f);
         float4 *mine = reinterpret_cast<float4 *>(o_w + (warp * 32 + lane) * kLaneStride);
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt)
-            mine[mt] = make_float4(fmaf(kVLevelScale, o[mt][0], rr[0]),
-                                   fmaf(kVLevelScale, o[mt][1], rr[1]),
-                                   fmaf(kVLevelScale, o[mt][2], rr[2]),
-                                   fmaf(kVLevelScale, o[mt][3], rr[3]));
+            mine[mt] = make_float4(o[mt][0] * osc, o[mt][1] * osc, o[mt][2] * osc, o[mt][3] * osc);
     }
     if (r == 0) {
         m_w[warp * kMaxGroup + 2 * c] = m_a;
@@ -706,8 +753,8 @@ decode_tc_kernel(const AttnParams p) {
             for (int w = 0; w < kTcWarps; ++w)
                 O = fmaf(wt[w * kMaxGroup + h], src[w * 32 * kLaneStride], O);
             const int64_t row = ((int64_t)s * p.Hq + g * G + h) * p.n_splits + split;
-            // 2^8 undoes the scale of P-prime; the block factor is S/15 (S/7 for 3 bits)
-            p.part_o[row * kD + d] = O * (kBits == 4 ? 256.0f / 15.0f : 256.0f / 7.0f);
+            // the block factor is S/15 (S/7 for 3 bits)
+            p.part_o[row * kD + d] = O * (kBits == 4 ? 1.0f / 15.0f : 1.0f / 7.0f);
             if (d == 0) p.part_ml[row] = ml_h[h];
         }
     }

@@ -141,14 +141,33 @@ tbq4_status run_attention(AttnParams p, void *workspace, size_t ws_bytes,
         return TBQ4_ERR_LAUNCH;
     dim3 g1(p.n_splits, p.Hkv, p.nseq);
     if (g_ev_before) cudaEventRecord(g_ev_before, st);
-    if (mq)
+    if (mq) {
         dmq::decode_mq_kernel<<<g1, dmq::kThreads, dmq::kSmemBytes, st>>>(p);
-    else if (paged)
-        decode_tc_kernel<true><<<g1, kTcWarps * 32, kTcSmemBytesPaged, st>>>(p);
-    else if (p.tbq3)
-        decode_tc_kernel<false, 3><<<g1, kTcWarps * 32, kTcSmemBytes, st>>>(p);
-    else
-        decode_tc_kernel<false><<<g1, kTcWarps * 32, kTcSmemBytes, st>>>(p);
+    } else {
+        // A programmatic dependent of the kernel before it: the split kernel
+        // sets up and issues its first cache copies, then waits for that
+        // kernel (griddepcontrol.wait) before it reads q or the lengths.
+        // Only the decode combine triggers early, once its own inputs are
+        // complete; after any other kernel this is an ordinary launch.
+        cudaLaunchConfig_t sc = {};
+        sc.gridDim = g1;
+        sc.blockDim = dim3(kTcWarps * 32);
+        sc.dynamicSmemBytes = paged ? kTcSmemBytesPaged : kTcSmemBytes;
+        sc.stream = st;
+        cudaLaunchAttribute sa[1];
+        sa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        sa[0].val.programmaticStreamSerializationAllowed = 1;
+        sc.attrs = sa;
+        sc.numAttrs = 1;
+        cudaError_t e;
+        if (paged)
+            e = cudaLaunchKernelEx(&sc, decode_tc_kernel<true, 4>, p);
+        else if (p.tbq3)
+            e = cudaLaunchKernelEx(&sc, decode_tc_kernel<false, 3>, p);
+        else
+            e = cudaLaunchKernelEx(&sc, decode_tc_kernel<false, 4>, p);
+        if (e != cudaSuccess) return TBQ4_ERR_LAUNCH;
+    }
     // The combine is a programmatic dependent launch: its CTAs are placed as
     // decode CTAs retire and wait in griddepcontrol.wait for the whole decode
     // grid, so no launch gap separates the two kernels.

@@ -81,6 +81,9 @@ def check_decode(got, want):
     bound = np.maximum(DECODE_MAX_ABS, half_ulp_fp16(want))
     worst = int(np.argmax(err - bound))
     ma, rl = float(err.max()), rel_l2(got, want)
+    print(f"decode max-abs {ma:.3e} (worst vs bound {float(err.flat[worst]):.3e} <= "
+          f"{float(bound.flat[worst]):.3e} at |o| {abs(float(want.flat[worst])):.3f}), "
+          f"rel-L2 {rl:.3e}")
     assert err.flat[worst] <= bound.flat[worst] and rl <= DECODE_REL_L2, (
         ma, float(err.flat[worst]), float(want.flat[worst]), rl)
     return ma, rl
