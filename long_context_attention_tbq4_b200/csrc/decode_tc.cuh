@@ -626,21 +626,32 @@ decode_tc_kernel(const AttnParams p) {
                     xw[tt][1] = __byte_perm(w1, w2, 0x5432);
                 }
             }
+            // The lo products of each group of m-tiles are issued one group
+            // later than its hi products, so two MMAs on one accumulator are
+            // four MMAs apart.
+            uint32_t pa[4], pe[4];                  // the previous group's operands
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {        // byte pairs -> dims 16r + 4q4 .. +3
-                const uint32_t sel = (q4 & 1) ? 0x7632u : 0x5410u;
-                const int w = q4 >> 1;
-                const uint32_t X = __byte_perm(xw[0][w], xw[1][w], sel);   // pair (2c, 2c+1)
-                const uint32_t Y = __byte_perm(xw[2][w], xw[3][w], sel);   // pair (2c+8, 2c+9)
-                const uint32_t Xs = X >> 8, Ys = Y >> 8;
-                // dims 16r+4q4+{0,1} -> m-tile 2q4, rows r / r+8;
-                // dims 16r+4q4+{2,3} -> m-tile 2q4+1
-                const uint32_t a0 = lvl_lo(X), a1 = lvl_hi(X), a2 = lvl_lo(Y), a3 = lvl_hi(Y);
-                const uint32_t e0 = lvl_lo(Xs), e1 = lvl_hi(Xs), e2 = lvl_lo(Ys), e3 = lvl_hi(Ys);
-                mma16816(o[2 * q4], a0, a1, a2, a3, pb[ks][0], pb[ks][1]);
-                mma16816(o[2 * q4 + 1], e0, e1, e2, e3, pb[ks][0], pb[ks][1]);
-                mma16816(o[2 * q4], a0, a1, a2, a3, pbl[ks][0], pbl[ks][1]);
-                mma16816(o[2 * q4 + 1], e0, e1, e2, e3, pbl[ks][0], pbl[ks][1]);
+            for (int q4 = 0; q4 < 5; ++q4) {        // byte pairs -> dims 16r + 4q4 .. +3
+                uint32_t na[4], ne[4];
+                if (q4 < 4) {
+                    const uint32_t sel = (q4 & 1) ? 0x7632u : 0x5410u;
+                    const int w = q4 >> 1;
+                    const uint32_t X = __byte_perm(xw[0][w], xw[1][w], sel);   // pair (2c, 2c+1)
+                    const uint32_t Y = __byte_perm(xw[2][w], xw[3][w], sel);   // pair (2c+8, 2c+9)
+                    const uint32_t Xs = X >> 8, Ys = Y >> 8;
+                    na[0] = lvl_lo(X); na[1] = lvl_hi(X); na[2] = lvl_lo(Y); na[3] = lvl_hi(Y);
+                    ne[0] = lvl_lo(Xs); ne[1] = lvl_hi(Xs); ne[2] = lvl_lo(Ys); ne[3] = lvl_hi(Ys);
+                    mma16816(o[2 * q4], na[0], na[1], na[2], na[3], pb[ks][0], pb[ks][1]);
+                    mma16816(o[2 * q4 + 1], ne[0], ne[1], ne[2], ne[3], pb[ks][0], pb[ks][1]);
+                }
+                if (q4 > 0) {
+                    mma16816(o[2 * q4 - 2], pa[0], pa[1], pa[2], pa[3], pbl[ks][0], pbl[ks][1]);
+                    mma16816(o[2 * q4 - 1], pe[0], pe[1], pe[2], pe[3], pbl[ks][0], pbl[ks][1]);
+                }
+                if (q4 < 4) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) { pa[k] = na[k]; pe[k] = ne[k]; }
+                }
             }
         }
 

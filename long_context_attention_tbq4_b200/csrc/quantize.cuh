@@ -58,15 +58,16 @@ __device__ __forceinline__ uint32_t encode_row(float v[4], uint32_t sbits, int l
 //             FMA), q = RN(q0 + e r).  rint is an add of 1.5 * 2^23 on the
 //             FMA pipe; the clamp is needed only for rows whose fp16 scale is
 //             zero, subnormal or saturated, and is applied to x for those.
-// Memory: rows go in groups of 8 in head-major order (row = (b Hkv + h)
-// n_new + t), so a group's 8 blocks are contiguous in the cache.  Lane l
+// Memory: rows go in groups of 8 consecutive positions of one (sequence, KV
+// head), so a group's 8 blocks are contiguous in the cache.  Lane l
 // takes row l % 8 of its warp's group and quarter l / 8 of that row.  One
 // CTA of 16 warps per SM; each warp streams its groups through a ring of
 // kQDepth shared-memory stages, one 512-byte cp.async.bulk per row (rows 528
 // bytes apart, so the eight lanes of a 16-byte read phase hit eight
 // different bank groups), and sends the copies of a later group into a stage
 // as soon as the rows are in registers.  The blocks go out from a per-warp
-// staging area as consecutive 16-bit pieces.
+// staging area, as one bulk shared -> global copy when the group's 8 blocks
+// are consecutive and 16-byte aligned, else as 16-bit pieces.
 // Paged destination: row (b, pos) goes to page table[b][pos / page_size],
 // row pos % page_size, of a pool [n_pages][Hkv][page_size][66].  A null
 // table means the contiguous cache [B][Hkv][capacity][66].
@@ -95,20 +96,68 @@ static_assert(kQSmemBytes <= 227 * 1024, "shared memory per CTA");
 static_assert(kQStageBytes % 16 == 0 && kQRowStride % 16 == 0 && kQOutBytes % 16 == 0,
               "bulk copies and staged rows stay 16-byte aligned");
 
-// kBits: 4 (TBQ4, 66-byte blocks) or 3 (TBQ3, 50-byte blocks).  Group k of a
-// CTA is group blockIdx.x + k gridDim.x, taken by warp k % kQWarps.
+// Unsigned division by a divisor fixed for the whole launch, as a multiply
+// and shifts (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994, Figure 4.1): with l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1, n / d = (t + ((n - t) >> 1)) >> (l - 1)
+// where t = umulhi(m, n), for every 32-bit n (d = 1: n itself).
+struct InvDiv {
+    uint32_t m, l;
+    __host__ __device__ static InvDiv make(uint32_t d) {      // d >= 1
+        InvDiv v;
+        v.l = 0;
+        while (v.l < 32 && (1ull << v.l) < d) ++v.l;
+        v.m = v.l == 0 ? 0u : (uint32_t)((((1ull << v.l) - d) << 32) / d + 1);
+        return v;
+    }
+    __device__ __forceinline__ uint32_t div(uint32_t n) const {
+        if (l == 0) return n;
+        const uint32_t t = __umulhi(m, n);
+        return (t + ((n - t) >> 1)) >> (l - 1);
+    }
+};
+
+// Bulk shared -> global copy of `bytes` (a multiple of 16; both addresses
+// 16-byte aligned), tracked by this thread's bulk-async group.
+__device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(dst), "r"(src), "r"(bytes) : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until this thread's bulk stores have read their shared-memory source.
+__device__ __forceinline__ void bulk_s2g_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Waits until this thread's bulk stores are complete.
+__device__ __forceinline__ void bulk_s2g_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// kBits: 4 (TBQ4, 66-byte blocks) or 3 (TBQ3, 50-byte blocks).  A group is 8
+// consecutive positions t0 .. t0+7 of one (sequence b, KV head h): groups
+// are numbered (b Hkv + h) gpb + t0 / 8 with gpb = ceil(n_new / 8).  Group k
+// of a CTA is group blockIdx.x + k gridDim.x, taken by warp k % kQWarps.
 template <int kBits>
 __global__ void __launch_bounds__(kQThreads, 1)
 quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
                      const int32_t *__restrict__ start_pos, int64_t capacity, uint64_t sign_lo,
-                     uint64_t sign_hi, const PageMap pm, uint8_t *__restrict__ cache) {
+                     uint64_t sign_hi, const PageMap pm, uint8_t *__restrict__ cache,
+                     const InvDiv div_gpb, const InvDiv div_hkv) {
     extern __shared__ __align__(128) uint8_t qsm[];
     constexpr int kBlk = kBits == 4 ? kBlockBytes : kBlockBytes3;
     constexpr int kPieces = kBlk / 2;                         // 16-bit pieces per block
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int rho = lane & 7, qq = lane >> 3;                 // row of the group, quarter
-    const uint32_t rows = (uint32_t)B * (uint32_t)n_new * (uint32_t)Hkv;    // < 2^31 (host)
-    const uint32_t groups = (rows + kQRows - 1) / kQRows;
+    // groups per (sequence, KV head); B Hkv gpb < 2^31 (the host bounds the rows)
+    const uint32_t gpb = ((uint32_t)n_new + kQRows - 1) / kQRows;
+    const uint32_t groups = (uint32_t)B * (uint32_t)Hkv * gpb;
+    // group gi -> sequence b, KV head h, first position t0
+    auto group_of = [&](uint32_t gi, uint32_t &b, uint32_t &h, uint32_t &t0) {
+        const uint32_t bh = div_gpb.div(gi);
+        t0 = (gi - bh * gpb) * kQRows;
+        b = div_hkv.div(bh);
+        h = bh - b * (uint32_t)Hkv;
+    };
     uint8_t *ring = qsm + warp * kQDepth * kQStageBytes;
     uint8_t *wout = qsm + kQRingBytes + warp * kQOutBytes;
     uint16_t *stage = reinterpret_cast<uint16_t *>(wout);                     // [8][kPieces]
@@ -131,9 +180,9 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
         if (lane == 0) mbar_expect_tx(bar0 + 8 * d, kQRows * 512);
         __syncwarp();
         if (lane < kQRows) {
-            const uint32_t r = min(gi * kQRows + lane, rows - 1);
-            const uint32_t t = r % (uint32_t)n_new, bh = r / (uint32_t)n_new;
-            const uint32_t h = bh % (uint32_t)Hkv, b = bh / (uint32_t)Hkv;
+            uint32_t b, h, t0;
+            group_of(gi, b, h, t0);
+            const uint32_t t = min(t0 + lane, (uint32_t)n_new - 1);
             const float *srow = src + (((int64_t)b * n_new + t) * Hkv + h) * kD;
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             bulk_g2s(smem_u32(ring + d * kQStageBytes + lane * kQRowStride), srow, 512,
@@ -151,12 +200,12 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
     for (; gi < groups; ++it, gi += gstride) {
         const int d = (int)(it % kQDepth);
         // this row's destination, while the rows load (one lane per row)
+        int64_t doff = -1;          // -1: nothing stored (past the end or a bad position)
         if (qq == 0) {
-            const uint32_t r = gi * kQRows + rho;
-            int64_t doff = -1;      // -1: nothing stored (past the end or a bad position)
-            if (r < rows) {
-                const uint32_t t = r % (uint32_t)n_new, bh = r / (uint32_t)n_new;
-                const uint32_t h = bh % (uint32_t)Hkv, b = bh / (uint32_t)Hkv;
+            uint32_t b, h, t0;
+            group_of(gi, b, h, t0);
+            const uint32_t t = t0 + rho;
+            if (t < (uint32_t)n_new) {
                 const int64_t pos = (int64_t)__ldg(start_pos + b) + t;
                 if (pos < 0 || pos >= capacity) {
                     record_status(4u /* TBQ4_ERR_CAPACITY */);
@@ -269,6 +318,9 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
             const float u = __fadd_rn(__fmul_rn(q, kL), kL);
             return __float_as_uint(__fadd_rn(u, 12582912.0f)) & (kBits == 4 ? 0xFu : 0x7u);
         };
+        // the previous group's bulk store must have read the staging area
+        if (lane == 0) bulk_s2g_wait_read();
+        __syncwarp();
         uint16_t *mine = stage + rho * kPieces;
         if (qq == 0) mine[0] = sb;
         if constexpr (kBits == 4) {
@@ -295,18 +347,33 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
                 mine[3 + 6 * qq + 3 * h2] = (uint16_t)(wd >> 32);
             }
         }
-        __syncwarp();
-        // store: the 8 blocks as 8 x kPieces consecutive 16-bit pieces
+        // store.  The group's 8 blocks usually land back to back (8
+        // consecutive positions of one KV head) on a 16-byte boundary
+        // (positions in steps of 8 from a multiple of 8): then one bulk copy
+        // of 8 kBlk bytes, issued by lane 0 after every lane's staging writes
+        // are made visible to the async proxy.  Otherwise (a ragged group, a
+        // skipped row, an unaligned start, a page boundary) each block goes out
+        // as 16-bit pieces.
+        const int64_t d0 = doffs[0], dme = doffs[rho];
+        const bool bulk = __all_sync(kFull, dme == d0 + (int64_t)rho * kBlk) && d0 >= 0 &&
+                          (d0 & 15) == 0;
+        if (bulk) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) bulk_s2g(cache + d0, smem_u32(stage), kQRows * kBlk);
+        } else {
+            __syncwarp();
 #pragma unroll
-        for (int k2 = 0; k2 < (kQRows * kPieces + 31) / 32; ++k2) {
-            const int j = lane + 32 * k2;
-            if (j < kQRows * kPieces) {
-                const int row = j / kPieces, pc = j - row * kPieces;
-                const int64_t off = doffs[row];
-                if (off >= 0) *reinterpret_cast<uint16_t *>(cache + off + 2 * pc) = stage[j];
+            for (int k2 = 0; k2 < (kQRows * kPieces + 31) / 32; ++k2) {
+                const int j = lane + 32 * k2;
+                if (j < kQRows * kPieces) {
+                    const int row = j / kPieces, pc = j - row * kPieces;
+                    const int64_t off = doffs[row];
+                    if (off >= 0) *reinterpret_cast<uint16_t *>(cache + off + 2 * pc) = stage[j];
+                }
             }
+            __syncwarp();
         }
-        __syncwarp();
     }
     // After a give-up, the copies this warp still has queued (the stage it
     // gave up on and the groups issued ahead of it) must land before the
@@ -321,6 +388,8 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
                 record_status(7u);
         }
     }
+    // the last bulk store completes before the CTA's shared memory goes away
+    if (lane == 0) bulk_s2g_wait_all();
 }
 
 

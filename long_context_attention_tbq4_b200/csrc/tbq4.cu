@@ -265,15 +265,20 @@ tbq4_status quantize_impl(const float *src, int B, int n_new, int Hkv, const int
     const void *fn = bits == 3 ? (const void *)quantize_rows_kernel<3>
                                : (const void *)quantize_rows_kernel<4>;
     if (!ensure_smem_attr(fn, kQSmemBytes, bits == 3 ? attr3 : attr4)) return TBQ4_ERR_LAUNCH;
-    // one CTA per SM, each over a strided share of the 8-row groups
-    int64_t blocks = ceil_div(rows, (int64_t)kQRows);
+    // one CTA per SM, each over a strided share of the 8-position groups of
+    // every (sequence, KV head)
+    const int64_t gpb = ceil_div(n_new, (int64_t)kQRows);
+    const int64_t groups = (int64_t)B * Hkv * gpb;
+    if (groups > 0x7FFFFFFFLL) return TBQ4_ERR_SHAPE;
+    const InvDiv div_gpb = InvDiv::make((uint32_t)gpb), div_hkv = InvDiv::make((uint32_t)Hkv);
+    int64_t blocks = groups;
     if (blocks > (int64_t)kNumSMs) blocks = (int64_t)kNumSMs;
     if (bits == 3)
         quantize_rows_kernel<3><<<(unsigned)blocks, kQThreads, kQSmemBytes, (cudaStream_t)stream>>>(
-            src, B, n_new, Hkv, start_pos, capacity, lo, hi, pm, cache);
+            src, B, n_new, Hkv, start_pos, capacity, lo, hi, pm, cache, div_gpb, div_hkv);
     else
         quantize_rows_kernel<4><<<(unsigned)blocks, kQThreads, kQSmemBytes, (cudaStream_t)stream>>>(
-            src, B, n_new, Hkv, start_pos, capacity, lo, hi, pm, cache);
+            src, B, n_new, Hkv, start_pos, capacity, lo, hi, pm, cache, div_gpb, div_hkv);
     return launch_status();
 }
 
