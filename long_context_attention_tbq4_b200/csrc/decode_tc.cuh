@@ -154,6 +154,24 @@ __device__ __forceinline__ uint32_t tbq3_nibbles(uint32_t g) {
     return t + 0x44444444u;                                       // i + 4, no carries
 }
 
+// 3-bit V levels straight from the packed indices, with no expansion to
+// nibbles.  For two tokens' 24-bit groups A and B (indices 8g .. 8g+7 at bits
+// 3k .. 3k+2), three byte permutations put every field inside the mantissa
+// bits of an fp16 half: [A0 A1 B0 B1] holds fields 0, 1, 2 at bits 0, 3, 6;
+// [A1 A2 B1 B2] fields 3, 4, 5 at bits 1, 4, 7; [A2 A3 B2 B3] fields 6, 7 at
+// bits 2, 5.  Masking a field gives the subnormal i 2^(b - 24); one HFMA2 by
+// 2^(14 - b) minus 7 2^-11 turns it into (2i - 7) 2^-11, exactly.  Returns
+// field f of A (low half) and of B (high half).
+template <int f>
+__device__ __forceinline__ uint32_t lvl3(uint32_t A, uint32_t B) {
+    constexpr uint32_t kSel[8] = {0x5410u, 0x5410u, 0x5410u, 0x6521u,
+                                  0x6521u, 0x6521u, 0x7632u, 0x7632u};
+    constexpr int kBit[8] = {0, 3, 6, 1, 4, 7, 2, 5};
+    constexpr uint32_t kMask = 0x00070007u << kBit[f];
+    constexpr uint32_t kMul = (uint32_t)(15 + 14 - kBit[f]) << 10;     // fp16 2^(14 - b)
+    return hfma2_u32(__byte_perm(A, B, kSel[f]) & kMask, kMul | (kMul << 16), 0x9B009B00u);
+}
+
 // kPaged: the caches are page pools addressed through p.block_table.
 // kBits: 4 (TBQ4, 66-byte blocks) or 3 (TBQ3, 50-byte blocks; the stage
 // layout is the same, a 3-bit chunk fills 1,600 of its 2,112 bytes).
@@ -601,6 +619,62 @@ decode_tc_kernel(const AttnParams p) {
         // ---- O^T += V^T P'^T ---------------------------------------------
         // thread (r, c): dims 16r .. 16r+15 (m-tile mt: rows r -> dim
         // 16r+2mt, r+8 -> dim 16r+2mt+1), tokens 16ks + {2c,2c+1,2c+8,2c+9}.
+        if constexpr (kBits == 3) {
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            // groups 2r and 2r+1 (bytes 6r .. 6r+5, dims 16r .. 16r+15) of
+            // tokens 16ks + {2c, 2c+1, 2c+8, 2c+9}; two aligned words always
+            // cover the 6 bytes (they start at an even offset)
+            uint32_t gw[4][2];
+#pragma unroll
+            for (int tt = 0; tt < 4; ++tt) {
+                const int tok = 16 * ks + (tt & 1) + 8 * (tt >> 1);
+                const int off = voff + tok * kBlk;
+                const uint32_t lo = ld_u32(vst + (off & ~3)), hi = ld_u32(vst + (off & ~3) + 4);
+                const uint32_t sh = (uint32_t)(off & 3) * 8u;
+                const uint32_t d0 = __funnelshift_r(lo, hi, sh), d1 = hi >> sh;
+                gw[tt][0] = d0;
+                gw[tt][1] = __funnelshift_r(d0, d1, 24);
+            }
+            // m-tile mt: dims 16r + 2mt (rows r) and 16r + 2mt + 1 (rows r + 8)
+            // = fields 2 (mt % 4), +1 of group 2r + mt / 4; as in the 4-bit
+            // path, each m-tile's lo product is issued after the next m-tile's
+            // hi product
+            uint32_t pa[4];
+#pragma unroll
+            for (int mt = 0; mt < 9; ++mt) {
+                uint32_t na[4];
+                if (mt < 8) {
+                    const int gg = mt >> 2;
+                    switch (mt & 3) {
+                    case 0:
+                        na[0] = lvl3<0>(gw[0][gg], gw[1][gg]); na[1] = lvl3<1>(gw[0][gg], gw[1][gg]);
+                        na[2] = lvl3<0>(gw[2][gg], gw[3][gg]); na[3] = lvl3<1>(gw[2][gg], gw[3][gg]);
+                        break;
+                    case 1:
+                        na[0] = lvl3<2>(gw[0][gg], gw[1][gg]); na[1] = lvl3<3>(gw[0][gg], gw[1][gg]);
+                        na[2] = lvl3<2>(gw[2][gg], gw[3][gg]); na[3] = lvl3<3>(gw[2][gg], gw[3][gg]);
+                        break;
+                    case 2:
+                        na[0] = lvl3<4>(gw[0][gg], gw[1][gg]); na[1] = lvl3<5>(gw[0][gg], gw[1][gg]);
+                        na[2] = lvl3<4>(gw[2][gg], gw[3][gg]); na[3] = lvl3<5>(gw[2][gg], gw[3][gg]);
+                        break;
+                    default:
+                        na[0] = lvl3<6>(gw[0][gg], gw[1][gg]); na[1] = lvl3<7>(gw[0][gg], gw[1][gg]);
+                        na[2] = lvl3<6>(gw[2][gg], gw[3][gg]); na[3] = lvl3<7>(gw[2][gg], gw[3][gg]);
+                        break;
+                    }
+                    mma16816(o[mt], na[0], na[1], na[2], na[3], pb[ks][0], pb[ks][1]);
+                }
+                if (mt > 0)
+                    mma16816(o[mt - 1], pa[0], pa[1], pa[2], pa[3], pbl[ks][0], pbl[ks][1]);
+                if (mt < 8) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) pa[k] = na[k];
+                }
+            }
+        }
+        } else {
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
             uint32_t xw[4][2];   // [token 2c, 2c+1, 2c+8, 2c+9][word]
@@ -608,16 +682,7 @@ decode_tc_kernel(const AttnParams p) {
             for (int tt = 0; tt < 4; ++tt) {
                 const int tok = 16 * ks + (tt & 1) + 8 * (tt >> 1);
                 const uint8_t *a = vst + voff + tok * kBlk;
-                if constexpr (kBits == 3) {
-                    // 6 bytes (two 24-bit groups) from an even offset: two
-                    // aligned words always cover them
-                    const int off = voff + tok * kBlk;
-                    const uint32_t lo = ld_u32(vst + (off & ~3)), hi = ld_u32(vst + (off & ~3) + 4);
-                    const uint32_t sh = (uint32_t)(off & 3) * 8u;
-                    const uint32_t d0 = __funnelshift_r(lo, hi, sh), d1 = hi >> sh;
-                    xw[tt][0] = tbq3_nibbles(d0 & 0x00FFFFFFu);
-                    xw[tt][1] = tbq3_nibbles(__funnelshift_r(d0, d1, 24) & 0x00FFFFFFu);
-                } else if (tt & 1) {     // odd token: its nibbles are 4-byte aligned
+                if (tt & 1) {     // odd token: its nibbles are 4-byte aligned
                     xw[tt][0] = ld_u32(a);
                     xw[tt][1] = ld_u32(a + 4);
                 } else {                 // even token: 2 bytes past a 4-byte boundary
@@ -655,6 +720,7 @@ decode_tc_kernel(const AttnParams p) {
             }
         }
 
+        }
         __syncwarp();
         if (stage2_pending) {                 // first chunk: the deferred stage 2
             stage2_pending = false;
