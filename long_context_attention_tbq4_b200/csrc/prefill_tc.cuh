@@ -27,6 +27,8 @@
 // M-tile's MMAs).  The row max is only moved (and O rescaled) when it grows
 // by more than 8 in log2 units.
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 #include "decode.cuh"
 #include "tcgen05.cuh"
@@ -448,18 +450,25 @@ prefill_tc_kernel(const PrefillParams p) {
                 const float2 negm = make_float2(-m, -m);
                 float2 lf[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
                 uint32_t pk[kTile / 2];
+                // The causal mask only on the few tiles that reach the
+                // diagonal: a separate loop, chosen once per tile, so the
+                // others carry no per-element compare and select.
+                auto fast_p = [&](auto masked) {
 #pragma unroll
-                for (int e = 0; e < kTile; e += 2) {
-                    float2 d = __fadd2_rn(make_float2(sr_[e], sr_[e + 1]), negm);
-                    if (diag) {
-                        if (e > rel) d.x = -INFINITY;
-                        if (e + 1 > rel) d.y = -INFINITY;
+                    for (int e = 0; e < kTile; e += 2) {
+                        float2 d = __fadd2_rn(make_float2(sr_[e], sr_[e + 1]), negm);
+                        if constexpr (decltype(masked)::value) {
+                            if (e > rel) d.x = -INFINITY;
+                            if (e + 1 > rel) d.y = -INFINITY;
+                        }
+                        const float2 pr = make_float2(tc::ex2(d.x), tc::ex2(d.y));
+                        lf[(e >> 1) & 1] = __fadd2_rn(lf[(e >> 1) & 1], pr);
+                        __nv_bfloat162 bb = __floats2bfloat162_rn(pr.x, pr.y);
+                        pk[e >> 1] = *reinterpret_cast<uint32_t *>(&bb);
                     }
-                    const float2 pr = make_float2(tc::ex2(d.x), tc::ex2(d.y));
-                    lf[(e >> 1) & 1] = __fadd2_rn(lf[(e >> 1) & 1], pr);
-                    __nv_bfloat162 bb = __floats2bfloat162_rn(pr.x, pr.y);
-                    pk[e >> 1] = *reinterpret_cast<uint32_t *>(&bb);
-                }
+                };
+                if (diag) fast_p(std::true_type{});
+                else fast_p(std::false_type{});
                 const float lt = (lf[0].x + lf[0].y) + (lf[1].x + lf[1].y);
                 if (!__any_sync(kFull, !(lt <= kFastSumLimit))) {
                     l += lt;
