@@ -74,7 +74,8 @@ def measured_peaks():
 KERNEL_SOURCES = {
     "decode_tc_kernel": ["common.cuh", "mbarrier.cuh", "quantize.cuh", "decode.cuh",
                          "decode_tc.cuh"],
-    "prefill_tc_kernel": ["common.cuh", "decode.cuh", "tcgen05.cuh", "prefill_tc.cuh"],
+    "prefill_tc_kernel": ["common.cuh", "mbarrier.cuh", "decode.cuh", "tcgen05.cuh",
+                          "prefill_tc.cuh"],
     "quantize_rows_kernel": ["common.cuh", "mbarrier.cuh", "quantize.cuh"],
 }
 
