@@ -71,7 +71,13 @@ typedef enum {
                                      position/length outside [0, capacity] */
     TBQ4_ERR_WORKSPACE = 5,       /* workspace smaller than required       */
     TBQ4_ERR_LAUNCH = 6,          /* a CUDA launch or query failed         */
-    TBQ4_ERR_DEVICE_TIMEOUT = 7   /* a bounded wait inside a kernel gave up */
+    TBQ4_ERR_DEVICE_TIMEOUT = 7,  /* a bounded wait inside a kernel gave up */
+    TBQ4_ERR_BOUNDS = 8           /* debug build only (libtbq4_debug.so, built
+                                     with -DTBQ4_DEBUG): a global access a
+                                     kernel derived from lengths, positions,
+                                     page ids or its split plan fell outside
+                                     its buffer; the access was skipped (a
+                                     tracked copy was redirected to offset 0) */
 } tbq4_status;
 
 /* Bytes of one block (66: the 2-byte scale and 64 bytes of 4-bit indices,
@@ -367,8 +373,9 @@ TBQ4_API void tbq4_set_timing_events(void *before, void *after);
 /* Synchronises `stream`, returns the first error code a kernel of this
  * library recorded on the current device since the last call (TBQ4_OK if
  * none) and clears it.  The device-side checks it reports (positions and
- * lengths against the capacity, bounded waits) guard the kernels above; the
- * page describes no counterpart.  TBQ4_ERR_LAUNCH if the synchronisation
+ * lengths against the capacity, bounded waits, and in the debug build the
+ * bounds checks of TBQ4_ERR_BOUNDS) guard the kernels above; the page
+ * describes no counterpart.  TBQ4_ERR_LAUNCH if the synchronisation
  * or the read fails. */
 TBQ4_API tbq4_status tbq4_get_device_status(void *stream);
 

@@ -2,13 +2,16 @@
 
 The library must have been built in-tree (``python
 long_context_attention_tbq4_b200/build.py``); if it is missing this module
-raises at import, there is no fallback implementation.
+raises at import, there is no fallback implementation.  With TBQ4_DEBUG=1 in
+the environment the debug build (libtbq4_debug.so, ``build.py --debug``: the
+kernels' bounds checks switched on) is loaded instead.
 """
 import ctypes as C
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libtbq4.so")
+DEBUG = os.environ.get("TBQ4_DEBUG", "0") == "1"
+LIB_PATH = os.path.join(_HERE, "libtbq4_debug.so" if DEBUG else "libtbq4.so")
 
 # Every symbol include/tbq4.h declares, with (restype, argtypes).
 _p, _i, _i32, _i64, _u64, _f, _sz = (C.c_void_p, C.c_int, C.c_int32, C.c_int64,
@@ -50,7 +53,7 @@ SIGNATURES = {
 STATUS_NAMES = {0: "TBQ4_OK", 1: "TBQ4_ERR_NULL", 2: "TBQ4_ERR_ALIGN",
                 3: "TBQ4_ERR_SHAPE", 4: "TBQ4_ERR_CAPACITY",
                 5: "TBQ4_ERR_WORKSPACE", 6: "TBQ4_ERR_LAUNCH",
-                7: "TBQ4_ERR_DEVICE_TIMEOUT"}
+                7: "TBQ4_ERR_DEVICE_TIMEOUT", 8: "TBQ4_ERR_BOUNDS"}
 
 
 class Tbq4Error(RuntimeError):
@@ -64,8 +67,8 @@ def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"{LIB_PATH} is missing: build the CUDA library with "
-            "`python long_context_attention_tbq4_b200/build.py` (there is no "
-            "CPU fallback)")
+            "`python long_context_attention_tbq4_b200/build.py"
+            + (" --debug" if DEBUG else "") + "` (there is no CPU fallback)")
     L = C.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(L, name)

@@ -28,6 +28,34 @@ __device__ __forceinline__ void record_status(unsigned code) {
     atomicCAS(&g_status, 0u, code);
 }
 
+// Debug build (compiled with -DTBQ4_DEBUG into libtbq4_debug.so): every
+// global access whose address a kernel derives from lengths, positions, page
+// ids or the split plan is checked against the extent of its buffer.  A
+// failed check records status 8 (TBQ4_ERR_BOUNDS) and the access is skipped,
+// or, for a copy tracked by an mbarrier, redirected to offset 0 so that the
+// barrier still completes.  In the release build the checks are constant true.
+#ifdef TBQ4_DEBUG
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
+
+// [off, off + len) inside [0, extent)?  Always true in the release build.
+__device__ __forceinline__ bool in_extent(int64_t off, int64_t len, int64_t extent) {
+    if constexpr (kDebugBounds) {
+        if (off < 0 || len < 0 || off > extent - len) {
+            record_status(8u /* TBQ4_ERR_BOUNDS */);
+            return false;
+        }
+    }
+    return true;
+}
+
+// off if [off, off + len) is inside [0, extent), else 0 (debug build only).
+__device__ __forceinline__ int64_t checked_off(int64_t off, int64_t len, int64_t extent) {
+    return in_extent(off, len, extent) ? off : 0;
+}
+
 // Four sign bits of the +-1 diagonal for elements 4*lane .. 4*lane+3:
 // s_i = -1 where bit (i % 64) of word i / 64 is set.
 __device__ __forceinline__ uint32_t lane_sign_bits(uint64_t lo, uint64_t hi, int lane) {

@@ -52,6 +52,10 @@ struct AttnParams {
     int page_size;              // tokens per page, a multiple of 32
     int64_t n_pages;
     int tbq3;                   // 1: 3-bit caches [..][50] (decode only)
+    // Extents, for the debug build's bounds checks: bytes of each of the K
+    // and V caches (or pools), entries of part_ml (part_o holds 128 floats
+    // per entry), elements of out.
+    int64_t cache_bytes, part_rows, out_elems;
 };
 
 // Byte offset of token t of (sequence s, KV head g) in a paged pool.  An
@@ -150,6 +154,7 @@ __device__ __forceinline__ void store_row(const AttnParams &p, int s, int h, flo
     const uint32_t sbits = lane_sign_bits(p.sign_lo, p.sign_hi, lane);
     const float c = rot_c();
     const int64_t oi = ((int64_t)s * p.Hq + h) * kD + 4 * lane;
+    if (!in_extent(oi, 4, p.out_elems)) return;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         float x = v[k] * c;
@@ -184,8 +189,9 @@ decode_combine_kernel(const AttnParams p) {
     // The lengths are an input of the split kernel, not one of its results,
     // so they are read before the wait and only the partials' loads follow it.
     const int32_t len = seq_length(p, p.q_len > 1 ? s / p.q_len : s);
-    const int used = used_splits(p, len);
     const int64_t row0 = ((int64_t)s * p.Hq + h) * p.n_splits;
+    int used = used_splits(p, len);
+    if (!in_extent(row0, used, p.part_rows)) used = 0;
     // Launched as a programmatic dependent of the split kernel: wait for all
     // of its partials (a no-op under an ordinary launch).  Then the next
     // decode step's split kernel may start: its caches were complete before
@@ -269,8 +275,9 @@ combine_rows_kernel(const AttnParams p, int n_rows) {
     const int rowid = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
     if (rowid >= n_rows) return;
     const int s = rowid / p.Hq, h = rowid - (rowid / p.Hq) * p.Hq;
-    const int used = used_splits(p, seq_length(p, s));
     const int64_t row0 = ((int64_t)s * p.Hq + h) * p.n_splits;
+    int used = used_splits(p, seq_length(p, s));
+    if (!in_extent(row0, used, p.part_rows)) used = 0;
     float4 O;
     float M, L;
     merge_split_run(p, row0, used, 0, 1, lane, O, M, L);

@@ -320,8 +320,10 @@ decode_mq_kernel(const AttnParams p) {
             const int r0 = piece * kPieceRows;
             if (piece < kTile / kPieceRows && r0 < rows) {
                 const uint32_t nb = (uint32_t)(min(kPieceRows, rows - r0)) * kBlockBytes;
-                const uint8_t *src = (kv ? vb : kb) + (int64_t)(tj + r0) * kBlockBytes;
-                bulk_g2s(dst + kv * kRawBytes + r0 * kBlockBytes, src, nb, raw_full(st));
+                int64_t off = (kb - p.k) + (int64_t)(tj + r0) * kBlockBytes;
+                if constexpr (kDebugBounds) off = checked_off(off, nb, p.cache_bytes);
+                bulk_g2s(dst + kv * kRawBytes + r0 * kBlockBytes, (kv ? p.v : p.k) + off, nb,
+                         raw_full(st));
             }
         }
     } else if (warp == 1) {
@@ -664,9 +666,11 @@ decode_mq_kernel(const AttnParams p) {
                     const int64_t row =
                         (((int64_t)s * QL + i) * p.Hq + g * G + h) * p.n_splits + split;
                     // sum_t P'_t (2n - 15) = 2^11 (O''_hi + O''_lo)
-                    p.part_o[row * kD + t] =
-                        (__uint_as_float(ov[k]) + __uint_as_float(ovl[k])) * ips15;
-                    if (t == 0) p.part_ml[row] = make_float2(m[k], L);
+                    if (in_extent(row, 1, p.part_rows)) {
+                        p.part_o[row * kD + t] =
+                            (__uint_as_float(ov[k]) + __uint_as_float(ovl[k])) * ips15;
+                        if (t == 0) p.part_ml[row] = make_float2(m[k], L);
+                    }
                 }
             }
         } else {

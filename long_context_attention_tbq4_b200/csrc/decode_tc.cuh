@@ -238,6 +238,8 @@ decode_tc_kernel(const AttnParams p) {
         const uint32_t dst = smem_u32(ring) + w * kWarpRing + st * kStageBytes;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_expect_tx(bar, 2 * bytes);
+        if constexpr (kDebugBounds)
+            ofs = checked_off((kb - p.k) + ofs, bytes, p.cache_bytes) - (kb - p.k);
         bulk_g2s(dst, kb + ofs, bytes, bar);
         bulk_g2s(dst + kChunkBytes, vb + ofs, bytes, bar);
     };
@@ -442,6 +444,7 @@ decode_tc_kernel(const AttnParams p) {
                 gofs = paged_offset(p, page_id(p, s, len - 1), g, len - 1, &gbad);
             else
                 gofs = s * p.seq_stride + g * p.head_stride + (int64_t)(len - 1) * kBlockBytes;
+            if (!gbad && !in_extent(gofs, kBlockBytes, p.cache_bytes)) gbad = true;
             if (gbad && lane == 0) record_status(4u);
 #pragma unroll
             for (int kv = 0; kv < 2; ++kv) {
@@ -830,9 +833,11 @@ decode_tc_kernel(const AttnParams p) {
             for (int w = 0; w < kTcWarps; ++w)
                 O = fmaf(wt[w * kMaxGroup + h], src[w * 32 * kLaneStride], O);
             const int64_t row = ((int64_t)s * p.Hq + g * G + h) * p.n_splits + split;
-            // the block factor is S/15 (S/7 for 3 bits)
-            p.part_o[row * kD + d] = O * (kBits == 4 ? 1.0f / 15.0f : 1.0f / 7.0f);
-            if (d == 0) p.part_ml[row] = ml_h[h];
+            if (in_extent(row, 1, p.part_rows)) {
+                // the block factor is S/15 (S/7 for 3 bits)
+                p.part_o[row * kD + d] = O * (kBits == 4 ? 1.0f / 15.0f : 1.0f / 7.0f);
+                if (d == 0) p.part_ml[row] = ml_h[h];
+            }
         }
     }
 }

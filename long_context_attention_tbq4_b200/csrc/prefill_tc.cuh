@@ -151,6 +151,9 @@ struct PrefillParams {
     uint64_t sign_lo, sign_hi;
     float *part_o;              // [n_new][Hq][n_splits][128]
     float2 *part_ml;            // [n_new][Hq][n_splits]
+    // extents, for the debug build's bounds checks: bytes of each cache,
+    // entries of part_ml
+    int64_t cache_bytes, part_rows;
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -253,9 +256,10 @@ prefill_tc_kernel(const PrefillParams p) {
                 const uint32_t dst = sbase + kOffRaw + st * kRawStageBytes;
                 fence_proxy_async();
                 mbar_expect_tx(raw_full(st), 2 * bytes);
-                bulk_g2s(dst, p.k + head_off + t0 * kBlockBytes, bytes, raw_full(st));
-                bulk_g2s(dst + kRawBytes, p.v + head_off + t0 * kBlockBytes, bytes,
-                             raw_full(st));
+                int64_t off = head_off + t0 * kBlockBytes;
+                if constexpr (kDebugBounds) off = checked_off(off, bytes, p.cache_bytes);
+                bulk_g2s(dst, p.k + off, bytes, raw_full(st));
+                bulk_g2s(dst + kRawBytes, p.v + off, bytes, raw_full(st));
             }
         }
       } else if (warp == 1) {
@@ -559,9 +563,9 @@ prefill_tc_kernel(const PrefillParams p) {
         }
         // ---- partial (O unnormalised, m, l) for this split -----------------
         const int h = 2 * pair + a;
-        const bool write = active && (i0 + row) < p.n_new;
         const int64_t prow =
             (((int64_t)(i0 + row) * p.Hq + g * p.G + h) * p.n_splits + split);
+        const bool write = active && (i0 + row) < p.n_new && in_extent(prow, 1, p.part_rows);
         if (active && n_tiles > 0 && ok &&
             mbar_wait_bounded(o_done(a), (n_tiles - 1) & 1, kSpin)) {
             tc::fence_after_sync();

@@ -75,6 +75,7 @@ struct PageMap {
     const int32_t *table;
     int max_pages, page_size;
     int64_t n_pages;
+    int64_t cache_bytes;        // bytes of the destination cache or pool (debug bounds checks)
 };
 
 // The 3-bit variant (TBQ3): the same rotation and scale, 8 levels
@@ -183,7 +184,9 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
             uint32_t b, h, t0;
             group_of(gi, b, h, t0);
             const uint32_t t = min(t0 + lane, (uint32_t)n_new - 1);
-            const float *srow = src + (((int64_t)b * n_new + t) * Hkv + h) * kD;
+            int64_t ridx = ((int64_t)b * n_new + t) * Hkv + h;
+            if constexpr (kDebugBounds) ridx = checked_off(ridx, 1, (int64_t)B * n_new * Hkv);
+            const float *srow = src + ridx * kD;
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             bulk_g2s(smem_u32(ring + d * kQStageBytes + lane * kQRowStride), srow, 512,
                      bar0 + 8 * d);
@@ -217,6 +220,7 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
                 } else {
                     doff = (((int64_t)b * Hkv + h) * capacity + pos) * kBlk;
                 }
+                if (doff >= 0 && !in_extent(doff, kBlk, pm.cache_bytes)) doff = -1;
             }
             doffs[rho] = doff;
         }
@@ -427,6 +431,7 @@ quantize_warp_rows_kernel(const float *__restrict__ src, int B, int n_new, int H
             } else {
                 doff = (((int64_t)b * Hkv + h) * capacity + pos) * kBlockBytes;
             }
+            if (doff >= 0 && !in_extent(doff, kBlockBytes, pm.cache_bytes)) doff = -1;
         }
         if (doff < 0) {
             if (lane == 0) record_status(4u /* TBQ4_ERR_CAPACITY */);

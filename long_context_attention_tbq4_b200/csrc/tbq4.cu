@@ -126,6 +126,11 @@ tbq4_status run_attention(AttnParams p, void *workspace, size_t ws_bytes,
     p.n_splits = w.n_splits;
     p.part_o = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.part_o);
     p.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) + w.part_ml);
+    p.part_rows = (int64_t)qrows * p.Hq * w.n_splits;
+    p.out_elems = (int64_t)qrows * p.Hq * kD;
+    p.cache_bytes = p.block_table
+        ? p.n_pages * p.Hkv * p.page_size * (int64_t)(p.tbq3 ? kBlockBytes3 : kBlockBytes)
+        : (int64_t)p.nseq * p.seq_stride;
     static bool attr_set[64] = {}, attr_paged[64] = {}, attr_mq[64] = {};  // once per device
     static bool attr_3[64] = {};
     const bool mq = p.q_len > 1, paged = p.block_table != nullptr;
@@ -238,7 +243,7 @@ namespace {
 constexpr int64_t kSmallAppendRows = 16384;
 
 tbq4_status quantize_impl(const float *src, int B, int n_new, int Hkv, const int32_t *start_pos,
-                          int64_t capacity, uint64_t sign_seed, const PageMap &pm,
+                          int64_t capacity, uint64_t sign_seed, const PageMap &map,
                           uint8_t *cache, void *stream, int bits = 4) {
     if (!src || !start_pos || !cache) return TBQ4_ERR_NULL;
     if (!aligned(src, 16) || !aligned(cache, 16) || !aligned(start_pos, 4))
@@ -248,6 +253,10 @@ tbq4_status quantize_impl(const float *src, int B, int n_new, int Hkv, const int
     if (n_new == 0) return TBQ4_OK;
     const int64_t rows = (int64_t)B * n_new * Hkv;
     if (rows > 0x7FFFFFFFLL) return TBQ4_ERR_SHAPE;      // rows are indexed in 32 bits
+    PageMap pm = map;
+    const int64_t blk = bits == 3 ? kBlockBytes3 : kBlockBytes;
+    pm.cache_bytes = pm.table ? pm.n_pages * Hkv * pm.page_size * blk
+                              : (int64_t)B * Hkv * capacity * blk;
     if (bits == 4 && rows < kSmallAppendRows) {
         // few rows: one warp per row over every SM
         uint64_t lo, hi;
@@ -318,7 +327,7 @@ tbq4_status tbq4_quantize_append_paged(const float *src, int B, int n_new, int H
     if (page_size < 32 || page_size % 32 != 0 || max_pages <= 0 || n_pages <= 0 ||
         n_pages > 0x7FFFFFFFLL)
         return TBQ4_ERR_SHAPE;
-    const PageMap pm = {block_table, max_pages, page_size, n_pages};
+    const PageMap pm = {block_table, max_pages, page_size, n_pages, 0};
     return quantize_impl(src, B, n_new, Hkv, start_pos, (int64_t)max_pages * page_size,
                          sign_seed, pm, pool, stream);
 }
@@ -595,6 +604,8 @@ tbq4_status tbq4_attn_prefill_chunk(const uint16_t *q, int n_new, int64_t n_cach
     pp.sign_hi = hi;
     pp.part_o = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.part_o);
     pp.part_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) + w.part_ml);
+    pp.cache_bytes = (int64_t)Hkv * pp.head_stride;
+    pp.part_rows = (int64_t)n_new * Hq * w.n_splits;
     if (g_ev_before) cudaEventRecord(g_ev_before, st);
     pre::prefill_tc_kernel<<<dim3(w.n_splits, w.mpairs), pre::kThreads, pre::kSmemBytes, st>>>(pp);
     if (g_ev_after) cudaEventRecord(g_ev_after, st);
@@ -617,6 +628,8 @@ tbq4_status tbq4_attn_prefill_chunk(const uint16_t *q, int n_new, int64_t n_cach
     c.part_ml = pp.part_ml;
     c.out = out;
     c.out_bf16 = 1;
+    c.part_rows = pp.part_rows;
+    c.out_elems = (int64_t)n_new * Hq * kD;
     // one warp per (position, head) row, a programmatic dependent launch
     const int n_rows = n_new * Hq;
     cudaLaunchConfig_t cfg = {};
@@ -667,6 +680,7 @@ const char *tbq4_status_string(tbq4_status s) {
         case TBQ4_ERR_WORKSPACE: return "workspace smaller than required";
         case TBQ4_ERR_LAUNCH: return "a CUDA launch or query failed";
         case TBQ4_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel gave up";
+        case TBQ4_ERR_BOUNDS: return "a bounds check of the debug build failed";
     }
     return "unknown status";
 }

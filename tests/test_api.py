@@ -42,6 +42,25 @@ def test_library_exports_every_declared_symbol(T):
         assert getattr(_lib.lib, n) is not None
 
 
+def test_debug_library_exports_every_declared_symbol():
+    # built here if missing (a few seconds of nvcc); no compute call
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "tbq4_build", os.path.join(ROOT, "long_context_attention_tbq4_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
+    path = build.build(debug=True)
+    assert path.endswith("libtbq4_debug.so")
+    out = subprocess.run(["nm", "-D", "--defined-only", path], check=True,
+                         capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (tbq[34]_\w+)", out))
+    for n in declared_symbols():
+        assert n in exported, n
+    lib = C.CDLL(path)
+    lib.tbq4_status_string.restype = C.c_char_p
+    assert b"debug" in lib.tbq4_status_string(8)
+
+
 def test_block_and_cache_bytes(T):
     assert T.tbq4_block_bytes() == 66
     assert T.tbq4_cache_bytes(1, 4, 262144) == 262144 * 4 * 66
@@ -141,7 +160,7 @@ def test_selftest_rejects_bad_poll_counts(T):
 
 def test_status_strings(T):
     from long_context_attention_tbq4_b200._lib import lib as L
-    for code in range(8):
+    for code in range(9):
         assert len(L.tbq4_status_string(code)) > 0
 
 
