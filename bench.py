@@ -186,7 +186,10 @@ L2_NOTE = ("inputs larger than L2: the steps cycle through 4 layers' caches (4 x
            "flushes L2 (512 MiB written, then read back) before every step instead")
 LAUNCH_NOTE = ("the K timed steps are one CUDA graph replayed once between two events, each "
                "step a split kernel + combine, the split kernel a programmatic dependent of "
-               "the combine before it; e2e runs the same steps eagerly with host copies")
+               "the combine before it; e2e: each step also copies its inputs in (one packed "
+               "copy from its own pinned buffer) and its output out (to its own pinned "
+               "buffer), the K steps captured as one graph and replayed once (the same steps "
+               "issued eagerly from Python: e2e.ms_per_step_eager)")
 
 
 def decode_workload():
@@ -336,41 +339,62 @@ def bench_decode(T, torch, case, N, step_bytes, kernel_bytes, steps, warmup, flu
     iso_ms = [e0.elapsed_time(e1) for e0, e1, _, _ in ev]
     del g_step
 
-    # ---- end to end, back to back: every step copies its q and new rows
-    # from pinned host memory and its output back, through the public API
-    q_h = torch.from_numpy(case.q).pin_memory()
-    kn_h = torch.from_numpy(np.ascontiguousarray(K[N - 1:N])[None]).pin_memory()
-    vn_h = torch.from_numpy(np.ascontiguousarray(V[N - 1:N])[None]).pin_memory()
+    # ---- end to end, back to back: every step copies its q and new rows in
+    # from pinned host memory (one packed copy, its own host buffer per step)
+    # and its output back out to its own pinned buffer, through the public
+    # API.  Timed two ways: the K steps captured as one CUDA graph (copy
+    # nodes, kernels, copy nodes; as a serving loop captures its decode
+    # steps) and replayed once between two events (the reported value), and
+    # the same steps issued eagerly from Python.
+    nq, nk = case.Hq * D, case.Hkv * D
+    n_e2e = max(steps, warmup)
+    packed = np.concatenate([case.q.reshape(-1), np.ascontiguousarray(K[N - 1]).reshape(-1),
+                             np.ascontiguousarray(V[N - 1]).reshape(-1)]).astype(np.float32)
+    in_h = [torch.from_numpy(packed.copy()).pin_memory() for _ in range(n_e2e)]
     out_h = [torch.empty((1, case.Hq, D), dtype=torch.float16).pin_memory()
-             for _ in range(steps)]
-    q_d, kn_d, vn_d = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
+             for _ in range(n_e2e)]
+    in_d = torch.empty_like(in_h[0], device=dev)
+    q_v = in_d[:nq].view(1, case.Hq, D)
+    kn_v = in_d[nq:nq + nk].view(1, case.Hkv, D)
+    vn_v = in_d[nq + nk:].view(1, case.Hkv, D)
 
     def e2e_step(i):
-        q_d.copy_(q_h, non_blocking=True)
-        kn_d.copy_(kn_h, non_blocking=True)
-        vn_d.copy_(vn_h, non_blocking=True)
-        step(i % N_LAYERS, q_d, kn_d, vn_d, out)
+        in_d.copy_(in_h[i], non_blocking=True)
+        step(i % N_LAYERS, q_v, kn_v, vn_v, out)
         out_h[i].copy_(out, non_blocking=True)
+
+    def timed(fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        return e0.elapsed_time(e1)
 
     for i in range(warmup):
         e2e_step(i)
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
+    e2e_eager_total = timed(lambda: [e2e_step(i) for i in range(steps)])
+    g_e2e = capture_graph(torch, lambda: [e2e_step(i) for i in range(steps)])
+    g_e2e.replay()                      # untimed: the graph's first replay
     torch.cuda.synchronize()
-    e0.record()
-    for i in range(steps):
-        e2e_step(i)
-    e1.record()
-    torch.cuda.synchronize()
-    barrier()
-    e2e_total = e0.elapsed_time(e1)
+    for o in out_h[:steps]:
+        o.zero_()
+    e2e_total = timed(g_e2e.replay)
+    del g_e2e
     assert T.tbq4_get_device_status() == 0
-    h2d = q_h.numel() * 4 + kn_h.numel() * 4 + vn_h.numel() * 4
-    d2h = out_h[0].numel() * 2
+    for o in out_h[:steps]:             # every step's output came back to the host
+        assert torch.equal(o, out_h[steps - 1]) and bool(o.abs().sum() > 0)
+    h2d_bytes = in_h[0].numel() * 4
+    d2h_bytes = out_h[0].numel() * 2
     return {"b2b_ms": b2b_ms, "step_ms": [b2b_ms / steps] * steps, "iso_ms": iso_ms,
             "eager_ms": eager_ms, "kern_ms": kern_ms, "e2e_ms": [e2e_total / steps] * steps,
-            "h2d": h2d, "d2h": d2h, "launches_per_step": 2, "out": out.float().cpu().numpy()}
+            "e2e_eager_ms": e2e_eager_total / steps,
+            "h2d": h2d_bytes, "d2h": d2h_bytes, "launches_per_step": 2,
+            "out": out.float().cpu().numpy()}
 
 
 def bench_prefill(T, torch, steps, warmup, flush):
@@ -592,15 +616,16 @@ def replica_totals(torch, dec, steps, world, step_bytes):
     """Whole-job figures of `world` independent replicas, each rank having
     timed `steps` decode steps (dec: per-step device times in ms).  Every time
     is the max over ranks; the value counts the bytes of all ranks.  Every
-    rank makes the same three reductions in the same order."""
+    rank makes the same four reductions in the same order."""
     total_ms = max_over_ranks(torch, float(np.sum(dec["step_ms"])))
     ms_per_step = total_ms / steps
     e2e_ms = max_over_ranks(torch, float(np.mean(dec["e2e_ms"])))
     eager_ms = max_over_ranks(torch, float(np.mean(dec["eager_ms"])))
+    e2e_eager_ms = max_over_ranks(torch, float(dec.get("e2e_eager_ms", 0.0)))
     return {"ms_per_step": ms_per_step,
             "value": world * step_bytes / (ms_per_step * 1e-3) / 1e9,
             "e2e_ms": e2e_ms, "e2e_value": world * step_bytes / (e2e_ms * 1e-3) / 1e9,
-            "eager_ms": eager_ms}
+            "eager_ms": eager_ms, "e2e_eager_ms": e2e_eager_ms}
 
 
 # -------------------------------------------------------------------- main
@@ -706,7 +731,11 @@ def main():
                      "l2": "flushed before every step"},
         "e2e": {"value": tot["e2e_value"], "unit": "GB/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": dec["h2d"],
-                "d2h_bytes_per_step": dec["d2h"]},
+                "d2h_bytes_per_step": dec["d2h"],
+                "timing": "the K steps with their copies captured as one CUDA graph, replayed "
+                          "once between two events",
+                "ms_per_step_eager": tot["e2e_eager_ms"],
+                "value_eager": world * step_bytes / (tot["e2e_eager_ms"] * 1e-3) / 1e9},
         "gpu_launches": dec["launches_per_step"] * args.steps,
         "clocks": clocks,
     }
