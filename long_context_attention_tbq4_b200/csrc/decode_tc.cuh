@@ -142,16 +142,16 @@ __device__ __forceinline__ void split3(int x, int8_t &c0, int8_t &c1, int8_t &c2
     c2 = (int8_t)((x1 - b1) >> 8);
 }
 
-// TBQ3 (3-bit) blocks hold index i where TBQ4 holds nibble n: with n = i + 4
-// the level 2n - 15 equals the 3-bit level 2i - 7, and only the block
-// factor changes (S/7 instead of S/15).  So the 3-bit kernel expands each
-// group of eight 3-bit indices (a 24-bit word) into eight nibbles n = i + 4
-// in a register and runs the 4-bit arithmetic unchanged.
-__device__ __forceinline__ uint32_t tbq3_nibbles(uint32_t g) {
-    uint32_t t = (g & 0x00000FFFu) | ((g & 0x00FFF000u) << 4);    // 4 fields per half
-    t = (t & 0x003F003Fu) | ((t & 0x0FC00FC0u) << 2);             // 2 fields per byte
-    t = (t & 0x07070707u) | ((t & 0x38383838u) << 1);             // one per nibble
-    return t + 0x44444444u;                                       // i + 4, no carries
+// TBQ3 (3-bit) K operand.  In a group of eight 3-bit indices (a 24-bit word,
+// index 8g + k at bits 3k) the indices of dimensions 2j and 2j + 1 already
+// form one 6-bit field i_even + 8 i_odd at bits 6j.  Spreading the four
+// fields to four bytes gives the same operand shape as the 4-bit raw bytes
+// (lo + 16 hi), with 8 in place of 16: the raw byte weighs q_odd, its low 3
+// bits (i_even) weigh 8 q_even - q_odd, and the products sum to
+// 8 sum_d i_d q_d.
+__device__ __forceinline__ uint32_t tbq3_pairs(uint32_t g) {
+    const uint32_t t = (g & 0x00000FFFu) | ((g & 0x00FFF000u) << 4);    // 2 fields per half
+    return (t & 0x003F003Fu) | ((t & 0x0FC00FC0u) << 2);                // 1 field per byte
 }
 
 // 3-bit V levels straight from the packed indices, with no expansion to
@@ -306,8 +306,9 @@ decode_tc_kernel(const AttnParams p) {
     // ---- q: rotate, normalise by a power of two, 18-bit integer ----------
     // q_int = rint(q_rot * 2^(18-e)) with 2^e > max|q_rot|, so |q_int| <= 2^18.
     // Per dimension pair j = (2j, 2j+1): u_j = q_int[2j+1] (weight of the raw
-    // byte) and w_j = 16 q_int[2j] - q_int[2j+1] (weight of its low nibble),
-    // each split into three signed bytes, pieces [3][head][pair].
+    // byte) and w_j = 16 q_int[2j] - q_int[2j+1] (weight of its low nibble;
+    // 8 q_int[2j] - q_int[2j+1] for the 3-bit pair bytes), each split into
+    // three signed bytes, pieces [3][head][pair].
     int8_t *qu8 = reinterpret_cast<int8_t *>(smem + kRingBytes + kBarBytes);   // [3][8][64]
     int8_t *qw8 = qu8 + 3 * kMaxGroup * 64;                              // [3][8][64]
     float *qpar = reinterpret_cast<float *>(qw8 + 3 * kMaxGroup * 64);   // [8][2]
@@ -327,7 +328,7 @@ decode_tc_kernel(const AttnParams p) {
 #pragma unroll
         for (int j = 0; j < 2; ++j) {                 // pairs 2 lane + j
             const int pair = 2 * lane + j;
-            const int u = qi[2 * j + 1], w = 16 * qi[2 * j] - qi[2 * j + 1];
+            const int u = qi[2 * j + 1], w = (kBits == 4 ? 16 : 8) * qi[2 * j] - qi[2 * j + 1];
             split3(u, qu8[(0 * kMaxGroup + warp) * 64 + pair], qu8[(1 * kMaxGroup + warp) * 64 + pair],
                    qu8[(2 * kMaxGroup + warp) * 64 + pair]);
             split3(w, qw8[(0 * kMaxGroup + warp) * 64 + pair], qw8[(1 * kMaxGroup + warp) * 64 + pair],
@@ -335,12 +336,13 @@ decode_tc_kernel(const AttnParams p) {
         }
         qsum = __reduce_add_sync(kFull, qsum);
         if (lane == 0) {
-            // log2 logit = (2 S - 15 sum q) * S_k * scale * log2(e) / 15 * 2^(e-18),
-            // and the integer MMAs return 16 S
+            // log2 logit = (2 S - 15 sum q) * S_k * scale * log2(e) / 15 * 2^(e-18)
+            // with S = sum n q and the integer MMAs returning 16 S; for 3 bits
+            // (2 S - 7 sum q) * S_k ... / 7 with S = sum i q, the MMAs returning 8 S
             const float fh = p.scale_log2 * (kBits == 4 ? 1.0f / 15.0f : 1.0f / 7.0f) *
                              ldexpf(1.0f, e - kQBits);
-            qpar[2 * warp + 0] = 0.125f * fh;
-            qpar[2 * warp + 1] = -15.0f * (float)qsum * fh;
+            qpar[2 * warp + 0] = (kBits == 4 ? 0.125f : 0.25f) * fh;
+            qpar[2 * warp + 1] = (kBits == 4 ? -15.0f : -7.0f) * (float)qsum * fh;
         }
     } else if (warp < kMaxGroup) {
         for (int k = lane; k < 3 * 64; k += 32) {
@@ -492,16 +494,17 @@ decode_tc_kernel(const AttnParams p) {
                     const uint32_t W0 = __funnelshift_r(wr[h][0], wr[h][1], ksh);
                     const uint32_t W1 = __funnelshift_r(wr[h][1], wr[h][2], ksh);
                     const uint32_t W2 = __funnelshift_r(wr[h][2], wr[h][3], ksh);
-                    xr[h][0] = tbq3_nibbles(W0 & 0x00FFFFFFu);
-                    xr[h][1] = tbq3_nibbles(__funnelshift_r(W0, W1, 24) & 0x00FFFFFFu);
-                    xr[h][2] = tbq3_nibbles(__funnelshift_r(W1, W2, 16) & 0x00FFFFFFu);
-                    xr[h][3] = tbq3_nibbles(W2 >> 8);
+                    xr[h][0] = tbq3_pairs(W0 & 0x00FFFFFFu);
+                    xr[h][1] = tbq3_pairs(__funnelshift_r(W0, W1, 24) & 0x00FFFFFFu);
+                    xr[h][2] = tbq3_pairs(__funnelshift_r(W1, W2, 16) & 0x00FFFFFFu);
+                    xr[h][3] = tbq3_pairs(W2 >> 8);
                 }
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const uint32_t x0 = xk0[i], x1 = xk1[i];                       // raw bytes
-                const uint32_t lo0 = x0 & 0x0F0F0F0Fu, lo1 = x1 & 0x0F0F0F0Fu;
+                constexpr uint32_t kLoMask = kBits == 4 ? 0x0F0F0F0Fu : 0x07070707u;
+                const uint32_t lo0 = x0 & kLoMask, lo1 = x1 & kLoMask;
 #pragma unroll
                 for (int pc = 0; pc < 3; ++pc) {
                     if (i == 0)
@@ -510,7 +513,7 @@ decode_tc_kernel(const AttnParams p) {
                         imma16832(acc[pc], x0, x1, lo0, lo1, qb[i][pc][0], qb[i][pc][1]);
                 }
             }
-            // 16 sum_d n_d q_int_d = 65536 acc2 + 256 acc1 + acc0
+            // 16 sum_d n_d q_int_d (3 bits: 8 sum_d i_d q_int_d) = 65536 acc2 + 256 acc1 + acc0
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 sc[tile][e] = fmaf((float)acc[2][e], 65536.0f, (float)(acc[1][e] * 256 + acc[0][e]));
