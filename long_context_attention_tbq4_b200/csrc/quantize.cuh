@@ -62,10 +62,12 @@ __device__ __forceinline__ uint32_t encode_row(float v[4], uint32_t sbits, int l
 // head), so a group's 8 blocks are contiguous in the cache.  Lane l
 // takes row l % 8 of its warp's group and quarter l / 8 of that row.  One
 // CTA of 16 warps per SM; each warp streams its groups through a ring of
-// kQDepth shared-memory stages, one 512-byte cp.async.bulk per row (rows 528
-// bytes apart, so the eight lanes of a 16-byte read phase hit eight
-// different bank groups), and sends the copies of a later group into a stage
-// as soon as the rows are in registers.  The blocks go out from a per-warp
+// kQDepth shared-memory stages (rows 528 bytes apart, so the eight lanes of a
+// 16-byte read phase hit eight different bank groups), each lane copying 16
+// bytes of every row with cp.async (one commit group per stage), and sends
+// the copies of a later group into a stage as soon as the rows are in
+// registers.  (One cp.async.bulk per row took longer: its operands go through
+// uniform registers, one lane at a time.)  The blocks go out from a per-warp
 // staging area, as one bulk shared -> global copy when the group's 8 blocks
 // are consecutive and 16-byte aligned, else as 16-bit pieces.
 // Paged destination: row (b, pos) goes to page table[b][pos / page_size],
@@ -92,7 +94,7 @@ constexpr int kQStageBytes = kQRows * kQRowStride;
 constexpr int kQOutBytes = kQRows * kBlockBytes + 16 + kQRows * 8;   // blocks, pad, destinations
 constexpr int kQThreads = kQWarps * 32;
 constexpr int kQRingBytes = kQWarps * kQDepth * kQStageBytes;
-constexpr int kQSmemBytes = kQRingBytes + kQWarps * kQOutBytes + kD * 4 + kQWarps * kQDepth * 8;
+constexpr int kQSmemBytes = kQRingBytes + kQWarps * kQOutBytes + kD * 4;
 static_assert(kQSmemBytes <= 227 * 1024, "shared memory per CTA");
 static_assert(kQStageBytes % 16 == 0 && kQRowStride % 16 == 0 && kQOutBytes % 16 == 0,
               "bulk copies and staged rows stay 16-byte aligned");
@@ -164,41 +166,39 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
     uint16_t *stage = reinterpret_cast<uint16_t *>(wout);                     // [8][kPieces]
     int64_t *doffs = reinterpret_cast<int64_t *>(wout + kQRows * kBlockBytes + 16);   // [8]
     float *sgn = reinterpret_cast<float *>(qsm + kQRingBytes + kQWarps * kQOutBytes);  // [128]
-    const uint32_t bar0 = smem_u32(sgn + kD) + warp * kQDepth * 8;
     if (threadIdx.x < kD) {
         const int i = threadIdx.x;
         const uint64_t w = i < 64 ? sign_lo : sign_hi;
         sgn[i] = ((w >> (i & 63)) & 1u) ? -1.0f : 1.0f;
     }
-    if (lane == 0) {
-        for (int d = 0; d < kQDepth; ++d) mbar_init(bar0 + 8 * d, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
     __syncthreads();
-    // the 8 rows of group gi into stage d, one bulk copy per lane 0..7 (rows
-    // past the end repeat the last row; nothing of theirs is stored)
+    // the 8 rows of group gi into stage d, lane l copying bytes 16 l .. 16 l
+    // + 15 of each (rows past the end repeat the last row; nothing of theirs
+    // is stored).  Every call commits one cp.async group, empty past the last
+    // group, so that waiting for all but the newest kQDepth - 1 groups always
+    // waits for the stage about to be read.
     auto load_group = [&](uint32_t gi, int d) {
-        if (lane == 0) mbar_expect_tx(bar0 + 8 * d, kQRows * 512);
-        __syncwarp();
-        if (lane < kQRows) {
+        if (gi < groups) {
             uint32_t b, h, t0;
             group_of(gi, b, h, t0);
-            const uint32_t t = min(t0 + lane, (uint32_t)n_new - 1);
-            int64_t ridx = ((int64_t)b * n_new + t) * Hkv + h;
-            if constexpr (kDebugBounds) ridx = checked_off(ridx, 1, (int64_t)B * n_new * Hkv);
-            const float *srow = src + ridx * kD;
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            bulk_g2s(smem_u32(ring + d * kQStageBytes + lane * kQRowStride), srow, 512,
-                     bar0 + 8 * d);
+            const uint32_t dst = smem_u32(ring + d * kQStageBytes) + 16 * lane;
+#pragma unroll
+            for (int r = 0; r < kQRows; ++r) {
+                const uint32_t t = min(t0 + r, (uint32_t)n_new - 1);
+                int64_t ridx = ((int64_t)b * n_new + t) * Hkv + h;
+                if constexpr (kDebugBounds) ridx = checked_off(ridx, 1, (int64_t)B * n_new * Hkv);
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                             ::"r"(dst + r * kQRowStride), "l"(src + ridx * kD + 4 * lane)
+                             : "memory");
+            }
         }
+        asm volatile("cp.async.commit_group;" ::: "memory");     // one group per slot, maybe empty
     };
     const uint32_t gstride = kQWarps * gridDim.x;
     uint32_t gi = blockIdx.x + warp * gridDim.x;
 #pragma unroll
-    for (int d = 0; d < kQDepth; ++d)
-        if (gi + d * gstride < groups) load_group(gi + d * gstride, d);
+    for (int d = 0; d < kQDepth; ++d) load_group(gi + d * gstride, d);
     const float neg = (qq & 1) ? -1.0f : 1.0f, neg2 = (qq & 2) ? -1.0f : 1.0f;
-    bool aborted = false;
     uint32_t it = 0;
     for (; gi < groups; ++it, gi += gstride) {
         const int d = (int)(it % kQDepth);
@@ -224,11 +224,8 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
             }
             doffs[rho] = doff;
         }
-        if (!mbar_wait_bounded(bar0 + 8 * d, (it / kQDepth) & 1u)) {
-            if (lane == 0) record_status(7u /* TBQ4_ERR_DEVICE_TIMEOUT */);
-            aborted = true;
-            break;
-        }
+        asm volatile("cp.async.wait_group %0;" ::"n"(kQDepth - 1) : "memory");
+        __syncwarp();
         float v[32];
         {
             const float4 *row = reinterpret_cast<const float4 *>(ring + d * kQStageBytes +
@@ -243,7 +240,7 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
             }
         }
         __syncwarp();
-        if (gi + kQDepth * gstride < groups) load_group(gi + kQDepth * gstride, d);
+        load_group(gi + kQDepth * gstride, d);
         // stride 1 with the signs folded in
         {
             const float4 *s4 = reinterpret_cast<const float4 *>(sgn + 32 * qq);
@@ -379,20 +376,9 @@ quantize_rows_kernel(const float *__restrict__ src, int B, int n_new, int Hkv,
             __syncwarp();
         }
     }
-    // After a give-up, the copies this warp still has queued (the stage it
-    // gave up on and the groups issued ahead of it) must land before the
-    // warp leaves: a CTA must not exit with bulk copies writing its shared
-    // memory.  Each gets one more bounded wait.
-    if (aborted) {
-#pragma unroll
-        for (int k = 0; k < kQDepth; ++k) {
-            if (gi + (uint32_t)k * gstride >= groups) break;
-            const uint32_t ik = it + (uint32_t)k;
-            if (!mbar_wait_bounded(bar0 + 8 * (ik % kQDepth), (ik / kQDepth) & 1u) && lane == 0)
-                record_status(7u);
-        }
-    }
     // the last bulk store completes before the CTA's shared memory goes away
+    // (every copy into shared memory was waited for in its iteration; the
+    // groups committed past the last one are empty)
     if (lane == 0) bulk_s2g_wait_all();
 }
 
