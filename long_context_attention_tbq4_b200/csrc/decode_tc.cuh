@@ -22,8 +22,8 @@
 // output errors of a few 1e-3 where one token dominates; 18 bits keep the
 // logit error below 1e-3 of a log2 unit even in the worst case.)
 // V operand: pairs of tokens are interleaved with PRMT so that one register
-// holds the same dimension of two tokens; the levels enter as (n - 8) 2^-10
-// and enter as (2n - 15) 2^-11 (see lvl_lo).  P' = p * S_v * ps (S_v the
+// holds the same dimension of two tokens; the levels enter as (2n - 15) 2^-11,
+// exactly (see lvl_lo).  P' = p * S_v * ps (S_v the
 // block scale of V, ps a per-warp power of two that keeps P' a normal fp16)
 // enters as two fp16 terms hi + lo, so O = sum_t p_t S_v,t (2n-15) / 15 once
 // 1 / ps is applied.
