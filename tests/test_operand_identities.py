@@ -14,6 +14,9 @@ against the plain definition, on every value it can take or on random data:
   multiply-add give the level (2n - 15) 2^-11 with no rounding.
 - 3-bit V: three byte permutations of two tokens' groups put every field
   inside an fp16 mantissa; the same one-FMA step gives (2i - 7) 2^-11.
+- Quantiser: x / S by RN(1/S), RN(x r), the exact residual and one FMA is
+  the correctly rounded quotient for every normal fp16 scale; adding
+  1.5 2^23 rounds u to the nearest integer, ties to even.
 
 The kernels' constants are restated here; the tests need no GPU and do not
 use the oracle.
@@ -143,3 +146,45 @@ def test_v3_level_from_packed_fields_is_exact():
             lo, hi = word & 0xFFFF, word >> 16
             assert _hfma(lo, mul, 0x9B00) == (2 * ia[f] - 7) * 2.0**-11
             assert _hfma(hi, mul, 0x9B00) == (2 * ib[f] - 7) * 2.0**-11
+
+
+def _fma32(a, b, c):
+    """float32 fused multiply-add, emulated: a*b is exact in float64 (two
+    24-bit significands); the sum is rounded to float64 and then to float32,
+    which differs from one rounding only when the float64 sum lands exactly
+    on a float32 rounding midpoint (the residual step below, x - q0 S, is
+    exact in float64, so only the last step could be affected, and a
+    difference would fail the comparison rather than hide one)."""
+    return (a.astype(np.float64) * b.astype(np.float64) + c.astype(np.float64)).astype(np.float32)
+
+
+def test_quantizer_division_is_the_correctly_rounded_quotient():
+    # every positive normal fp16 scale, against values inside [-S, S] (the
+    # encoder clamps to that range where the scale is not within 2^-11 of max|x|)
+    s_bits = np.arange(0x0400, 0x7C00, dtype=np.uint16)
+    S = s_bits.view(np.float16).astype(np.float32)
+    S = np.repeat(S, 64)
+    x = (RNG.uniform(-1.0, 1.0, S.size).astype(np.float32) * S).astype(np.float32)
+    x[::17] = S[::17]
+    x[1::17] = -S[1::17]
+    r = (np.float32(1.0) / S).astype(np.float32)            # RN(1/S)
+    q0 = (x * r).astype(np.float32)                         # RN(x r)
+    e = _fma32(-q0, S, x)                                   # x - q0 S, exact
+    q = _fma32(e, r, q0)                                    # RN(q0 + e r)
+    want = (x / S).astype(np.float32)                       # IEEE x / S
+    # a subnormal quotient cannot change an index (|x/S| << 1/15 there)
+    normal = np.abs(want) >= np.float32(2.0**-126)
+    assert np.array_equal(q[normal], want[normal])
+
+
+def test_rint_by_adding_1_5_times_2_23_is_round_half_even():
+    for L in (7.5, 3.5):                                     # 4-bit and 3-bit codebooks
+        top = 2 * L
+        u = np.concatenate([np.linspace(-0.004, top + 0.004, 200001),
+                            np.arange(0, int(top) + 1) + 0.5,  # exact ties
+                            np.arange(0, int(top) + 1) - 0.5]).astype(np.float32)
+        u = u[(u >= -0.004) & (u <= top + 0.004)]
+        got = ((u + np.float32(12582912.0)).astype(np.float32).view(np.uint32) &
+               np.uint32(0xF if L == 7.5 else 0x7))
+        want = np.rint(u.astype(np.float64)).astype(np.int64)   # numpy rint: half to even
+        assert np.array_equal(got.astype(np.int64), np.clip(want, 0, int(top)))
