@@ -17,6 +17,8 @@
 #include <cmath>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 namespace {
 
 using namespace tbq4;
@@ -27,6 +29,17 @@ constexpr size_t kWsAlign = 256;
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// An NVTX range around an entry point's launches, named after the entry
+// point, so timeline and kernel profilers can select one call's kernels
+// (ncu --nvtx --nvtx-include).  Header-only NVTX: with no tool attached a
+// push and a pop cost a few nanoseconds of host time.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 // SplitMix64 (Steele, Lea & Flood 2014): the two words whose bits are the
 // +-1 diagonal (bit set -> -1).
@@ -118,6 +131,10 @@ tbq4_status launch_status() {
 
 tbq4_status run_attention(AttnParams p, void *workspace, size_t ws_bytes,
                           cudaStream_t st) {
+    const NvtxRange range(p.q_len > 1 ? "tbq4_attn_decode_mq"
+                          : p.block_table ? "tbq4_attn_decode_paged"
+                          : p.tbq3 ? "tbq3_attn_decode"
+                          : p.k_new ? "tbq4_attn_decode_append" : "tbq4_attn_decode");
     if (p.split_tokens <= 0 || p.split_tokens % 32 != 0) return TBQ4_ERR_SHAPE;
     const int qrows = p.nseq * (p.q_len > 1 ? p.q_len : 1);    // combine rows per head
     const WsLayout w = attn_ws_layout(qrows, p.Hq, p.max_len, p.split_tokens);
@@ -245,6 +262,8 @@ constexpr int64_t kSmallAppendRows = 16384;
 tbq4_status quantize_impl(const float *src, int B, int n_new, int Hkv, const int32_t *start_pos,
                           int64_t capacity, uint64_t sign_seed, const PageMap &map,
                           uint8_t *cache, void *stream, int bits = 4) {
+    const NvtxRange range(bits == 3 ? "tbq3_quantize_append"
+                          : map.table ? "tbq4_quantize_append_paged" : "tbq4_quantize_append");
     if (!src || !start_pos || !cache) return TBQ4_ERR_NULL;
     if (!aligned(src, 16) || !aligned(cache, 16) || !aligned(start_pos, 4))
         return TBQ4_ERR_ALIGN;
@@ -558,6 +577,7 @@ tbq4_status tbq4_attn_prefill_chunk(const uint16_t *q, int n_new, int64_t n_cach
                                     float softmax_scale, uint64_t sign_seed,
                                     void *workspace, size_t ws_bytes, uint16_t *out,
                                     void *stream) {
+    const NvtxRange range("tbq4_attn_prefill_chunk");
     if (!q || !k_cache || !v_cache || !workspace || !out) return TBQ4_ERR_NULL;
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
         !aligned(workspace, kWsAlign) || !aligned(out, 2))
