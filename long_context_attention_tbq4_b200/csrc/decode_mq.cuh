@@ -181,8 +181,8 @@ decode_mq_kernel(const AttnParams p) {
     const int32_t t0 = split * p.split_tokens;
     const int32_t t1 = min(len, t0 + p.split_tokens);
     const int n_tiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
+    // this (sequence, KV head)'s cache rows start kb - p.k bytes into both caches
     const uint8_t *kb = p.k + s * p.seq_stride + g * p.head_stride;
-    const uint8_t *vb = p.v + s * p.seq_stride + g * p.head_stride;
 
     // barriers
     const uint32_t bar0 = sbase + kOffBar;
